@@ -1,0 +1,341 @@
+// mxq_oracle.cpp -- plain, slow, CPU reference of the MXFP4 quantized linear layer.
+//
+// TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or calls
+// this file; only the test suite, the package's smoke check and the CPU-baseline
+// leg of the benchmark do.  It shares no code, header, table or constant with
+// the CUDA library: every value below is derived here from the definitions.
+//
+// What it computes, and where each step comes from:
+//
+//  * MXFP4 block format -- 32 consecutive elements along K share one E8M0
+//    (power-of-two, no mantissa) scale; elements are 4-bit E2M1.
+//      [MXAttention: Data-Free Optimal Scaling and Pre-Normalization Quantization
+//       for MXFP4 Attention -- "What it actually does", Universal Optimal Scaling]
+//      [AMD Quark ... FLUX.1-dev MXFP4 -- "MXFP4とは何か": 32-element blocks share
+//       one scale factor]
+//    E2M1 magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6} and the E8M0 bias of 127 are the
+//    OCP Microscaling (MX) v1.0 element / scale formats.
+//  * OCP scale rule (stock OCP MXFP4): block exponent = floor(log2 amax) - 2, i.e.
+//    the smallest e with amax / 2^e < 8 (2 = E2M1 emax), clamped to [-127, 127].
+//  * UOS rule: the scaling boundary Qmax = 7.25, read as the smallest e with
+//    amax / 2^e <= 7.25, clamped to [-127, 127].
+//      [MXAttention -- TL;DR and "What it actually does": Qmax = 7.25]
+//  * E2M1 element: round to nearest, ties to the even code index, saturating at
+//    6, sign bit always kept (so -0 and small negatives encode to 0x8).
+//  * Fixed 128-point block-Hadamard rotation: a deterministic, parameter-free
+//    rotation.  [AMD Quark adds native W4A8 ... Wan2.2 -- "Quark quantization
+//    pipeline and mixed-precision selection": fixed Hadamard rotations, no
+//    learned parameters]  Normalised Sylvester H/sqrt(128) applied by an FP32
+//    butterfly in a fixed order (stride 1, 2, 4, ..., 64), then one multiply by
+//    fl32(1/sqrt(128)).
+//  * FP8 E4M3 static activations (W4A8): q = E4M3_RNE_satfinite(fl32(x * inv_s))
+//    with inv_s = fl32(1/s), s the static per-tensor scale.
+//      [AMD Quark adds native W4A8 -- "MXFP4 formats and precision levels"]
+//  * GEMM: the kernel consumes MX operands directly, with no dequantisation
+//    phase, so its exact result is the GEMM of the dequantised operands:
+//      y[m][n] = alpha * sum_k deqA[m][k] * deqB[n][k] + bias[n]   (in FP64).
+//      [AMD Quark ... FLUX.1-dev MXFP4 -- "AMD Instinctプラットフォーム上の拡散
+//       モデル向けMXFP4量子化": the GEMM takes MXFP4 inputs with no dequant phase]
+//  * Scale-factor memory layout (not given by the pages; a reading): rows padded
+//    to a multiple of 128, scale columns to a multiple of 4, 512-byte atoms of
+//    128 rows x 4 scale columns, byte
+//      ((r/128)*(C/4) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + (c%4),
+//    padding bytes 0x00.  This is a separate function (oracle_sf_swizzle) applied
+//    to the logical [rows][K/32] scale array.
+//
+// Build: g++ -O2 -std=c++17 -ffp-contract=off -fPIC -shared -pthread
+// (no -ffast-math: every float operation below is a correctly rounded IEEE op).
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+namespace {
+
+constexpr int kBlock = 32;        // MX block size along K
+constexpr int kHadamardN = 128;   // block-Hadamard length along K
+[[maybe_unused]] constexpr int kRuleOCP = 0;
+constexpr int kRuleUOS = 1;
+
+float bf16_bits_to_float(uint16_t b) {
+  uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+// E2M1 magnitudes, index = the 3 low bits of a code.
+const double kE2M1Magnitude[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+// Runs fn(row_begin, row_end) over [0, rows) on nthreads std::threads.
+template <class Fn>
+void parallel_rows(int64_t rows, int nthreads, Fn fn) {
+  if (nthreads < 1) nthreads = 1;
+  if (rows < nthreads) nthreads = static_cast<int>(std::max<int64_t>(rows, 1));
+  if (nthreads == 1) {
+    fn(int64_t{0}, rows);
+    return;
+  }
+  std::vector<std::thread> pool;
+  const int64_t chunk = (rows + nthreads - 1) / nthreads;
+  for (int t = 0; t < nthreads; ++t) {
+    const int64_t b = t * chunk;
+    const int64_t e = std::min(rows, b + chunk);
+    if (b >= e) break;
+    pool.emplace_back([=] { fn(b, e); });
+  }
+  for (auto& th : pool) th.join();
+}
+
+}  // namespace
+
+extern "C" {
+
+// ---------------------------------------------------------------- element codecs
+
+// E2M1 encode of a value already divided by its block scale.
+// Nearest of the eight magnitudes to a = min(|v|, 6); on an exact tie the
+// candidate with the even index wins.  Bit 3 = sign bit of v, always kept.
+uint8_t oracle_e2m1_encode(double v) {
+  const int sign = std::signbit(v) ? 1 : 0;
+  double a = std::fabs(v);
+  if (a > 6.0) a = 6.0;
+  int best = 0;
+  double best_dist = INFINITY;
+  for (int i = 0; i < 8; ++i) {
+    const double d = std::fabs(a - kE2M1Magnitude[i]);
+    if (d < best_dist || (d == best_dist && i % 2 == 0)) {
+      best = i;
+      best_dist = d;
+    }
+  }
+  return static_cast<uint8_t>((sign << 3) | best);
+}
+
+double oracle_e2m1_decode(uint8_t code) {
+  const double mag = kE2M1Magnitude[code & 7];
+  return (code & 8) ? -mag : mag;
+}
+
+// FP8 E4M3 (OCP "FN" variant: no infinities, S.1111.111 is NaN) decode.
+double oracle_e4m3_decode(uint8_t code) {
+  const int sign = code >> 7;
+  const int exp_field = (code >> 3) & 0xF;
+  const int man = code & 7;
+  double mag;
+  if (exp_field == 0xF && man == 7) {
+    mag = NAN;
+  } else if (exp_field == 0) {
+    mag = std::ldexp(static_cast<double>(man), -9);  // subnormal: man/8 * 2^-6
+  } else {
+    mag = std::ldexp(1.0 + man / 8.0, exp_field - 7);
+  }
+  return sign ? -mag : mag;
+}
+
+// FP8 E4M3 encode: round to nearest, ties to even code (the even mantissa), with
+// saturation to the largest finite magnitude 448 ("satfinite"); sign bit kept.
+uint8_t oracle_e4m3_encode(double v) {
+  const int sign = std::signbit(v) ? 1 : 0;
+  double a = std::fabs(v);
+  if (a > 448.0) a = 448.0;
+  // Magnitudes of every non-negative finite code 0x00..0x7E, ascending.
+  static const std::vector<double> table = [] {
+    std::vector<double> t(0x7F);
+    for (int c = 0; c <= 0x7E; ++c) t[c] = oracle_e4m3_decode(static_cast<uint8_t>(c));
+    return t;
+  }();
+  int best = 0;
+  double best_dist = INFINITY;
+  for (int c = 0; c <= 0x7E; ++c) {
+    const double d = std::fabs(a - table[c]);
+    if (d < best_dist || (d == best_dist && c % 2 == 0)) {
+      best = c;
+      best_dist = d;
+    }
+  }
+  return static_cast<uint8_t>((sign << 7) | best);
+}
+
+// ---------------------------------------------------------------- block scale
+
+// Shared block exponent e (scale 2^e, stored as the E8M0 byte e + 127).
+//   OCP: smallest e in [-127, 127] with amax / 2^e <  8
+//   UOS: smallest e in [-127, 127] with amax / 2^e <= 7.25
+// amax = 0 gives e = -127 (byte 0x00).
+int oracle_block_exponent(double amax, int rule) {
+  for (int e = -127; e <= 127; ++e) {
+    if (rule == kRuleUOS) {
+      if (amax <= std::ldexp(7.25, e)) return e;
+    } else {
+      if (amax < std::ldexp(8.0, e)) return e;
+    }
+  }
+  return 127;  // only reached by non-finite amax, which is out of contract
+}
+
+// ---------------------------------------------------------------- rotation
+
+// 128-point normalised Sylvester-Hadamard on one chunk, in FP32, fixed order.
+void oracle_fwht128(const float* x, float* y) {
+  float t[kHadamardN];
+  for (int i = 0; i < kHadamardN; ++i) t[i] = x[i];
+  for (int h = 1; h < kHadamardN; h *= 2) {
+    for (int i = 0; i < kHadamardN; ++i) {
+      if (i & h) continue;
+      const float a = t[i];
+      const float b = t[i + h];
+      t[i] = a + b;
+      t[i + h] = a - b;
+    }
+  }
+  const float c = static_cast<float>(1.0 / std::sqrt(128.0));
+  for (int i = 0; i < kHadamardN; ++i) y[i] = t[i] * c;
+}
+
+float oracle_hadamard_scale(void) { return static_cast<float>(1.0 / std::sqrt(128.0)); }
+
+// ---------------------------------------------------------------- SF layout
+
+int64_t oracle_sf_padded_rows(int64_t rows) { return (rows + 127) / 128 * 128; }
+int64_t oracle_sf_padded_cols(int64_t K) { return (K / kBlock + 3) / 4 * 4; }
+int64_t oracle_sf_bytes(int64_t rows, int64_t K) {
+  return oracle_sf_padded_rows(rows) * oracle_sf_padded_cols(K);
+}
+
+int64_t oracle_sf_offset(int64_t r, int64_t c, int64_t K) {
+  const int64_t C = oracle_sf_padded_cols(K);
+  return ((r / 128) * (C / 4) + c / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4);
+}
+
+// logical [rows][K/32] -> physical swizzled buffer of oracle_sf_bytes(rows, K),
+// padding bytes 0x00.
+void oracle_sf_swizzle(const uint8_t* logical, int64_t rows, int64_t K, uint8_t* physical) {
+  const int64_t nb = K / kBlock;
+  std::memset(physical, 0, static_cast<size_t>(oracle_sf_bytes(rows, K)));
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t c = 0; c < nb; ++c) physical[oracle_sf_offset(r, c, K)] = logical[r * nb + c];
+}
+
+void oracle_sf_unswizzle(const uint8_t* physical, int64_t rows, int64_t K, uint8_t* logical) {
+  const int64_t nb = K / kBlock;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t c = 0; c < nb; ++c) logical[r * nb + c] = physical[oracle_sf_offset(r, c, K)];
+}
+
+// ---------------------------------------------------------------- quantizers
+
+// Optional rotation of one row: y = FP32 values the quantiser sees.
+static void row_to_float(const uint16_t* xrow, int64_t K, int hadamard, float* y) {
+  for (int64_t k = 0; k < K; ++k) y[k] = bf16_bits_to_float(xrow[k]);
+  if (hadamard) {
+    float tmp[kHadamardN];
+    for (int64_t c0 = 0; c0 < K; c0 += kHadamardN) {
+      oracle_fwht128(y + c0, tmp);
+      std::memcpy(y + c0, tmp, sizeof tmp);
+    }
+  }
+}
+
+// MXFP4 quantisation of rows x K BF16 values (row stride ld elements).
+// codes: [rows][K/2] bytes, element k in byte k/2, low nibble when k is even.
+// sf_logical: [rows][K/32] E8M0 bytes.
+void oracle_quantize_mxfp4(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, int rule,
+                           int hadamard, uint8_t* codes, uint8_t* sf_logical, int nthreads) {
+  parallel_rows(rows, nthreads, [&](int64_t r0, int64_t r1) {
+    std::vector<float> y(static_cast<size_t>(K));
+    for (int64_t r = r0; r < r1; ++r) {
+      row_to_float(x + r * ld, K, hadamard, y.data());
+      for (int64_t b = 0; b < K / kBlock; ++b) {
+        const float* blk = y.data() + b * kBlock;
+        double amax = 0.0;
+        for (int i = 0; i < kBlock; ++i) amax = std::max(amax, std::fabs(static_cast<double>(blk[i])));
+        const int e = oracle_block_exponent(amax, rule);
+        sf_logical[r * (K / kBlock) + b] = static_cast<uint8_t>(e + 127);
+        for (int i = 0; i < kBlock; ++i) {
+          const int64_t k = b * kBlock + i;
+          const uint8_t q = oracle_e2m1_encode(std::ldexp(static_cast<double>(blk[i]), -e));
+          uint8_t& byte = codes[r * (K / 2) + k / 2];
+          if (k % 2 == 0) byte = static_cast<uint8_t>((byte & 0xF0) | q);
+          else            byte = static_cast<uint8_t>((byte & 0x0F) | (q << 4));
+        }
+      }
+    }
+  });
+}
+
+// Returns the rotated FP32 values the quantiser sees (for tests).
+void oracle_rotate_rows(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, int hadamard,
+                        float* y) {
+  for (int64_t r = 0; r < rows; ++r) row_to_float(x + r * ld, K, hadamard, y + r * K);
+}
+
+// Static FP8 E4M3 activation quantisation: q = E4M3(fl32(x * inv_scale)).
+void oracle_quantize_fp8(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, float inv_scale,
+                         uint8_t* q, int nthreads) {
+  parallel_rows(rows, nthreads, [&](int64_t r0, int64_t r1) {
+    for (int64_t r = r0; r < r1; ++r)
+      for (int64_t k = 0; k < K; ++k) {
+        const float v = bf16_bits_to_float(x[r * ld + k]) * inv_scale;  // fl32 product
+        q[r * K + k] = oracle_e4m3_encode(static_cast<double>(v));
+      }
+  });
+}
+
+// ---------------------------------------------------------------- dequantisation
+
+// MXFP4 -> FP64: value = E2M1(code) * 2^(sf - 127), sf read from the swizzled buffer.
+void oracle_dequant_mxfp4(const uint8_t* codes, const uint8_t* sf_physical, int64_t rows,
+                          int64_t K, double* out) {
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t k = 0; k < K; ++k) {
+      const uint8_t byte = codes[r * (K / 2) + k / 2];
+      const uint8_t q = (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+      const int sf = sf_physical[oracle_sf_offset(r, k / kBlock, K)];
+      out[r * K + k] = std::ldexp(oracle_e2m1_decode(q), sf - 127);
+    }
+}
+
+// ---------------------------------------------------------------- GEMM
+
+// y[i][n] = alpha * sum_k A(row_idx[i], k) * B(n, k) + bias[n], FP64, unrounded.
+//   a_kind 0: A is MXFP4 (a_codes [M][K/2] + swizzled a_sf)
+//   a_kind 1: A is FP8 E4M3 (a_codes [M][K]; a_sf unused)
+//   B is MXFP4 (b_codes [N][K/2] + swizzled b_sf); bias: N BF16 values or null.
+void oracle_gemm(int a_kind, const uint8_t* a_codes, const uint8_t* a_sf, int64_t M,
+                 const uint8_t* b_codes, const uint8_t* b_sf, int64_t N, int64_t K, double alpha,
+                 const uint16_t* bias, const int64_t* row_idx, int64_t n_rows, double* y,
+                 int nthreads) {
+  std::vector<double> B(static_cast<size_t>(N * K));
+  oracle_dequant_mxfp4(b_codes, b_sf, N, K, B.data());
+  parallel_rows(n_rows, nthreads, [&](int64_t i0, int64_t i1) {
+    std::vector<double> a(static_cast<size_t>(K));
+    for (int64_t i = i0; i < i1; ++i) {
+      const int64_t m = row_idx[i];
+      if (a_kind == 0) {
+        for (int64_t k = 0; k < K; ++k) {
+          const uint8_t byte = a_codes[m * (K / 2) + k / 2];
+          const uint8_t q = (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+          const int sf = a_sf[oracle_sf_offset(m, k / kBlock, K)];
+          a[k] = std::ldexp(oracle_e2m1_decode(q), sf - 127);
+        }
+      } else {
+        for (int64_t k = 0; k < K; ++k) a[k] = oracle_e4m3_decode(a_codes[m * K + k]);
+      }
+      for (int64_t n = 0; n < N; ++n) {
+        const double* b = B.data() + n * K;
+        double acc = 0.0;
+        for (int64_t k = 0; k < K; ++k) acc += a[k] * b[k];
+        double v = alpha * acc;
+        if (bias) v += static_cast<double>(bf16_bits_to_float(bias[n]));
+        y[i * N + n] = v;
+      }
+    }
+  });
+  (void)M;
+}
+
+}  // extern "C"
