@@ -1,0 +1,173 @@
+/*
+ * mxq.h -- C ABI of libmxq: the MXFP4 quantized linear layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer, as the pages state the problem:
+ *   - weights are quantised offline to OCP MXFP4 for both W4A4 and W4A8;
+ *   - activations are quantised dynamically to MXFP4 (W4A4) or statically to
+ *     FP8 E4M3 with one per-tensor scale (W4A8);
+ *     [AMD Quark adds native W4A8 mixed-precision for Wan2.2 video generation on
+ *      MI350 -- "Quark quantization pipeline and mixed-precision selection",
+ *      bullets "MXFP4 formats and precision levels" and "Native execution paths"]
+ *   - the GEMM consumes the MX operands directly, with no dequantisation phase and
+ *     no conversion to FP16/BF16 in between;
+ *     [AMD Quark ... FLUX.1-dev MXFP4 on MI350 -- "AMD Instinctプラットフォーム上の
+ *      拡散モデル向けMXFP4量子化", and "MXFP4とは何か": 32-element blocks share one
+ *      scale factor]
+ *   - an optional fixed (parameter-free) Hadamard rotation precedes quantisation;
+ *     [Wan2.2 page above -- "Fixed rotation selector"]
+ *   - the block scale can follow the stock OCP rule or the data-free UOS boundary
+ *     Qmax = 7.25.  [MXAttention: Data-Free Optimal Scaling and Pre-Normalization
+ *     Quantization for MXFP4 Attention -- TL;DR, "What it actually does"]
+ *
+ * Conventions common to every call
+ *   - Every pointer argument is a DEVICE pointer (cudaMalloc'd or equivalent) on the
+ *     current CUDA device, at least 16-byte aligned.  The caller allocates and owns
+ *     every buffer; the library allocates no device memory and keeps no per-call
+ *     state (it reads its own static device status word, see mxq_debug_poll).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronises it.  Calls are thread-safe.
+ *   - Arguments are validated on the host before anything is launched; on any
+ *     error nothing is launched and a status other than MXQ_OK is returned.  A
+ *     launch failure returns MXQ_ERR_CUDA.  No C++ exception crosses this ABI.
+ *   - Matrices are row-major.  X[M][K] activations (BF16), W[N][K] weights (BF16,
+ *     nn.Linear convention, K-major), D[M][N] output (BF16).
+ *
+ * Data layouts (a reading: the pages do not fix them)
+ *   - MXFP4 codes: [rows][K/2] bytes, row stride exactly K/2.  Element k sits in
+ *     byte k/2, low nibble when k is even.  Nibble = sign<<3 | index, index 0..7 <->
+ *     magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6} (OCP MX v1.0 E2M1).
+ *   - Scale factors (E8M0, byte = e + 127, value 2^e): one byte per (row, 32-block).
+ *     Physical buffer of mxq_sf_bytes(rows, K) bytes: rows padded to R = 128*ceil(rows/128),
+ *     scale columns to C = 4*ceil((K/32)/4); the scale of (row r, block c) is at byte
+ *       ((r/128)*(C/4) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + (c%4)
+ *     (512-byte atoms of 128 rows x 4 blocks, the tcgen05 block-scale operand layout).
+ *     Padding bytes are written as 0x00.
+ *   - FP8 activations: [M][K] E4M3 bytes, row stride exactly K.
+ */
+#ifndef MXQ_H_
+#define MXQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MXQ_API __attribute__((visibility("default")))
+#else
+#define MXQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+/* Identical to cudaStream_t / CUstream. */
+typedef struct CUstream_st* mxq_stream_t;
+
+typedef enum {
+  MXQ_OK = 0,
+  MXQ_ERR_INVALID_ARG = 1, /* null pointer, bad enum, non-finite / non-positive scale  */
+  MXQ_ERR_SHAPE = 2,       /* dimension out of range or not a required multiple         */
+  MXQ_ERR_ALIGN = 3,       /* pointer or leading dimension misaligned                   */
+  MXQ_ERR_UNSUPPORTED = 4, /* no sm_100 device current, or configuration not built      */
+  MXQ_ERR_CUDA = 5,        /* a CUDA runtime / driver call failed                       */
+  MXQ_ERR_TIMEOUT = 6      /* a kernel gave up a bounded wait (reported by mxq_debug_poll) */
+} mxq_status;
+
+typedef enum {
+  MXQ_SCALE_OCP = 0, /* e = floor(log2 amax) - 2: smallest e with amax/2^e <  8    */
+  MXQ_SCALE_UOS = 1  /* smallest e with amax/2^e <= 7.25 (Qmax of the UOS boundary) */
+} mxq_scale_rule;
+
+typedef enum {
+  MXQ_ACT_MXFP4 = 0,   /* dynamic MXFP4 activations (W4A4)            */
+  MXQ_ACT_FP8_E4M3 = 1 /* static per-tensor FP8 E4M3 activations (W4A8) */
+} mxq_act_format;
+
+/* Human-readable name of a status code (static string, never NULL). */
+MXQ_API const char* mxq_status_string(mxq_status status);
+
+/* Size in bytes of the padded, swizzled scale-factor buffer for a [rows][K]
+ * MXFP4 tensor (K a multiple of 32).  Returns -1 for invalid sizes. */
+MXQ_API int64_t mxq_sf_bytes(int64_t rows, int64_t K);
+
+/*
+ * mxq_quantize_act -- dynamic activation quantisation, one pass over X.
+ *
+ * MXFP4 (fmt = MXQ_ACT_MXFP4): for each row and each 32-element block along K:
+ *   optional y = x * H128/sqrt(128) per 128-element chunk (hadamard128 != 0; fixed
+ *   butterfly order, FP32), amax = max |y| over the block, exponent e by `rule`
+ *   (clamped to [-127, 127], amax = 0 -> e = -127), codes = E2M1 round-to-nearest-
+ *   even of y * 2^-e with saturation at 6 and the sign bit kept; scale byte e + 127.
+ *   Writes q_out ([M][K/2] codes) and sf_out (mxq_sf_bytes(M, K) bytes, padding 0).
+ *   `act_scale` is ignored.
+ * FP8 (fmt = MXQ_ACT_FP8_E4M3): q = E4M3_RNE_satfinite(fl32(x * fl32(1/act_scale)))
+ *   for the static per-tensor scale act_scale > 0 (dequantised value = q * act_scale).
+ *   Writes q_out ([M][K] bytes); sf_out must be NULL; rule and hadamard128 must be
+ *   MXQ_SCALE_OCP and 0.
+ *
+ * x_bf16: device [M][ldx] BF16; 1 <= M <= 8388480 (65535 tiles of 128 rows; FP8 mode
+ * allows up to 2^31); 32 <= K <= 2^22 with K % 32 == 0 (K % 128 == 0 when hadamard128);
+ * ldx >= K and ldx % 8 == 0.
+ * Errors: MXQ_ERR_INVALID_ARG, MXQ_ERR_SHAPE, MXQ_ERR_ALIGN, MXQ_ERR_CUDA.
+ */
+MXQ_API mxq_status mxq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                            mxq_act_format fmt, mxq_scale_rule rule, int hadamard128,
+                            float act_scale, void* q_out, void* sf_out, mxq_stream_t stream);
+
+/*
+ * mxq_pack_weight -- offline MXFP4 weight quantisation (run once, not on the hot path).
+ *
+ * Same per-block arithmetic as the MXFP4 activation quantiser, on W[N][K] rows:
+ * codes_out [N][K/2], sf_out mxq_sf_bytes(N, K) bytes.  Use rule = MXQ_SCALE_OCP for
+ * "OCP MXFP4 weights"; hadamard128 must equal the activation side's setting (the
+ * library cannot check this: X R (W R)^T = X W^T only when both sides rotate).
+ * w_bf16: device [N][ldw] BF16, 1 <= N <= 8388480, 32 <= K <= 2^22, K % 32 == 0
+ * (K % 128 == 0 when hadamard128), ldw >= K, ldw % 8 == 0.
+ */
+MXQ_API mxq_status mxq_pack_weight(const void* w_bf16, int64_t N, int64_t K, int64_t ldw,
+                           mxq_scale_rule rule, int hadamard128, void* codes_out, void* sf_out,
+                           mxq_stream_t stream);
+
+/*
+ * mxq_gemm_w4a4 -- D[M][N] = bf16_rne(alpha * sum_k deqA[m][k] * deqB[n][k] + bias[n])
+ * with deq = E2M1 value * 2^(scale byte - 127), accumulated in FP32 on the tensor
+ * cores (tcgen05.mma kind::mxf4 block_scale) without dequantising either operand.
+ *
+ * a_codes [M][K/2] + a_sf (mxq_sf_bytes(M, K)); b_codes [N][K/2] + b_sf
+ * (mxq_sf_bytes(N, K)), both as written by the quantiser / packer.
+ * bias_bf16: NULL or [N] BF16.  d_bf16: [M][ldd] BF16, ldd >= N, ldd % 8 == 0.
+ * 1 <= M, N <= 2^30 (any value: ragged tiles are handled); 128 <= K <= 2^22, K % 128 == 0.
+ * alpha must be finite.
+ */
+MXQ_API mxq_status mxq_gemm_w4a4(const void* a_codes, const void* a_sf, const void* b_codes,
+                         const void* b_sf, int64_t M, int64_t N, int64_t K, float alpha,
+                         const void* bias_bf16, void* d_bf16, int64_t ldd, mxq_stream_t stream);
+
+/*
+ * mxq_gemm_w4a8 -- D[M][N] = bf16_rne(act_scale * sum_k e4m3(A[m][k]) * deqB[n][k] + bias[n])
+ * on the tensor cores (tcgen05.mma kind::mxf8f6f4 block_scale: A = E4M3 with unit
+ * block scales, B = E2M1 with its E8M0 block scales); the per-tensor activation
+ * scale is applied in the FP32 epilogue.
+ *
+ * a_e4m3 [M][K] as written by mxq_quantize_act(fmt = MXQ_ACT_FP8_E4M3, same act_scale);
+ * b_codes/b_sf as for W4A4 (b_codes must be 32-byte aligned).  Shapes as for W4A4.
+ */
+MXQ_API mxq_status mxq_gemm_w4a8(const void* a_e4m3, float act_scale, const void* b_codes,
+                         const void* b_sf, int64_t M, int64_t N, int64_t K, const void* bias_bf16,
+                         void* d_bf16, int64_t ldd, mxq_stream_t stream);
+
+/*
+ * mxq_debug_poll -- reads and clears the library's device status word, written by a
+ * kernel that gave up one of its bounded waits (each wait on a barrier or a copy is
+ * capped at about a second, after which the kernel records MXQ_ERR_TIMEOUT, drains
+ * its own copies in flight, releases its tensor memory and returns).  Synchronises
+ * the current device.  Returns MXQ_OK when no kernel has reported anything.
+ */
+MXQ_API mxq_status mxq_debug_poll(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXQ_H_ */

@@ -1,0 +1,266 @@
+// mxq.cu -- libmxq: the C ABI of include/mxq.h (host-side validation, TMA tensor-map
+// encoding and launches) over the sm_100a kernels in quantize.cuh and gemm.cuh.
+// One translation unit, so the library's device status word exists exactly once.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "mxq.h"
+#include "gemm.cuh"
+#include "quantize.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Per-device facts, looked up once per device.
+struct DeviceInfo {
+  bool ok = false;
+  int sm_count = 0;
+};
+
+DeviceInfo device_info(int dev) {
+  static DeviceInfo info[64];
+  static std::once_flag once[64];
+  if (dev < 0 || dev >= 64) return {};
+  std::call_once(once[dev], [dev] {
+    cudaDeviceProp p;
+    if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return;
+    info[dev].ok = (p.major == 10 && p.minor == 0);
+    info[dev].sm_count = p.multiProcessorCount;
+  });
+  return info[dev];
+}
+
+mxq_status current_device(DeviceInfo* out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MXQ_ERR_CUDA;
+  *out = device_info(dev);
+  if (!out->ok) return MXQ_ERR_UNSUPPORTED;
+  return MXQ_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+mxq_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+// 2-D tensor map over a row-major [rows][cols] matrix.
+bool make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t cols, uint64_t rows,
+                  uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool kW4A8>
+mxq_status launch_gemm(const void* a, const void* a_sf, const void* b, const void* b_sf, int64_t M, int64_t N,
+                       int64_t K, float alpha, const void* bias, void* d, int64_t ldd, cudaStream_t stream) {
+  DeviceInfo dev;
+  mxq_status st = current_device(&dev);
+  if (st != MXQ_OK) return st;
+  CUtensorMap ta, tb, td;
+  bool ok;
+  if (kW4A8) {
+    ok = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K, M, K, 128, mxq::kBM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, b, K, N, K / 2, 128, mxq::kBN,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    ok = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K / 2, M, K / 2, 128, mxq::kBM,
+                      CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K / 2, N, K / 2, 128, mxq::kBN,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+  }
+  ok = ok && make_tmap_2d(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, N, M, ldd * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (!ok) return MXQ_ERR_CUDA;
+
+  using S = mxq::GemmShape<kW4A8>;
+  auto kernel = mxq::mx_gemm_kernel<kW4A8>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [&] {
+    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return MXQ_ERR_CUDA;
+  const int64_t tiles = ((M + mxq::kBM - 1) / mxq::kBM) * ((N + mxq::kBN - 1) / mxq::kBN);
+  const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+  kernel<<<grid, mxq::kGemmThreads, S::kSmemBytes, stream>>>(
+      ta, tb, td, static_cast<const uint8_t*>(a_sf), static_cast<const uint8_t*>(b_sf),
+      static_cast<const __nv_bfloat16*>(bias), static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), alpha);
+  return launch_status();
+}
+
+mxq_status check_gemm_shapes(const void* a, const void* b, const void* b_sf, const void* d, int64_t M, int64_t N,
+                             int64_t K, int64_t ldd, const void* bias) {
+  if (!a || !b || !b_sf || !d) return MXQ_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 128 || K % 128 != 0) return MXQ_ERR_SHAPE;
+  if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30) || K > (int64_t(1) << 22)) return MXQ_ERR_SHAPE;
+  const int64_t tiles = ((M + mxq::kBM - 1) / mxq::kBM) * ((N + mxq::kBN - 1) / mxq::kBN);
+  if (tiles > INT32_MAX) return MXQ_ERR_SHAPE;  // tile indices are 32-bit in the kernel
+  if (ldd < N || ldd % 8 != 0) return MXQ_ERR_ALIGN;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(b_sf, 16) || !aligned(d, 16)) return MXQ_ERR_ALIGN;
+  if (bias && !aligned(bias, 16)) return MXQ_ERR_ALIGN;
+  return MXQ_OK;
+}
+
+mxq_status launch_mxfp4(bool weight, const void* x, int64_t rows, int64_t K, int64_t ld, mxq_scale_rule rule,
+                        int hadamard, void* codes, void* sf, cudaStream_t stream) {
+  // grid.x: 128-column tiles (K <= 2^22 keeps it <= 32768), grid.y: 128-row tiles.
+  const dim3 grid(static_cast<unsigned>((K + 127) / 128), static_cast<unsigned>((rows + 127) / 128));
+  const auto* xp = static_cast<const uint16_t*>(x);
+  auto* cp = static_cast<uint8_t*>(codes);
+  auto* sp = static_cast<uint8_t*>(sf);
+  const bool uos = rule == MXQ_SCALE_UOS;
+  const int sel = (hadamard ? 2 : 0) | (uos ? 1 : 0);
+  if (weight) {
+    switch (sel) {
+      case 0: mxq::pack_weight_mxfp4_kernel<false, false><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ld, cp, sp); break;
+      case 1: mxq::pack_weight_mxfp4_kernel<false, true><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ld, cp, sp); break;
+      case 2: mxq::pack_weight_mxfp4_kernel<true, false><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ld, cp, sp); break;
+      default: mxq::pack_weight_mxfp4_kernel<true, true><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ld, cp, sp); break;
+    }
+  } else {
+    switch (sel) {
+      case 0: mxq::quantize_act_mxfp4_kernel<false, false><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ld, cp, sp); break;
+      case 1: mxq::quantize_act_mxfp4_kernel<false, true><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ld, cp, sp); break;
+      case 2: mxq::quantize_act_mxfp4_kernel<true, false><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ld, cp, sp); break;
+      default: mxq::quantize_act_mxfp4_kernel<true, true><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ld, cp, sp); break;
+    }
+  }
+  return launch_status();
+}
+
+mxq_status check_quant_args(const void* x, int64_t rows, int64_t K, int64_t ld, mxq_scale_rule rule, int hadamard,
+                            const void* q, const void* sf) {
+  if (!x || !q || !sf) return MXQ_ERR_INVALID_ARG;
+  if (rule != MXQ_SCALE_OCP && rule != MXQ_SCALE_UOS) return MXQ_ERR_INVALID_ARG;
+  // rows <= 65535 * 128 keeps grid.y within its limit
+  if (rows < 1 || rows > int64_t(65535) * 128 || K < 32 || K % 32 != 0 || K > (int64_t(1) << 22)) return MXQ_ERR_SHAPE;
+  if (hadamard && K % 128 != 0) return MXQ_ERR_SHAPE;
+  if (ld < K || ld % 8 != 0) return MXQ_ERR_ALIGN;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(sf, 16)) return MXQ_ERR_ALIGN;
+  return MXQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mxq_status_string(mxq_status s) {
+  switch (s) {
+    case MXQ_OK: return "MXQ_OK";
+    case MXQ_ERR_INVALID_ARG: return "MXQ_ERR_INVALID_ARG";
+    case MXQ_ERR_SHAPE: return "MXQ_ERR_SHAPE";
+    case MXQ_ERR_ALIGN: return "MXQ_ERR_ALIGN";
+    case MXQ_ERR_UNSUPPORTED: return "MXQ_ERR_UNSUPPORTED";
+    case MXQ_ERR_CUDA: return "MXQ_ERR_CUDA";
+    case MXQ_ERR_TIMEOUT: return "MXQ_ERR_TIMEOUT";
+  }
+  return "MXQ_ERR_UNKNOWN";
+}
+
+int64_t mxq_sf_bytes(int64_t rows, int64_t K) {
+  if (rows < 1 || K < 32 || K % 32 != 0) return -1;
+  return (rows + 127) / 128 * 128 * ((K / 32 + 3) / 4 * 4);
+}
+
+mxq_status mxq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, mxq_act_format fmt,
+                            mxq_scale_rule rule, int hadamard128, float act_scale, void* q_out, void* sf_out,
+                            mxq_stream_t stream) {
+  if (fmt == MXQ_ACT_FP8_E4M3) {
+    if (!x_bf16 || !q_out || sf_out) return MXQ_ERR_INVALID_ARG;
+    if (rule != MXQ_SCALE_OCP || hadamard128) return MXQ_ERR_INVALID_ARG;
+    if (!(act_scale > 0.f) || !std::isfinite(act_scale)) return MXQ_ERR_INVALID_ARG;
+    if (M < 1 || M > (int64_t(1) << 31) || K < 32 || K % 32 != 0 || K > (int64_t(1) << 22)) return MXQ_ERR_SHAPE;
+    if (ldx < K || ldx % 8 != 0) return MXQ_ERR_ALIGN;
+    if (!aligned(x_bf16, 16) || !aligned(q_out, 16)) return MXQ_ERR_ALIGN;
+    const float inv = 1.0f / act_scale;  // fl32(1 / s), IEEE division on the host
+    if (!std::isfinite(inv)) return MXQ_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    mxq_status st = current_device(&dev);
+    if (st != MXQ_OK) return st;
+    const int64_t chunks = M * (K / 8);
+    int64_t blocks = (chunks + mxq::kQuantThreads - 1) / mxq::kQuantThreads;
+    const int64_t cap = static_cast<int64_t>(dev.sm_count) * 16;
+    if (blocks > cap) blocks = cap;
+    mxq::quantize_act_fp8_kernel<<<static_cast<unsigned>(blocks), mxq::kQuantThreads, 0, stream>>>(
+        static_cast<const uint16_t*>(x_bf16), M, K, ldx, inv, static_cast<uint8_t*>(q_out));
+    return launch_status();
+  }
+  if (fmt != MXQ_ACT_MXFP4) return MXQ_ERR_INVALID_ARG;
+  mxq_status st = check_quant_args(x_bf16, M, K, ldx, rule, hadamard128, q_out, sf_out);
+  if (st != MXQ_OK) return st;
+  DeviceInfo dev;
+  st = current_device(&dev);
+  if (st != MXQ_OK) return st;
+  return launch_mxfp4(false, x_bf16, M, K, ldx, rule, hadamard128, q_out, sf_out, stream);
+}
+
+mxq_status mxq_pack_weight(const void* w_bf16, int64_t N, int64_t K, int64_t ldw, mxq_scale_rule rule,
+                           int hadamard128, void* codes_out, void* sf_out, mxq_stream_t stream) {
+  mxq_status st = check_quant_args(w_bf16, N, K, ldw, rule, hadamard128, codes_out, sf_out);
+  if (st != MXQ_OK) return st;
+  DeviceInfo dev;
+  st = current_device(&dev);
+  if (st != MXQ_OK) return st;
+  return launch_mxfp4(true, w_bf16, N, K, ldw, rule, hadamard128, codes_out, sf_out, stream);
+}
+
+mxq_status mxq_gemm_w4a4(const void* a_codes, const void* a_sf, const void* b_codes, const void* b_sf, int64_t M,
+                         int64_t N, int64_t K, float alpha, const void* bias_bf16, void* d_bf16, int64_t ldd,
+                         mxq_stream_t stream) {
+  if (!a_sf) return MXQ_ERR_INVALID_ARG;
+  if (!std::isfinite(alpha)) return MXQ_ERR_INVALID_ARG;
+  mxq_status st = check_gemm_shapes(a_codes, b_codes, b_sf, d_bf16, M, N, K, ldd, bias_bf16);
+  if (st != MXQ_OK) return st;
+  if (!aligned(a_sf, 16)) return MXQ_ERR_ALIGN;
+  return launch_gemm<false>(a_codes, a_sf, b_codes, b_sf, M, N, K, alpha, bias_bf16, d_bf16, ldd, stream);
+}
+
+mxq_status mxq_gemm_w4a8(const void* a_e4m3, float act_scale, const void* b_codes, const void* b_sf, int64_t M,
+                         int64_t N, int64_t K, const void* bias_bf16, void* d_bf16, int64_t ldd,
+                         mxq_stream_t stream) {
+  if (!(act_scale > 0.f) || !std::isfinite(act_scale)) return MXQ_ERR_INVALID_ARG;
+  mxq_status st = check_gemm_shapes(a_e4m3, b_codes, b_sf, d_bf16, M, N, K, ldd, bias_bf16);
+  if (st != MXQ_OK) return st;
+  if (!aligned(b_codes, 32)) return MXQ_ERR_ALIGN;  // 16U4_ALIGN16B tensor maps need 32-byte bases
+  return launch_gemm<true>(a_e4m3, nullptr, b_codes, b_sf, M, N, K, act_scale, bias_bf16, d_bf16, ldd, stream);
+}
+
+mxq_status mxq_debug_poll(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return MXQ_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, mxq::g_status, sizeof v) != cudaSuccess) return MXQ_ERR_CUDA;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(mxq::g_status, &zero, sizeof zero) != cudaSuccess) return MXQ_ERR_CUDA;
+    return static_cast<mxq_status>(v);
+  }
+  return MXQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,198 @@
+"""Thin Python binding of libmxq (the C ABI in include/mxq.h).
+
+Argument marshalling only: every step of the quantized linear layer runs in the
+library's sm_100a kernels.  Functions named ``mxq_*`` mirror the C entry points one
+for one (device buffers may be given as torch CUDA tensors or raw integer device
+pointers); the lower-case helpers below them allocate the output tensors and call
+the ``mxq_*`` functions.  There is no fallback: if the shared library is missing or
+the device is not an sm_100 GPU, calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmxq.so")
+
+MXQ_OK = 0
+STATUS_NAMES = {0: "MXQ_OK", 1: "MXQ_ERR_INVALID_ARG", 2: "MXQ_ERR_SHAPE", 3: "MXQ_ERR_ALIGN",
+                4: "MXQ_ERR_UNSUPPORTED", 5: "MXQ_ERR_CUDA", 6: "MXQ_ERR_TIMEOUT"}
+MXQ_SCALE_OCP, MXQ_SCALE_UOS = 0, 1
+MXQ_ACT_MXFP4, MXQ_ACT_FP8_E4M3 = 0, 1
+
+EXPORTED = ("mxq_status_string", "mxq_sf_bytes", "mxq_quantize_act", "mxq_pack_weight", "mxq_gemm_w4a4",
+            "mxq_gemm_w4a8", "mxq_debug_poll")
+
+
+class MxqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libmxq.so from the package directory (built by ``build.py``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"libmxq.so not built ({_LIB_PATH}); run `python -m mxfp4_block_scaled_mxq_b200.build`")
+    L = ctypes.CDLL(_LIB_PATH)
+    P, I64, I32, F32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    L.mxq_status_string.argtypes = [I32]
+    L.mxq_status_string.restype = ctypes.c_char_p
+    L.mxq_sf_bytes.argtypes = [I64, I64]
+    L.mxq_sf_bytes.restype = I64
+    L.mxq_quantize_act.argtypes = [P, I64, I64, I64, I32, I32, I32, F32, P, P, P]
+    L.mxq_quantize_act.restype = I32
+    L.mxq_pack_weight.argtypes = [P, I64, I64, I64, I32, I32, P, P, P]
+    L.mxq_pack_weight.restype = I32
+    L.mxq_gemm_w4a4.argtypes = [P, P, P, P, I64, I64, I64, F32, P, P, I64, P]
+    L.mxq_gemm_w4a4.restype = I32
+    L.mxq_gemm_w4a8.argtypes = [P, F32, P, P, I64, I64, I64, P, P, I64, P]
+    L.mxq_gemm_w4a8.restype = I32
+    L.mxq_debug_poll.argtypes = []
+    L.mxq_debug_poll.restype = I32
+    _lib = L
+    return L
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("libmxq takes device buffers: got a CPU tensor")
+    if not t.is_contiguous():
+        raise ValueError("libmxq buffers must be contiguous (use the leading-dimension argument for strides)")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str) -> None:
+    if status != MXQ_OK:
+        raise MxqError(status, where)
+
+
+# ------------------------------------------------------------------ C entry points
+def mxq_status_string(status: int) -> str:
+    return lib().mxq_status_string(int(status)).decode()
+
+
+def mxq_sf_bytes(rows: int, K: int) -> int:
+    return int(lib().mxq_sf_bytes(int(rows), int(K)))
+
+
+def mxq_quantize_act(x, M, K, ldx, fmt, rule, hadamard128, act_scale, q_out, sf_out, stream=None) -> None:
+    _check(lib().mxq_quantize_act(_ptr(x), int(M), int(K), int(ldx), int(fmt), int(rule), int(bool(hadamard128)),
+                                  float(act_scale), _ptr(q_out), _ptr(sf_out), _stream(stream)), "mxq_quantize_act")
+
+
+def mxq_pack_weight(w, N, K, ldw, rule, hadamard128, codes_out, sf_out, stream=None) -> None:
+    _check(lib().mxq_pack_weight(_ptr(w), int(N), int(K), int(ldw), int(rule), int(bool(hadamard128)),
+                                 _ptr(codes_out), _ptr(sf_out), _stream(stream)), "mxq_pack_weight")
+
+
+def mxq_gemm_w4a4(a_codes, a_sf, b_codes, b_sf, M, N, K, alpha, bias, d, ldd, stream=None) -> None:
+    _check(lib().mxq_gemm_w4a4(_ptr(a_codes), _ptr(a_sf), _ptr(b_codes), _ptr(b_sf), int(M), int(N), int(K),
+                               float(alpha), _ptr(bias), _ptr(d), int(ldd), _stream(stream)), "mxq_gemm_w4a4")
+
+
+def mxq_gemm_w4a8(a_e4m3, act_scale, b_codes, b_sf, M, N, K, bias, d, ldd, stream=None) -> None:
+    _check(lib().mxq_gemm_w4a8(_ptr(a_e4m3), float(act_scale), _ptr(b_codes), _ptr(b_sf), int(M), int(N), int(K),
+                               _ptr(bias), _ptr(d), int(ldd), _stream(stream)), "mxq_gemm_w4a8")
+
+
+def mxq_debug_poll() -> int:
+    return int(lib().mxq_debug_poll())
+
+
+# ------------------------------------------------------------------ allocating helpers
+def _bf16_2d(x: torch.Tensor, name: str) -> torch.Tensor:
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError(f"{name}: expected a 2-D bfloat16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError(f"{name}: rows must be contiguous")
+    return x
+
+
+def quantize_act(x: torch.Tensor, rule: int = MXQ_SCALE_OCP, hadamard128: bool = False, out=None, stream=None):
+    """Dynamic MXFP4 quantisation of X[M][K] -> (codes [M][K/2] uint8, sf uint8[mxq_sf_bytes(M, K)])."""
+    x = _bf16_2d(x, "x")
+    M, K = x.shape
+    if out is None:
+        out = (torch.empty(M, K // 2, dtype=torch.uint8, device=x.device),
+               torch.empty(mxq_sf_bytes(M, K), dtype=torch.uint8, device=x.device))
+    q, sf = out
+    mxq_quantize_act(x.data_ptr(), M, K, x.stride(0), MXQ_ACT_MXFP4, rule, hadamard128, 1.0, q, sf, stream)
+    return q, sf
+
+
+def quantize_act_fp8(x: torch.Tensor, act_scale: float, out=None, stream=None) -> torch.Tensor:
+    """Static FP8 E4M3 quantisation of X[M][K] with per-tensor scale s -> uint8 [M][K]."""
+    x = _bf16_2d(x, "x")
+    M, K = x.shape
+    q = torch.empty(M, K, dtype=torch.uint8, device=x.device) if out is None else out
+    mxq_quantize_act(x.data_ptr(), M, K, x.stride(0), MXQ_ACT_FP8_E4M3, MXQ_SCALE_OCP, False, act_scale, q, None,
+                     stream)
+    return q
+
+
+def pack_weight(w: torch.Tensor, rule: int = MXQ_SCALE_OCP, hadamard128: bool = False, stream=None):
+    """Offline MXFP4 packing of W[N][K] -> (codes [N][K/2] uint8, sf uint8[mxq_sf_bytes(N, K)])."""
+    w = _bf16_2d(w, "w")
+    N, K = w.shape
+    codes = torch.empty(N, K // 2, dtype=torch.uint8, device=w.device)
+    sf = torch.empty(mxq_sf_bytes(N, K), dtype=torch.uint8, device=w.device)
+    mxq_pack_weight(w.data_ptr(), N, K, w.stride(0), rule, hadamard128, codes, sf, stream)
+    return codes, sf
+
+
+def _out_bf16(M: int, N: int, device) -> torch.Tensor:
+    """[M][N] BF16 view of a buffer whose rows are padded to a multiple of 8 elements
+    (the output's row stride must be a multiple of 16 bytes)."""
+    ldd = (N + 7) // 8 * 8
+    return torch.empty(M, ldd, dtype=torch.bfloat16, device=device)[:, :N]
+
+
+def gemm_w4a4(a_codes, a_sf, b_codes, b_sf, M, N, K, alpha=1.0, bias=None, out=None, stream=None) -> torch.Tensor:
+    """D[M][N] (BF16) = alpha * deq(A) deq(B)^T + bias, on the tensor cores."""
+    d = _out_bf16(M, N, a_codes.device) if out is None else out
+    mxq_gemm_w4a4(a_codes, a_sf, b_codes, b_sf, M, N, K, alpha, bias, d.data_ptr(), d.stride(0), stream)
+    return d
+
+
+def gemm_w4a8(a_e4m3, act_scale, b_codes, b_sf, M, N, K, bias=None, out=None, stream=None) -> torch.Tensor:
+    """D[M][N] (BF16) = act_scale * e4m3(A) deq(B)^T + bias, on the tensor cores."""
+    d = _out_bf16(M, N, a_e4m3.device) if out is None else out
+    mxq_gemm_w4a8(a_e4m3, act_scale, b_codes, b_sf, M, N, K, bias, d.data_ptr(), d.stride(0), stream)
+    return d
+
+
+def linear_w4a4(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE_OCP, hadamard128: bool = False,
+                bias=None, stream=None) -> torch.Tensor:
+    """The quantized linear layer: dynamic MXFP4 quantisation of X, then the W4A4 GEMM."""
+    M, K = x.shape
+    q, sf = quantize_act(x, rule, hadamard128, stream=stream)
+    return gemm_w4a4(q, sf, w_codes, w_sf, M, N, K, 1.0, bias, stream=stream)
+
+
+def linear_w4a8(x: torch.Tensor, act_scale: float, w_codes, w_sf, N: int, bias=None, stream=None) -> torch.Tensor:
+    """The W4A8 layer: static FP8 quantisation of X, then the W4A8 GEMM."""
+    M, K = x.shape
+    q = quantize_act_fp8(x, act_scale, stream=stream)
+    return gemm_w4a8(q, act_scale, w_codes, w_sf, M, N, K, bias, stream=stream)

@@ -1,0 +1,108 @@
+"""Host-only checks of the C ABI: the library loads, exports exactly the entry points
+include/mxq.h declares, and rejects bad arguments before touching any device.
+No kernel is launched here."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from mxfp4_block_scaled_mxq_b200 import build, mxq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return mxq.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "mxq.h")).read()
+    return sorted(set(re.findall(r"MXQ_API\s+[\w\s\*]+?\b(mxq_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_bound_entry_points():
+    assert declared_functions() == sorted(mxq.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert isinstance(getattr(L, name), ctypes._CFuncPtr)
+
+
+def test_status_strings(L):
+    for code, name in mxq.STATUS_NAMES.items():
+        assert mxq.mxq_status_string(code) == name
+    assert mxq.mxq_status_string(99) == "MXQ_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("rows,K", [(1, 32), (128, 512), (130, 96), (32760, 5120), (32760, 13824), (3, 4064)])
+def test_sf_bytes_matches_oracle_layout(L, rows, K):
+    assert mxq.mxq_sf_bytes(rows, K) == oracle.sf_bytes(rows, K)
+
+
+def test_sf_bytes_rejects_bad_sizes(L):
+    assert mxq.mxq_sf_bytes(0, 32) == -1
+    assert mxq.mxq_sf_bytes(4, 33) == -1
+    assert mxq.mxq_sf_bytes(4, 0) == -1
+
+
+def _status(fn, *args):
+    return getattr(mxq.lib(), fn)(*args)
+
+
+FAKE = 1 << 20  # a 16-byte-aligned non-null value; never dereferenced (validation fails first)
+
+
+def test_quantize_validation_happens_before_any_launch(L):
+    INV, SHAPE, ALIGN = 1, 2, 3
+    q = lambda *a: L.mxq_quantize_act(*a)
+    assert q(None, 4, 32, 32, 0, 0, 0, 1.0, FAKE, FAKE, None) == INV          # null x
+    assert q(FAKE, 4, 32, 32, 0, 0, 0, 1.0, FAKE, None, None) == INV          # null sf for MXFP4
+    assert q(FAKE, 4, 32, 32, 0, 7, 0, 1.0, FAKE, FAKE, None) == INV          # bad rule
+    assert q(FAKE, 4, 32, 32, 9, 0, 0, 1.0, FAKE, FAKE, None) == INV          # bad format
+    assert q(FAKE, 0, 32, 32, 0, 0, 0, 1.0, FAKE, FAKE, None) == SHAPE        # M = 0
+    assert q(FAKE, 4, 48, 48, 0, 0, 0, 1.0, FAKE, FAKE, None) == SHAPE        # K % 32
+    assert q(FAKE, 4, 96, 96, 0, 0, 1, 1.0, FAKE, FAKE, None) == SHAPE        # hadamard needs K % 128
+    assert q(FAKE, 4, 64, 60, 0, 0, 0, 1.0, FAKE, FAKE, None) == ALIGN        # ldx < K
+    assert q(FAKE + 2, 4, 64, 64, 0, 0, 0, 1.0, FAKE, FAKE, None) == ALIGN    # misaligned x
+    assert q(FAKE, 4, 64, 64, 1, 0, 0, 1.0, FAKE, FAKE, None) == INV          # FP8 must not get sf
+    assert q(FAKE, 4, 64, 64, 1, 0, 0, 0.0, FAKE, None, None) == INV          # FP8 scale <= 0
+    assert q(FAKE, 4, 64, 64, 1, 0, 0, float("nan"), FAKE, None, None) == INV
+    assert q(FAKE, 4, 64, 64, 1, 1, 0, 1.0, FAKE, None, None) == INV          # FP8 with UOS rule
+    assert q(FAKE, 4, 64, 64, 1, 0, 1, 1.0, FAKE, None, None) == INV          # FP8 with hadamard
+
+
+def test_gemm_validation_happens_before_any_launch(L):
+    INV, SHAPE, ALIGN = 1, 2, 3
+    g4 = lambda *a: L.mxq_gemm_w4a4(*a)
+    ok = (FAKE, FAKE, FAKE, FAKE, 128, 256, 256, 1.0, None, FAKE, 256, None)
+    args = list(ok)
+    args[0] = None
+    assert g4(*args) == INV
+    args = list(ok); args[1] = None
+    assert g4(*args) == INV
+    args = list(ok); args[6] = 192
+    assert g4(*args) == SHAPE                                                # K % 128
+    args = list(ok); args[4] = 0
+    assert g4(*args) == SHAPE
+    args = list(ok); args[10] = 250
+    assert g4(*args) == ALIGN                                                # ldd < N
+    args = list(ok); args[9] = FAKE + 8
+    assert g4(*args) == ALIGN
+    args = list(ok); args[7] = float("inf")
+    assert g4(*args) == INV
+    g8 = lambda *a: L.mxq_gemm_w4a8(*a)
+    assert g8(FAKE, 0.0, FAKE, FAKE, 128, 256, 256, None, FAKE, 256, None) == INV
+    assert g8(FAKE, 1.0, FAKE + 16, FAKE, 128, 256, 256, None, FAKE, 256, None) == ALIGN  # B needs 32 B
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        mxq.quantize_act(torch.zeros(4, 32, dtype=torch.bfloat16))

@@ -1,0 +1,173 @@
+"""GPU parity of the quantized linear layer (quantiser + tcgen05 GEMM + epilogue)
+against the FP64 oracle on the oracle's own quantisation of the same BF16 inputs:
+max|D - y_ref| / max|y_ref| <= 5e-3.  Small shapes are compared in full; the
+full-size workloads on a deterministic row sample (first rows, last row, the ragged
+tail tile and rows spread across M) in the same launch configuration the benchmark
+times."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mxfp4_block_scaled_mxq_b200 import build, inputs, mxq
+from parity import GEMM_TOL, assert_status_clean, gemm_rel_err, oracle_w4a4, oracle_w4a8, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    mxq.lib()
+    yield
+    assert_status_clean()
+
+
+def run_w4a4(x, w, rule_a=mxq.MXQ_SCALE_OCP, hadamard=False, alpha=1.0, bias=None):
+    xd, wd = x.cuda(), w.cuda()
+    M, K = xd.shape
+    N = wd.shape[0]
+    wc, wsf = mxq.pack_weight(wd, mxq.MXQ_SCALE_OCP, hadamard)
+    q, sf = mxq.quantize_act(xd, rule_a, hadamard)
+    d = mxq.gemm_w4a4(q, sf, wc, wsf, M, N, K, alpha, None if bias is None else bias.cuda())
+    torch.cuda.synchronize()
+    return d
+
+
+def check_w4a4(x, w, rows=None, **kw):
+    M = x.shape[0]
+    rows = np.arange(M) if rows is None else rows
+    d = run_w4a4(x, w, **kw)
+    rule_a = kw.get("rule_a", mxq.MXQ_SCALE_OCP)
+    y = oracle_w4a4(x, w, rows, rule_a=rule_a, hadamard=kw.get("hadamard", False), alpha=kw.get("alpha", 1.0),
+                    bias=kw.get("bias"))
+    err = gemm_rel_err(d, rows, y)
+    assert err <= GEMM_TOL, err
+    return d, err
+
+
+def test_tiny_config():
+    x, w = inputs.tiny(seed=0)
+    check_w4a4(x, w)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 256), (130, 200, 384), (257, 520, 128), (64, 1000, 640),
+                                   (300, 256, 1280)])
+def test_ragged_tiles(M, N, K):
+    """M and N not multiples of the 128 x 256 tile, K % 256 == 128 (half last stage)."""
+    x = inputs.heavy_tailed_bf16(M, K, seed=M)
+    w = inputs.normal_bf16(N, K, 0.02, seed=N)
+    check_w4a4(x, w)
+
+
+def test_bias_and_alpha():
+    x = inputs.normal_bf16(200, 512, 1.0, seed=1)
+    w = inputs.normal_bf16(300, 512, 0.02, seed=2)
+    bias = (torch.randn(300, generator=torch.Generator().manual_seed(3)) * 0.5).to(torch.bfloat16)
+    check_w4a4(x, w, alpha=0.37, bias=bias)
+
+
+def test_adversarial_scales_gemm_only():
+    """Random codes with scale bytes over a wide range, fed straight to the GEMM."""
+    rng = np.random.default_rng(9)
+    M, N, K = 192, 320, 512
+    a_codes = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    b_codes = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    a_sl = rng.integers(100, 150, (M, K // 32), dtype=np.uint8)
+    b_sl = rng.integers(100, 150, (N, K // 32), dtype=np.uint8)
+    a_sf, b_sf = oracle.sf_swizzle(a_sl, M, K), oracle.sf_swizzle(b_sl, N, K)
+    y = oracle.gemm(a_codes, a_sf, b_codes, b_sf, M, N, K)
+    t = lambda a: torch.from_numpy(a).cuda()
+    d = mxq.gemm_w4a4(t(a_codes), t(a_sf), t(b_codes), t(b_sf), M, N, K)
+    torch.cuda.synchronize()
+    assert gemm_rel_err(d, np.arange(M), y) <= GEMM_TOL
+
+
+@pytest.mark.parametrize("rule", [mxq.MXQ_SCALE_OCP, mxq.MXQ_SCALE_UOS])
+def test_hadamard_rotated_layer(rule):
+    x, ws = inputs.wan_attn(M=700)
+    check_w4a4(x, ws[0][:640], rule_a=rule, hadamard=True)
+
+
+def test_rotation_preserves_the_product():
+    """X R (W R)^T approximates X W^T about as well as the unrotated layer does."""
+    x, ws = inputs.wan_attn(M=256)
+    w = ws[1][:512]
+    ref = x.double() @ w.double().T
+    plain = run_w4a4(x, w).cpu().double()
+    rot = run_w4a4(x, w, hadamard=True).cpu().double()
+    e_plain = (plain - ref).norm() / ref.norm()
+    e_rot = (rot - ref).norm() / ref.norm()
+    assert e_rot < 0.3 and e_plain < 0.3
+
+
+def test_w4a8_small():
+    x, w, x_cal = inputs.flux_w4a8(M=300)
+    w = w[:520]
+    s = inputs.static_fp8_scale(x_cal)
+    xd, wd = x.cuda(), w.cuda()
+    wc, wsf = mxq.pack_weight(wd)
+    d = mxq.linear_w4a8(xd, s, wc, wsf, w.shape[0])
+    torch.cuda.synchronize()
+    rows = np.arange(x.shape[0])
+    y = oracle_w4a8(x, w, s, rows)
+    assert gemm_rel_err(d, rows, y) <= GEMM_TOL
+
+
+def test_w4a8_bias():
+    x, w, x_cal = inputs.flux_w4a8(M=130)
+    w = w[:300]
+    s = inputs.static_fp8_scale(x_cal)
+    bias = (torch.randn(300, generator=torch.Generator().manual_seed(5))).to(torch.bfloat16)
+    wc, wsf = mxq.pack_weight(w.cuda())
+    d = mxq.linear_w4a8(x.cuda(), s, wc, wsf, 300, bias=bias.cuda())
+    torch.cuda.synchronize()
+    rows = np.arange(130)
+    assert gemm_rel_err(d, rows, oracle_w4a8(x, w, s, rows, bias=bias)) <= GEMM_TOL
+
+
+@pytest.mark.parametrize("M", [16, 64, 256, 1024])
+def test_m_sweep_small(M):
+    x, w = inputs.m_sweep(M, device="cuda")
+    check_w4a4(x.cpu(), w.cpu(), rows=sample_rows(M, 256))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("which", ["up", "down"])
+def test_full_size_wan_ffn(which):
+    x, w = inputs.wan_ffn(which=which, device="cuda")
+    rows = sample_rows(x.shape[0], 96)
+    d = run_w4a4(x, w)
+    y = oracle_w4a4(x, w, rows)
+    assert gemm_rel_err(d, rows, y) <= GEMM_TOL
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("which", ["qkv", "mlp"])
+def test_full_size_flux_w4a8(which):
+    x, w, x_cal = inputs.flux_w4a8(which=which, device="cuda")
+    s = inputs.static_fp8_scale(x_cal)
+    wc, wsf = mxq.pack_weight(w)
+    d = mxq.linear_w4a8(x, s, wc, wsf, w.shape[0])
+    torch.cuda.synchronize()
+    rows = sample_rows(x.shape[0], 128)
+    assert gemm_rel_err(d, rows, oracle_w4a8(x, w, s, rows)) <= GEMM_TOL
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("rule", [mxq.MXQ_SCALE_OCP, mxq.MXQ_SCALE_UOS])
+def test_full_size_hadamard_projection(rule):
+    x, ws = inputs.wan_attn(device="cuda")
+    rows = sample_rows(x.shape[0], 96)
+    d = run_w4a4(x, ws[2], rule_a=rule, hadamard=True)
+    y = oracle_w4a4(x, ws[2], rows, rule_a=rule, hadamard=True)
+    assert gemm_rel_err(d, rows, y) <= GEMM_TOL
+
+
+@pytest.mark.slow
+def test_m_sweep_largest():
+    x, w = inputs.m_sweep(65536, device="cuda")
+    rows = sample_rows(65536, 64)
+    d = run_w4a4(x, w)
+    assert gemm_rel_err(d, rows, oracle_w4a4(x, w, rows)) <= GEMM_TOL

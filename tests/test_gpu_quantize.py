@@ -1,0 +1,132 @@
+"""GPU parity of the quantisers: codes and E8M0 scales must equal the oracle's bit
+for bit, over the whole physical scale buffer (padding included)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mxfp4_block_scaled_mxq_b200 import build, inputs, mxq
+from parity import assert_status_clean
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    mxq.lib()
+    yield
+    assert_status_clean()
+
+
+def _check_mxfp4(x: torch.Tensor, rule=mxq.MXQ_SCALE_OCP, hadamard=False, weight=False, rows=None):
+    xd = x.cuda()
+    if weight:
+        q, sf = mxq.pack_weight(xd, rule, hadamard)
+    else:
+        q, sf = mxq.quantize_act(xd, rule, hadamard)
+    torch.cuda.synchronize()
+    M, K = x.shape
+    q = q.cpu().numpy()
+    sf = sf.cpu().numpy()
+    if rows is None:
+        want_q, want_sl = oracle.quantize_mxfp4(x.cpu(), rule=rule, hadamard=hadamard)
+        np.testing.assert_array_equal(q, want_q)
+        np.testing.assert_array_equal(sf, oracle.sf_swizzle(want_sl, M, K))
+    else:
+        want_q, want_sl = oracle.quantize_mxfp4(x.cpu()[torch.as_tensor(rows)], rule=rule, hadamard=hadamard)
+        np.testing.assert_array_equal(q[rows], want_q)
+        got_sl = oracle.sf_unswizzle(sf, M, K)
+        np.testing.assert_array_equal(got_sl[rows], want_sl)
+
+
+def _all_finite_bf16(perm_seed=None) -> torch.Tensor:
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    finite = bits[((bits >> 7) & 0xFF) != 0xFF].astype(np.uint16)
+    if perm_seed is not None:
+        finite = np.random.default_rng(perm_seed).permutation(finite)
+    n = finite.size // 128 * 128
+    t = torch.from_numpy(finite[:n].astype(np.int16)).view(torch.bfloat16)
+    return t.reshape(-1, 128)
+
+
+@pytest.mark.parametrize("rule", [mxq.MXQ_SCALE_OCP, mxq.MXQ_SCALE_UOS])
+def test_every_bf16_value(rule):
+    _check_mxfp4(_all_finite_bf16(), rule)           # blocks of neighbouring bit patterns
+    _check_mxfp4(_all_finite_bf16(perm_seed=1), rule)  # the same values under other block scales
+
+
+def test_tiny_config_ocp():
+    x, w = inputs.tiny(seed=0)
+    _check_mxfp4(x)
+    _check_mxfp4(w, weight=True)
+
+
+def test_edge_blocks():
+    K = 256
+    x = torch.zeros(9, K)
+    x[1, :32] = -0.0
+    x[2, :32] = torch.tensor(np.float32(1e-40))            # FP32/BF16 subnormal block
+    x[3, :32] = 1.0
+    x[3, 7] = 7.25                                          # UOS tie
+    x[4, :32] = -8.0
+    x[5, 0] = 3.3895313892515355e38                         # BF16 max
+    x[5, 32] = -3.3895313892515355e38
+    x[6, :32] = 5.0
+    x[6, 0] = 7.0
+    x[7, :] = torch.linspace(-7.5, 7.5, K)
+    x[8, 64:96] = torch.tensor([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0] * 4)
+    xb = x.to(torch.bfloat16)
+    for rule in (mxq.MXQ_SCALE_OCP, mxq.MXQ_SCALE_UOS):
+        for had in (False, True):
+            _check_mxfp4(xb, rule, had)
+
+
+@pytest.mark.parametrize("M,K", [(1, 32), (7, 96), (130, 160), (129, 384), (300, 4064)])
+def test_ragged_shapes(M, K):
+    x = inputs.heavy_tailed_bf16(M, K, seed=M + K)
+    _check_mxfp4(x, mxq.MXQ_SCALE_OCP)
+    _check_mxfp4(x, mxq.MXQ_SCALE_UOS, weight=True)
+
+
+def test_leading_dimension():
+    full = inputs.normal_bf16(70, 320, 1.0, seed=3).cuda()
+    view = full[:, 64:320]        # ldx = 320, K = 256
+    q, sf = torch.empty(70, 128, dtype=torch.uint8, device="cuda"), torch.empty(mxq.mxq_sf_bytes(70, 256), dtype=torch.uint8, device="cuda")
+    mxq.mxq_quantize_act(view.data_ptr(), 70, 256, 320, mxq.MXQ_ACT_MXFP4, mxq.MXQ_SCALE_OCP, 0, 1.0, q, sf)
+    want_q, want_sl = oracle.quantize_mxfp4(full.cpu()[:, 64:].contiguous())
+    np.testing.assert_array_equal(q.cpu().numpy(), want_q)
+    np.testing.assert_array_equal(sf.cpu().numpy(), oracle.sf_swizzle(want_sl, 70, 256))
+
+
+@pytest.mark.parametrize("rule", [mxq.MXQ_SCALE_OCP, mxq.MXQ_SCALE_UOS])
+def test_hadamard_attention_activations(rule):
+    x, ws = inputs.wan_attn(M=1000)
+    _check_mxfp4(x, rule, hadamard=True)
+    _check_mxfp4(ws[0][:300], mxq.MXQ_SCALE_OCP, hadamard=True, weight=True)
+
+
+def test_fp8_static_activations():
+    x, _, x_cal = inputs.flux_w4a8(M=512)
+    s = inputs.static_fp8_scale(x_cal)
+    q = mxq.quantize_act_fp8(x.cuda(), s)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(q.cpu().numpy(), oracle.quantize_fp8(x, s))
+    # out-of-calibration values saturate, signs and zeros are kept
+    y = torch.tensor([[0.0, -0.0, 1e-30, -1e-30, 1e6, -1e6, 448.0, 3.0] * 4], dtype=torch.bfloat16)
+    q = mxq.quantize_act_fp8(y.cuda(), 1.0)
+    np.testing.assert_array_equal(q.cpu().numpy(), oracle.quantize_fp8(y, 1.0))
+
+
+@pytest.mark.slow
+def test_full_size_wan_ffn_up_activations():
+    x, _ = inputs.wan_ffn(which="up", device="cuda")
+    _check_mxfp4(x.cpu(), mxq.MXQ_SCALE_OCP)
+
+
+@pytest.mark.slow
+def test_full_size_wan_ffn_down_sampled_rows():
+    x, _ = inputs.wan_ffn(which="down", device="cuda")
+    from parity import sample_rows
+    _check_mxfp4(x.cpu(), mxq.MXQ_SCALE_OCP, rows=sample_rows(x.shape[0], 512))
