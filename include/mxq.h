@@ -106,9 +106,9 @@ MXQ_API int64_t mxq_sf_bytes(int64_t rows, int64_t K);
  *   Writes q_out ([M][K] bytes); sf_out must be NULL; rule and hadamard128 must be
  *   MXQ_SCALE_OCP and 0.
  *
- * x_bf16: device [M][ldx] BF16; 1 <= M <= 8388480 (65535 tiles of 128 rows; FP8 mode
- * allows up to 2^31); 32 <= K <= 2^22 with K % 32 == 0 (K % 128 == 0 when hadamard128);
- * ldx >= K and ldx % 8 == 0.
+ * x_bf16: device [M][ldx] BF16, 32-byte aligned; 1 <= M <= 8388480 (65535 tiles of 128
+ * rows; FP8 mode allows up to 2^31); 32 <= K <= 2^22 with K % 32 == 0 (K % 128 == 0 when
+ * hadamard128); ldx >= K and ldx % 16 == 0 (32-byte aligned rows).
  * Errors: MXQ_ERR_INVALID_ARG, MXQ_ERR_SHAPE, MXQ_ERR_ALIGN, MXQ_ERR_CUDA.
  */
 MXQ_API mxq_status mxq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
@@ -122,8 +122,8 @@ MXQ_API mxq_status mxq_quantize_act(const void* x_bf16, int64_t M, int64_t K, in
  * codes_out [N][K/2], sf_out mxq_sf_bytes(N, K) bytes.  Use rule = MXQ_SCALE_OCP for
  * "OCP MXFP4 weights"; hadamard128 must equal the activation side's setting (the
  * library cannot check this: X R (W R)^T = X W^T only when both sides rotate).
- * w_bf16: device [N][ldw] BF16, 1 <= N <= 8388480, 32 <= K <= 2^22, K % 32 == 0
- * (K % 128 == 0 when hadamard128), ldw >= K, ldw % 8 == 0.
+ * w_bf16: device [N][ldw] BF16, 32-byte aligned, 1 <= N <= 8388480, 32 <= K <= 2^22,
+ * K % 32 == 0 (K % 128 == 0 when hadamard128), ldw >= K, ldw % 16 == 0.
  */
 MXQ_API mxq_status mxq_pack_weight(const void* w_bf16, int64_t N, int64_t K, int64_t ldw,
                            mxq_scale_rule rule, int hadamard128, void* codes_out, void* sf_out,

@@ -10,6 +10,7 @@
 
 #include "mxq.h"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "quantize.cuh"
 
 namespace {
@@ -77,12 +78,73 @@ bool make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D tensor map over a swizzled scale-factor buffer of `rows` rows and K columns:
+// (byte in 128-byte chunk, chunk in atom, atom along K, 128-row tile); a box of
+// {128, 4, atoms, row_tiles} lands as contiguous 512-byte atoms, [row tile][atom].
+bool make_tmap_sf(CUtensorMap* m, const void* base, int64_t rows, int64_t K, uint32_t atoms, uint32_t row_tiles) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return false;
+  const uint64_t atoms_per_row_tile = static_cast<uint64_t>(K) / 128;
+  const cuuint64_t dims[4] = {128, 4, atoms_per_row_tile, static_cast<cuuint64_t>((rows + 127) / 128)};
+  const cuuint64_t strides[3] = {128, 512, atoms_per_row_tile * 512};
+  const cuuint32_t box[4] = {128, 4, atoms, row_tiles};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Two-CTA path (one 256 x 256 tile per CTA pair), persistent over as many pairs as
+// can be resident at once.
+template <bool kW4A8>
+mxq_status launch_gemm_pair(const void* a, const void* a_sf, const void* b, const void* b_sf, int64_t M, int64_t N,
+                            int64_t K, float alpha, const void* bias, void* d, int64_t ldd, cudaStream_t stream) {
+  using S = mxq::PairShape<kW4A8>;
+  auto kernel = mxq::mx_gemm_pair_kernel<kW4A8>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  static int max_clusters = 0;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
+    if (attr_err != cudaSuccess) return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(mxq::kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = S::kSmemBytes;
+    attr_err = cudaOccupancyMaxActiveClusters(&max_clusters, kernel, &cfg);
+  });
+  if (attr_err != cudaSuccess || max_clusters < 1) return MXQ_ERR_CUDA;
+
+  CUtensorMap ta, tb, tsa, tsb, td;
+  bool ok;
+  if (kW4A8) {
+    ok = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K, M, K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, b, K, N, K / 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    tsa = tb;  // unused: E4M3 activations carry unit scales
+  } else {
+    ok = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K / 2, M, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K / 2, N, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_tmap_sf(&tsa, a_sf, M, K, S::kAtoms, 1);
+  }
+  ok = ok && make_tmap_sf(&tsb, b_sf, N, K, S::kAtoms, 2) &&
+       make_tmap_2d(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, N, M, ldd * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (!ok) return MXQ_ERR_CUDA;
+  const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  const int clusters = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
+  kernel<<<2 * clusters, mxq::kGemmThreads, S::kSmemBytes, stream>>>(
+      ta, tb, tsa, tsb, td, static_cast<const __nv_bfloat16*>(bias), static_cast<int>(M), static_cast<int>(N),
+      static_cast<int>(K), alpha);
+  return launch_status();
+}
+
 template <bool kW4A8>
 mxq_status launch_gemm(const void* a, const void* a_sf, const void* b, const void* b_sf, int64_t M, int64_t N,
                        int64_t K, float alpha, const void* bias, void* d, int64_t ldd, cudaStream_t stream) {
   DeviceInfo dev;
   mxq_status st = current_device(&dev);
   if (st != MXQ_OK) return st;
+  if (M > mxq::kBM) return launch_gemm_pair<kW4A8>(a, a_sf, b, b_sf, M, N, K, alpha, bias, d, ldd, stream);
   CUtensorMap ta, tb, td;
   bool ok;
   if (kW4A8) {
@@ -161,8 +223,9 @@ mxq_status check_quant_args(const void* x, int64_t rows, int64_t K, int64_t ld, 
   // rows <= 65535 * 128 keeps grid.y within its limit
   if (rows < 1 || rows > int64_t(65535) * 128 || K < 32 || K % 32 != 0 || K > (int64_t(1) << 22)) return MXQ_ERR_SHAPE;
   if (hadamard && K % 128 != 0) return MXQ_ERR_SHAPE;
-  if (ld < K || ld % 8 != 0) return MXQ_ERR_ALIGN;
-  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(sf, 16)) return MXQ_ERR_ALIGN;
+  // 32-byte loads of 16 BF16 values: 32-byte aligned rows
+  if (ld < K || ld % 16 != 0) return MXQ_ERR_ALIGN;
+  if (!aligned(x, 32) || !aligned(q, 16) || !aligned(sf, 16)) return MXQ_ERR_ALIGN;
   return MXQ_OK;
 }
 
@@ -196,14 +259,14 @@ mxq_status mxq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ld
     if (rule != MXQ_SCALE_OCP || hadamard128) return MXQ_ERR_INVALID_ARG;
     if (!(act_scale > 0.f) || !std::isfinite(act_scale)) return MXQ_ERR_INVALID_ARG;
     if (M < 1 || M > (int64_t(1) << 31) || K < 32 || K % 32 != 0 || K > (int64_t(1) << 22)) return MXQ_ERR_SHAPE;
-    if (ldx < K || ldx % 8 != 0) return MXQ_ERR_ALIGN;
-    if (!aligned(x_bf16, 16) || !aligned(q_out, 16)) return MXQ_ERR_ALIGN;
+    if (ldx < K || ldx % 16 != 0) return MXQ_ERR_ALIGN;
+    if (!aligned(x_bf16, 32) || !aligned(q_out, 16)) return MXQ_ERR_ALIGN;
     const float inv = 1.0f / act_scale;  // fl32(1 / s), IEEE division on the host
     if (!std::isfinite(inv)) return MXQ_ERR_INVALID_ARG;
     DeviceInfo dev;
     mxq_status st = current_device(&dev);
     if (st != MXQ_OK) return st;
-    const int64_t chunks = M * (K / 8);
+    const int64_t chunks = M * (K / 16);
     int64_t blocks = (chunks + mxq::kQuantThreads - 1) / mxq::kQuantThreads;
     const int64_t cap = static_cast<int64_t>(dev.sm_count) * 16;
     if (blocks > cap) blocks = cap;

@@ -11,12 +11,15 @@
 // native W4A8 ... Wan2.2 -- "MXFP4 formats and precision levels"]; the rotation is
 // the fixed, parameter-free Hadamard of the same page ("Fixed rotation selector").
 //
-// The pass is bound by HBM bandwidth (2 bytes in, 0.53 bytes out per element), so the
-// design is about bytes in flight: each thread issues eight 16-byte loads before it
-// computes anything, loads are fully coalesced (a warp reads 2 rows x 256 bytes per
-// instruction), and the block scales of a 128 x 128 tile are assembled in shared
-// memory and leave as one 512-byte atom.
+// The pass is bound by HBM bandwidth (2 bytes in, 0.53 bytes out per element) as long
+// as it issues few enough instructions per element, so each thread owns 16
+// consecutive elements (one 32-byte load; a warp reads 1 KB per instruction), the
+// non-rotated path takes the block amax on packed BF16 pairs, a 32-element block
+// spans two lanes (one shuffle), and each block's scale byte goes straight into the
+// CTA's 512-byte scale atom in shared memory, which leaves as one coalesced write.
 #pragma once
+
+#include <cuda_bf16.h>
 
 #include <cstdint>
 
@@ -24,20 +27,21 @@
 
 namespace mxq {
 
-constexpr int kQuantThreads = 256;   // 8 warps; a CTA owns 128 rows x 128 K columns
+constexpr int kQuantThreads = 256;                 // 8 warps; a CTA owns 128 rows x 128 K columns
 constexpr uint32_t kInvSqrt128Bits = 0x3DB504F3u;  // fl32(1 / sqrt(128))
 
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+__device__ __forceinline__ void ld_stream_v8(const void* p, uint32_t (&w)[8]) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
                : "l"(p));
-  return v;
 }
 
-// Two non-negative floats -> one byte of two E2M1 magnitudes (round to nearest even,
-// saturating at 6): `lo` in bits 0-3, `hi` in bits 4-7.
-__device__ __forceinline__ uint32_t e2m1x2_magnitude(float lo, float hi) {
+// Two floats -> one byte of two E2M1 codes (round to nearest even, saturating at 6):
+// `lo` in bits 0-3, `hi` in bits 4-7.  The conversion keeps the sign bit of its input
+// in bit 3 of each code, also for -0 and for negative values that round to zero
+// (0x8) -- the sign rule of the format as defined here; the exhaustive BF16 parity
+// tests check this against the oracle.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
   uint32_t out;
   asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
       : "=r"(out)
@@ -45,9 +49,9 @@ __device__ __forceinline__ uint32_t e2m1x2_magnitude(float lo, float hi) {
   return out;
 }
 
-// Two non-negative floats -> two E4M3 magnitudes (RNE, saturating at 448): `lo` in
-// bits 0-7, `hi` in bits 8-15.
-__device__ __forceinline__ uint32_t e4m3x2_magnitude(float lo, float hi) {
+// Two floats -> two E4M3 codes (RNE, saturating at 448, sign kept): `lo` in bits 0-7,
+// `hi` in bits 8-15.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   uint32_t out;
   asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\tcvt.u32.u16 %0, t;\n\t}"
       : "=r"(out)
@@ -55,41 +59,61 @@ __device__ __forceinline__ uint32_t e4m3x2_magnitude(float lo, float hi) {
   return out;
 }
 
-__device__ __forceinline__ void bf16x8_to_float(const uint4& v, float (&f)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+__device__ __forceinline__ void bf16x16_to_float(const uint32_t (&w)[8], float (&f)[16]) {
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < 8; ++j) {
     f[2 * j] = __uint_as_float(w[j] << 16);
     f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
   }
+}
+
+// Largest |x| over 16 BF16 values held as 8 packed pairs, as FP32 bits (exact).
+// Magnitudes are compared with the packed BF16 max; non-negative BF16 patterns order
+// like unsigned integers, which combines the two halves.
+__device__ __forceinline__ uint32_t bf16x16_absmax(const uint32_t (&w)[8]) {
+  uint32_t t = w[0] & 0x7FFF7FFFu;
+  __nv_bfloat162 m = *reinterpret_cast<const __nv_bfloat162*>(&t);
+#pragma unroll
+  for (int j = 1; j < 8; ++j) {
+    const uint32_t a = w[j] & 0x7FFF7FFFu;
+    m = __hmax2(m, *reinterpret_cast<const __nv_bfloat162*>(&a));
+  }
+  const uint32_t mb = *reinterpret_cast<const uint32_t*>(&m);
+  return max(mb & 0xFFFFu, mb >> 16) << 16;
 }
 
 // Block exponent from the block's absolute maximum (integer arithmetic on the FP32
 // bit pattern, no log2).  OCP: floor(log2 amax) - 2.  UOS: one more when the
 // significand exceeds 1.8125 = 7.25 / 4, i.e. amax > 7.25 * 2^(OCP exponent);
 // biased exponents 0 and 1 give an OCP exponent below -127, which clamps to -127
-// where amax <= 7.25 * 2^-127 always holds, so they never bump.
+// where amax <= 7.25 * 2^-127 always holds, so they never bump.  A non-finite amax
+// (an FP32 overflow inside the rotation of finite BF16 inputs) satisfies neither
+// rule for any e, and takes the largest exponent, 127.
 template <bool kUOS>
-__device__ __forceinline__ int block_exponent(float amax) {
-  const uint32_t bits = __float_as_uint(amax);
-  const int biased = static_cast<int>(bits >> 23);  // amax >= 0
+__device__ __forceinline__ int block_exponent(uint32_t amax_bits) {
+  const int biased = static_cast<int>(amax_bits >> 23);  // amax >= 0
+  if (biased == 255) return 127;
   int e = biased - 127 - 2;
-  if (kUOS && biased >= 2 && (bits & 0x7FFFFFu) > 0x680000u) e += 1;
-  e = e < -127 ? -127 : e;
-  e = e > 126 ? 126 : e;  // only non-finite input (out of contract) reaches 126+
-  return e;
+  if (kUOS && biased >= 2 && (amax_bits & 0x7FFFFFu) > 0x680000u) e += 1;
+  return e < -127 ? -127 : e;  // a finite amax gives e <= 126
 }
 
-// 128-point normalised Sylvester-Hadamard across the 16 lanes of a half-warp, each
-// lane holding 8 consecutive elements (element j = 8 * (lane % 16) + i).  Butterfly
-// strides 1, 2, 4 inside the thread, then 8, 16, 32, 64 across lanes (xor 1, 2, 4, 8),
-// each stage (t_i, t_i+h) <- (t_i + t_i+h, t_i - t_i+h) in FP32 round-to-nearest, then
-// one multiply by fl32(1/sqrt(128)) -- the exact order of the definition.
-__device__ __forceinline__ void fwht128_halfwarp(float (&f)[8], int l16) {
+// 2^-e for e in [-127, 127]: a normal float down to 2^-126, the subnormal 2^-127 at e = 127.
+__device__ __forceinline__ float exp2_neg(int e) {
+  return e < 127 ? __uint_as_float(static_cast<uint32_t>(127 - e) << 23) : __uint_as_float(0x00400000u);
+}
+
+// 128-point normalised Sylvester-Hadamard across 8 consecutive lanes, each holding 16
+// consecutive elements (element j = 16 * (lane % 8) + i).  Butterfly strides 1, 2, 4,
+// 8 inside the thread, then 16, 32, 64 across lanes (xor 1, 2, 4); every stage is
+// (t_i, t_i+h) <- (t_i + t_i+h, t_i - t_i+h) in FP32 round-to-nearest, then one
+// multiply by fl32(1/sqrt(128)) -- the order of the definition, so the result is
+// bit-identical to the element-by-element butterfly.
+__device__ __forceinline__ void fwht128_8lanes(float (&f)[16], int l8) {
 #pragma unroll
-  for (int h = 1; h < 8; h *= 2) {
+  for (int h = 1; h < 16; h *= 2) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 16; ++i) {
       if (i & h) continue;
       const float a = f[i], b = f[i + h];
       f[i] = __fadd_rn(a, b);
@@ -97,85 +121,89 @@ __device__ __forceinline__ void fwht128_halfwarp(float (&f)[8], int l16) {
     }
   }
 #pragma unroll
-  for (int bit = 0; bit < 4; ++bit) {
-    const bool upper = (l16 >> bit) & 1;
+  for (int bit = 0; bit < 3; ++bit) {
+    const bool upper = (l8 >> bit) & 1;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 16; ++i) {
       const float p = __shfl_xor_sync(0xffffffffu, f[i], 1 << bit);
       f[i] = upper ? __fsub_rn(p, f[i]) : __fadd_rn(f[i], p);
     }
   }
   const float c = __uint_as_float(kInvSqrt128Bits);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) f[i] = __fmul_rn(f[i], c);
+  for (int i = 0; i < 16; ++i) f[i] = __fmul_rn(f[i], c);
 }
 
 // One CTA quantises rows [128*by, +128) x K columns [128*bx, +128) of x[rows][ld]:
-// codes [rows][K/2], and the CTA's 512-byte scale atom (rows beyond `rows`, and
-// blocks beyond K, are written as 0x00 padding).
+// codes [rows][K/2] and the tile's 512-byte scale atom (rows beyond `rows` and blocks
+// beyond K stay 0x00 padding).  Thread (warp w, lane l) owns, in iteration i, row
+// 16w + 4i + l/8 and elements [16 * (l%8), +16) of the tile's 128 columns.
 template <bool kHadamard, bool kUOS>
 __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__ x, int64_t rows, int64_t K,
                                                     int64_t ld, uint8_t* __restrict__ codes,
                                                     uint8_t* __restrict__ sf) {
-  __shared__ __align__(16) uint32_t atom[128];  // u32 (r%32)*4 + r/32 holds blocks 0..3 of row r
+  __shared__ __align__(16) uint8_t atom[512];  // byte (r%32)*16 + (r/32)*4 + block
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int half = lane >> 4, l16 = lane & 15;
+  const int l8 = lane & 7;
   const int64_t row0 = static_cast<int64_t>(blockIdx.y) * 128;
-  const int64_t k = static_cast<int64_t>(blockIdx.x) * 128 + 8 * l16;
-  const bool k_ok = k < K;  // K % 32 == 0: a 32-block is entirely in or out
+  const int64_t k = static_cast<int64_t>(blockIdx.x) * 128 + 16 * l8;
+  const bool k_ok = k < K;  // K % 32 == 0: a 16-element chunk is entirely in or out
 
-  if (tid < 128) atom[tid] = 0u;
+  reinterpret_cast<uint32_t*>(atom)[tid & 127] = 0u;
 
-  uint4 v[8];
+  uint32_t w[4][8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int64_t row = row0 + 16 * warp + 2 * i + half;
-    v[i] = (row < rows && k_ok) ? ld_stream_v4(x + row * ld + k) : make_uint4(0, 0, 0, 0);
+  for (int i = 0; i < 4; ++i) {
+    const int64_t row = row0 + 16 * warp + 4 * i + (lane >> 3);
+    if (row < rows && k_ok) {
+      ld_stream_v8(x + row * ld + k, w[i]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) w[i][j] = 0u;
+    }
   }
   __syncthreads();  // atom zeroed
 
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = 16 * warp + 2 * i + half;  // row within the tile
+  for (int i = 0; i < 4; ++i) {
+    const int r = 16 * warp + 4 * i + (lane >> 3);  // row within the tile
     const int64_t row = row0 + r;
-    float f[8];
-    bf16x8_to_float(v[i], f);
-    if (kHadamard) fwht128_halfwarp(f, l16);
-
-    float amax = 0.f;
+    float f[16];
+    bf16x16_to_float(w[i], f);
+    uint32_t amax;
+    if (kHadamard) {
+      fwht128_8lanes(f, l8);
+      float m = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    const int e = block_exponent<kUOS>(amax);
-    const float inv_scale = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e, exact
-
-    uint32_t packed = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float a0 = f[2 * j], a1 = f[2 * j + 1];
-      uint32_t byte = e2m1x2_magnitude(__fmul_rn(fabsf(a0), inv_scale), __fmul_rn(fabsf(a1), inv_scale));
-      byte |= ((__float_as_uint(a0) >> 31) << 3) | ((__float_as_uint(a1) >> 31) << 7);
-      packed |= byte << (8 * j);
+      for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(f[j]));
+      amax = __float_as_uint(m);
+    } else {
+      amax = bf16x16_absmax(w[i]);
     }
-    if (row < rows && k_ok) *reinterpret_cast<uint32_t*>(codes + row * (K / 2) + k / 2) = packed;
+    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));  // the other half of the block
+    const int e = block_exponent<kUOS>(amax);
+    const float s = exp2_neg(e);  // exact power of two
 
-    // Scale bytes of this row's four blocks sit in lanes 0, 4, 8, 12 of the half-warp.
-    const uint32_t sbyte = (row < rows && k_ok) ? static_cast<uint32_t>(e + 127) : 0u;
-    const int base = lane & 16;
-    const uint32_t b0 = __shfl_sync(0xffffffffu, sbyte, base + 0);
-    const uint32_t b1 = __shfl_sync(0xffffffffu, sbyte, base + 4);
-    const uint32_t b2 = __shfl_sync(0xffffffffu, sbyte, base + 8);
-    const uint32_t b3 = __shfl_sync(0xffffffffu, sbyte, base + 12);
-    if (l16 == 0) atom[(r & 31) * 4 + (r >> 5)] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    uint32_t out[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint32_t packed = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        packed |= e2m1x2(__fmul_rn(f[8 * q + 2 * j], s), __fmul_rn(f[8 * q + 2 * j + 1], s)) << (8 * j);
+      out[q] = packed;
+    }
+    if (row < rows && k_ok) {
+      *reinterpret_cast<uint2*>(codes + row * (K / 2) + k / 2) = make_uint2(out[0], out[1]);
+      if ((l8 & 1) == 0) atom[(r & 31) * 16 + (r >> 5) * 4 + (l8 >> 1)] = static_cast<uint8_t>(e + 127);
+    }
   }
   __syncthreads();
   if (tid < 32) {
     const int64_t atoms_per_row_tile = (K + 127) / 128;
     const int64_t idx = static_cast<int64_t>(blockIdx.y) * atoms_per_row_tile + blockIdx.x;
-    const uint4 w = reinterpret_cast<const uint4*>(atom)[tid];
-    reinterpret_cast<uint4*>(sf + idx * 512)[tid] = w;
+    reinterpret_cast<uint4*>(sf + idx * 512)[tid] = reinterpret_cast<const uint4*>(atom)[tid];
   }
 }
 
@@ -195,33 +223,28 @@ __global__ void __launch_bounds__(kQuantThreads) pack_weight_mxfp4_kernel(
 }
 
 // Static FP8: q = E4M3_RNE_satfinite(fl32(x * inv_scale)), sign bit kept.  Each thread
-// converts 8-element chunks (16 bytes in, 8 bytes out) in a grid-stride loop.
+// converts 16-element chunks (32 bytes in, 16 bytes out) in a grid-stride loop.
 __global__ void __launch_bounds__(kQuantThreads) quantize_act_fp8_kernel(const uint16_t* __restrict__ x, int64_t M,
                                                                           int64_t K, int64_t ldx, float inv_scale,
                                                                           uint8_t* __restrict__ q) {
-  const int64_t chunks_per_row = K / 8;
+  const int64_t chunks_per_row = K / 16;
   const int64_t total = M * chunks_per_row;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < total; c += stride) {
     const int64_t row = c / chunks_per_row;
-    const int64_t k = (c - row * chunks_per_row) * 8;
-    float f[8];
-    bf16x8_to_float(ld_stream_v4(x + row * ldx + k), f);
-    uint32_t w[2];
+    const int64_t k = (c - row * chunks_per_row) * 16;
+    uint32_t w[8];
+    ld_stream_v8(x + row * ldx + k, w);
+    float f[16];
+    bf16x16_to_float(w, f);
+    uint32_t o[4];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      uint32_t out = 0;
-#pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        const float a0 = __fmul_rn(f[4 * j + 2 * p], inv_scale);
-        const float a1 = __fmul_rn(f[4 * j + 2 * p + 1], inv_scale);
-        uint32_t two = e4m3x2_magnitude(fabsf(a0), fabsf(a1));
-        two |= ((__float_as_uint(a0) >> 31) << 7) | ((__float_as_uint(a1) >> 31) << 15);
-        out |= two << (16 * p);
-      }
-      w[j] = out;
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t lo = e4m3x2(__fmul_rn(f[4 * j], inv_scale), __fmul_rn(f[4 * j + 1], inv_scale));
+      const uint32_t hi = e4m3x2(__fmul_rn(f[4 * j + 2], inv_scale), __fmul_rn(f[4 * j + 3], inv_scale));
+      o[j] = lo | (hi << 16);
     }
-    *reinterpret_cast<uint2*>(q + row * K + k) = make_uint2(w[0], w[1]);
+    *reinterpret_cast<uint4*>(q + row * K + k) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 

@@ -71,6 +71,8 @@ def test_quantize_validation_happens_before_any_launch(L):
     assert q(FAKE, 4, 96, 96, 0, 0, 1, 1.0, FAKE, FAKE, None) == SHAPE        # hadamard needs K % 128
     assert q(FAKE, 4, 64, 60, 0, 0, 0, 1.0, FAKE, FAKE, None) == ALIGN        # ldx < K
     assert q(FAKE + 2, 4, 64, 64, 0, 0, 0, 1.0, FAKE, FAKE, None) == ALIGN    # misaligned x
+    assert q(FAKE + 16, 4, 64, 64, 0, 0, 0, 1.0, FAKE, FAKE, None) == ALIGN   # x needs 32 bytes
+    assert q(FAKE, 4, 64, 72, 0, 0, 0, 1.0, FAKE, FAKE, None) == ALIGN        # ldx % 16
     assert q(FAKE, 4, 64, 64, 1, 0, 0, 1.0, FAKE, FAKE, None) == INV          # FP8 must not get sf
     assert q(FAKE, 4, 64, 64, 1, 0, 0, 0.0, FAKE, None, None) == INV          # FP8 scale <= 0
     assert q(FAKE, 4, 64, 64, 1, 0, 0, float("nan"), FAKE, None, None) == INV

@@ -61,6 +61,28 @@ def test_ragged_tiles(M, N, K):
     check_w4a4(x, w)
 
 
+@pytest.mark.parametrize("M,N,K", [(129, 384, 384), (256, 128, 256), (257, 136, 640), (511, 264, 128),
+                                   (384, 512, 1152)])
+def test_cta_pair_edges(M, N, K):
+    """Shapes for the two-CTA path (M > 128): a nearly empty second CTA, B tiles whose
+    second half is missing or ragged, a half last K stage, exact multiples."""
+    x = inputs.heavy_tailed_bf16(M, K, seed=M + 7)
+    w = inputs.normal_bf16(N, K, 0.02, seed=N + 7)
+    check_w4a4(x, w)
+
+
+def test_w4a8_cta_pair_edges():
+    x, w, x_cal = inputs.flux_w4a8(M=129)
+    w = w[:136, :384].contiguous()
+    x = x[:, :384].contiguous()
+    s = inputs.static_fp8_scale(x_cal)
+    wc, wsf = mxq.pack_weight(w.cuda())
+    d = mxq.linear_w4a8(x.cuda(), s, wc, wsf, 136)
+    torch.cuda.synchronize()
+    rows = np.arange(129)
+    assert gemm_rel_err(d, rows, oracle_w4a8(x, w, s, rows)) <= GEMM_TOL
+
+
 def test_bias_and_alpha():
     x = inputs.normal_bf16(200, 512, 1.0, seed=1)
     w = inputs.normal_bf16(300, 512, 0.02, seed=2)
