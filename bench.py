@@ -31,9 +31,15 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MXFP4 W4A4 GEMM TFLOPS incl. act-quant and % of B200 dense FP4 peak"
+METRIC_W4A8 = "MXFP4 W4A8 GEMM TFLOPS incl. act-quant and % of B200 dense FP8 peak"
 UNIT = "TFLOP/s"
 NOMINAL_FP4_TFLOPS = 9000.0          # dense FP4, nominal
+NOMINAL_FP8_TFLOPS = 4500.0          # dense FP8, nominal (kind::mxf8f6f4 runs at the FP8 rate)
 FP4_PER_BF16 = 4.0                   # nominal FP4 : BF16 dense ratio (9 / 2.25 PFLOP/s)
+FP8_PER_BF16 = 2.0                   # nominal FP8 : BF16 dense ratio (4.5 / 2.25 PFLOP/s)
+# DRAM traffic per launch of the dominant kernel, from an ncu capture (see profiles/); None if
+# the kernel changed since the counters were taken.
+TRAFFIC = {}
 WORKLOAD = "Wan2.2-A14B FFN W4A4 (up 32760x5120->13824, down 32760x13824->5120), dynamic MXFP4 acts, OCP rule"
 M_TOK, D_MODEL, D_FF = 32760, 5120, 13824
 
@@ -41,13 +47,16 @@ M_TOK, D_MODEL, D_FF = 32760, 5120, 13824
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["mxq", "reference"], default="mxq")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=5)
-    p.add_argument("--m", type=int, default=M_TOK, help="token count (profiling of smaller cases)")
+    p.add_argument("--m", type=int, default=0, help="token count (0: the workload's own)")
+    p.add_argument("--workload", choices=["wan_ffn", "wan_attn_hadamard", "flux_w4a8", "m_sweep"],
+                   default="wan_ffn")
+    p.add_argument("--rule", choices=["ocp", "uos"], default="ocp", help="activation scale rule")
     return p.parse_args()
 
 
@@ -169,6 +178,101 @@ def run_reference(args, rank, world):
     }))
 
 
+# ------------------------------------------------------------------ workloads
+class Part:
+    """One kernel launch of the step: kind 'quant' (HBM-bound) or 'gemm' (tensor-bound)."""
+
+    def __init__(self, label, kind, fn, flops=0.0, nbytes=0.0, peak_kind="fp4"):
+        self.label, self.kind, self.fn, self.flops, self.nbytes, self.peak_kind = label, kind, fn, flops, nbytes, peak_kind
+
+
+def quant_bytes(M, K, fp8=False):
+    """Algorithmic bytes of one activation-quantiser launch: BF16 in, codes (+ scales) out."""
+    return M * K * 2 + (M * K if fp8 else M * K // 2 + M * K // 32)
+
+
+def build_workload(name, dev, M, seed, rule_name):
+    """Returns (description, parts, inputs [(device tensor)], outputs [(device tensor)], flops per step)."""
+    import torch
+    from mxfp4_block_scaled_mxq_b200 import inputs, mxq
+
+    rule = mxq.MXQ_SCALE_UOS if rule_name == "uos" else mxq.MXQ_SCALE_OCP
+
+    def qbufs(rows, K):
+        return (torch.empty(rows, K // 2, dtype=torch.uint8, device=dev),
+                torch.empty(mxq.mxq_sf_bytes(rows, K), dtype=torch.uint8, device=dev))
+
+    def out(rows, N):
+        return torch.empty(rows, N, dtype=torch.bfloat16, device=dev)
+
+    def w4a4_layer(label, x, w, hadamard, qb=None, share_quant=False):
+        """Parts for quantise(x) (unless shared) + GEMM against packed w."""
+        rows, K = x.shape
+        N = w.shape[0]
+        wc, wsf = mxq.pack_weight(w, mxq.MXQ_SCALE_OCP, hadamard)
+        qb = qb if qb is not None else qbufs(rows, K)
+        d = out(rows, N)
+        parts = []
+        if not share_quant:
+            parts.append(Part(f"quant_{label}", "quant",
+                              lambda: mxq.quantize_act(x, rule, hadamard, out=qb), nbytes=quant_bytes(rows, K)))
+        parts.append(Part(f"gemm_{label}", "gemm",
+                          lambda: mxq.gemm_w4a4(qb[0], qb[1], wc, wsf, rows, N, K, out=d),
+                          flops=2.0 * rows * N * K))
+        return parts, qb, d
+
+    if name == "wan_ffn":
+        x_up, w_up = inputs.wan_ffn(seed=seed, which="up", device=dev, M=M)
+        x_dn, w_dn = inputs.wan_ffn(seed=seed, which="down", device=dev, M=M)
+        p1, _, d1 = w4a4_layer("up", x_up, w_up, False)
+        p2, _, d2 = w4a4_layer("down", x_dn, w_dn, False)
+        rows = x_up.shape[0]
+        desc = WORKLOAD if rows == M_TOK else WORKLOAD.replace("32760", str(rows))
+        if rule_name == "uos":
+            desc = desc.replace("OCP rule", "UOS rule")
+        return desc, p1 + p2, [x_up, x_dn], [d1, d2], sum(p.flops for p in p1 + p2)
+
+    if name == "wan_attn_hadamard":
+        x, ws = inputs.wan_attn(seed=4000 + seed - 2000, device=dev, M=M)
+        x_o = inputs.heavy_tailed_bf16(x.shape[0], x.shape[1], seed + 77, device=dev)
+        pq, qb, dq = w4a4_layer("q", x, ws[0], True)
+        pk, _, dk = w4a4_layer("k", x, ws[1], True, qb=qb, share_quant=True)
+        pv, _, dv = w4a4_layer("v", x, ws[2], True, qb=qb, share_quant=True)
+        po, _, do = w4a4_layer("o", x_o, ws[3], True)
+        parts = pq + pk + pv + po
+        desc = (f"Wan2.2 attention projections W4A4 with 128-point block-Hadamard, Q/K/V/O "
+                f"{x.shape[0]}x5120->5120, {rule_name.upper()} rule")
+        return desc, parts, [x, x_o], [dq, dk, dv, do], sum(p.flops for p in parts)
+
+    if name == "flux_w4a8":
+        x, w_qkv, x_cal = inputs.flux_w4a8(which="qkv", device=dev, M=M)
+        _, w_mlp, _ = inputs.flux_w4a8(which="mlp", device=dev, M=M)
+        s = inputs.static_fp8_scale(x_cal)
+        rows, K = x.shape
+        q8 = torch.empty(rows, K, dtype=torch.uint8, device=dev)
+        parts = [Part("quant_fp8", "quant", lambda: mxq.quantize_act_fp8(x, s, out=q8),
+                      nbytes=quant_bytes(rows, K, fp8=True))]
+        outs = []
+        for label, w in (("qkv", w_qkv), ("mlp", w_mlp)):
+            wc, wsf = mxq.pack_weight(w)
+            d = out(rows, w.shape[0])
+            outs.append(d)
+            parts.append(Part(f"gemm_{label}", "gemm",
+                              (lambda wc=wc, wsf=wsf, N=w.shape[0], d=d:
+                               mxq.gemm_w4a8(q8, s, wc, wsf, rows, N, K, out=d)),
+                              flops=2.0 * rows * w.shape[0] * K, peak_kind="fp8"))
+        desc = f"FLUX.1-dev-shaped W4A8: M={rows}, QKV 3072->9216 and MLP 3072->12288, static FP8 E4M3 acts"
+        return desc, parts, [x], outs, sum(p.flops for p in parts)
+
+    if name == "m_sweep":
+        x, w = inputs.m_sweep(M, device=dev)
+        p, _, d = w4a4_layer("up", x, w, False)
+        desc = f"M sweep W4A4: M={M}, 5120->13824, N(0,1) acts"
+        return desc, p, [x], [d], sum(q.flops for q in p)
+
+    raise ValueError(f"unknown workload {name}")
+
+
 # ------------------------------------------------------------------ our arm
 def main():
     args = parse()
@@ -182,7 +286,7 @@ def main():
 
     import torch
     import torch.distributed as dist
-    from mxfp4_block_scaled_mxq_b200 import inputs, mxq
+    from mxfp4_block_scaled_mxq_b200 import mxq
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -191,36 +295,19 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     mxq.lib()
 
-    # Inputs (per rank its own token batch), weights packed once before timing.
-    seed = 2000 + 100 * rank
-    x_up, w_up = inputs.wan_ffn(seed=seed, which="up", device=dev, M=args.m)
-    x_dn, w_dn = inputs.wan_ffn(seed=seed, which="down", device=dev, M=args.m)
-    wc_up, wsf_up = mxq.pack_weight(w_up)
-    wc_dn, wsf_dn = mxq.pack_weight(w_dn)
-    M = x_up.shape[0]
-    q_up = (torch.empty(M, D_MODEL // 2, dtype=torch.uint8, device=dev),
-            torch.empty(mxq.mxq_sf_bytes(M, D_MODEL), dtype=torch.uint8, device=dev))
-    q_dn = (torch.empty(M, D_FF // 2, dtype=torch.uint8, device=dev),
-            torch.empty(mxq.mxq_sf_bytes(M, D_FF), dtype=torch.uint8, device=dev))
-    d_up = torch.empty(M, D_FF, dtype=torch.bfloat16, device=dev)
-    d_dn = torch.empty(M, D_MODEL, dtype=torch.bfloat16, device=dev)
+    # Inputs (per rank its own token batch); weights packed once before timing.
+    default_m = {"wan_ffn": M_TOK, "wan_attn_hadamard": M_TOK, "flux_w4a8": 3584, "m_sweep": 1024}[args.workload]
+    M = args.m if args.m else default_m
+    desc, parts, x_in, d_out, flops_step = build_workload(args.workload, dev, M, 2000 + 100 * rank, args.rule)
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
+        for i, p in enumerate(parts):
+            if ev is not None:
+                ev[i].record(stream)
+            p.fn()
         if ev is not None:
-            ev[0].record(stream)
-        mxq.quantize_act(x_up, mxq.MXQ_SCALE_OCP, False, out=q_up)
-        if ev is not None:
-            ev[1].record(stream)
-        mxq.gemm_w4a4(q_up[0], q_up[1], wc_up, wsf_up, M, D_FF, D_MODEL, out=d_up)
-        if ev is not None:
-            ev[2].record(stream)
-        mxq.quantize_act(x_dn, mxq.MXQ_SCALE_OCP, False, out=q_dn)
-        if ev is not None:
-            ev[3].record(stream)
-        mxq.gemm_w4a4(q_dn[0], q_dn[1], wc_dn, wsf_dn, M, D_MODEL, D_FF, out=d_dn)
-        if ev is not None:
-            ev[4].record(stream)
+            ev[len(parts)].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -246,64 +333,81 @@ def main():
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
-    flops_gemm = 2.0 * M * D_MODEL * D_FF
-    flops_step = 2 * flops_gemm
     value = world * flops_step * args.steps / (ms / 1e3) / 1e12
 
-    # Per-kernel durations (a second, separately timed pass with events between launches).
+    # Per-launch durations (a second, separately timed pass with events between launches).
     n_prof = max(5, min(20, args.steps))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_prof)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)] for _ in range(n_prof)]
     for e in evs:
         step(e)
     torch.cuda.synchronize(dev)
-    seg = [[e[i].elapsed_time(e[i + 1]) for e in evs] for i in range(4)]
-    quant_up_ms, gemm_up_ms, quant_dn_ms, gemm_dn_ms = (statistics.mean(s) for s in seg)
+    part_ms = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(len(parts))]
     if mxq.mxq_debug_poll() != 0:
         raise RuntimeError("a kernel reported a timeout during timing")
 
     peaks, peak_kind = measured_peaks()
-    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
-    gemm_ms = (gemm_up_ms + gemm_dn_ms) / 2
-    achieved = flops_gemm / (gemm_ms / 1e3) / 1e12
-    quant_bytes = lambda K: M * K * 2 + M * K // 2 + M * K // 32
-    q_gbs_up = quant_bytes(D_MODEL) / (quant_up_ms / 1e3) / 1e9
-    q_gbs_dn = quant_bytes(D_FF) / (quant_dn_ms / 1e3) / 1e9
-
+    # The timed region lasts a fraction of a second with clocks at their maximum, so the
+    # denominator is the burst (not the power-capped sustained) measured BF16 rate scaled by
+    # the nominal dtype ratio -- the larger, more conservative choice.
+    peak_of = {"fp4": peaks["bf16_tflops"] * FP4_PER_BF16, "fp8": peaks["bf16_tflops"] * FP8_PER_BF16}
+    parts_out = {}
+    for p, t in zip(parts, part_ms):
+        if p.kind == "gemm":
+            parts_out[p.label] = {"ms": t, "tflops": p.flops / (t / 1e3) / 1e12}
+        else:
+            parts_out[p.label] = {"ms": t, "gbs": p.nbytes / (t / 1e3) / 1e9}
+    gemm_t = sum(t for p, t in zip(parts, part_ms) if p.kind == "gemm")
+    quant_t = sum(t for p, t in zip(parts, part_ms) if p.kind == "quant")
+    gemm_parts = [p for p in parts if p.kind == "gemm"]
+    quant_parts = [p for p in parts if p.kind == "quant"]
+    gemm_kind = gemm_parts[0].peak_kind
+    achieved_g = sum(p.flops for p in gemm_parts) / (gemm_t / 1e3) / 1e12
+    achieved_q = sum(p.nbytes for p in quant_parts) / (quant_t / 1e3) / 1e9 if quant_parts else None
+    kernel_name = ("mx_gemm_pair_kernel" if M > 128 else "mx_gemm_kernel") + (
+        "<W4A8> (tcgen05 kind::mxf8f6f4)" if gemm_kind == "fp8" else "<W4A4> (tcgen05 kind::mxf4)")
+    if gemm_t >= quant_t:
+        roofline = {"bound": "tensor", "kernel": kernel_name, "achieved": achieved_g, "peak": peak_of[gemm_kind],
+                    "unit": "TFLOP/s", "frac": achieved_g / peak_of[gemm_kind],
+                    "peak_source": f"{peak_kind} bf16_tflops (burst) x "
+                                   f"{FP4_PER_BF16 if gemm_kind == 'fp4' else FP8_PER_BF16} (nominal ratio)",
+                    "traffic": TRAFFIC.get(args.workload)}
+    else:
+        roofline = {"bound": "hbm", "kernel": "quantize_act", "achieved": achieved_q, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": achieved_q / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
+                    "traffic": None}
+    nominal = NOMINAL_FP4_TFLOPS if gemm_kind == "fp4" else NOMINAL_FP8_TFLOPS
     result = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC if args.workload in ("wan_ffn", "m_sweep", "wan_attn_hadamard") else METRIC_W4A8,
+        "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "mxfp4 (e2m1 x e8m0, fp32 accumulate)", "data": "synthetic",
-        "config": {"workload": WORKLOAD if M == M_TOK else WORKLOAD.replace("32760", str(M)), "M": M,
-                   "d_model": D_MODEL, "d_ff": D_FF,
-                   "parallelism": f"replicas x{world} (token batches, no collective)",
-                   "l2": "inputs larger than L2 (> 2 GB of traffic per step), no explicit flush"},
-        "pct_of_dense_fp4_peak": 100.0 * value / world / NOMINAL_FP4_TFLOPS,
-        "roofline": {"bound": "tensor", "kernel": "mx_gemm_kernel<W4A4> (tcgen05 kind::mxf4)",
-                     "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
-                     "peak_source": f"{peak_kind} bf16_tflops_sustained x {FP4_PER_BF16} (nominal FP4:BF16)",
-                     "traffic": None},
-        "parts_ms": {"quant_up": quant_up_ms, "gemm_up": gemm_up_ms, "quant_down": quant_dn_ms,
-                     "gemm_down": gemm_dn_ms},
-        "quantizer": {"bound": "hbm", "achieved_up": q_gbs_up, "achieved_down": q_gbs_dn, "unit": "GB/s",
-                      "peak": peaks["hbm_gbs"], "frac_up": q_gbs_up / peaks["hbm_gbs"],
-                      "frac_down": q_gbs_dn / peaks["hbm_gbs"]},
-        "gpu_launches": 4 * args.steps,
+        "vs_baseline": None,
+        "dtype": "mxfp4 (e2m1 x e8m0, fp32 accumulate)" if gemm_kind == "fp4"
+                 else "e4m3 x mxfp4 (e8m0 scales, fp32 accumulate)",
+        "data": "synthetic",
+        "config": {"workload": desc, "M": M, "parallelism": f"replicas x{world} (token batches, no collective)",
+                   "l2": "inputs larger than L2 (> 100 MB of traffic per step), no explicit flush"},
+        "pct_of_dense_peak": 100.0 * value / world / nominal,
+        "roofline": roofline,
+        "gemm": {"achieved": achieved_g, "unit": "TFLOP/s", "peak": peak_of[gemm_kind],
+                 "frac": achieved_g / peak_of[gemm_kind]},
+        "quantizer": ({"achieved": achieved_q, "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                       "frac": achieved_q / peaks["hbm_gbs"]} if quant_parts else None),
+        "parts": parts_out,
+        "gpu_launches": len(parts) * args.steps,
         "clocks": clocks.summary(),
     }
 
-    # End to end through the public API: pinned host X in, D back to the host, every step.
+    # End to end through the public API: pinned host inputs in, outputs back, every step.
     if not args.no_e2e:
-        xh_up = x_up.cpu().pin_memory()
-        xh_dn = x_dn.cpu().pin_memory()
-        dh_up = torch.empty(d_up.shape, dtype=d_up.dtype, pin_memory=True)
-        dh_dn = torch.empty(d_dn.shape, dtype=d_dn.dtype, pin_memory=True)
+        hin = [x.cpu().pin_memory() for x in x_in]
+        hout = [torch.empty(d.shape, dtype=d.dtype, pin_memory=True) for d in d_out]
 
         def e2e_step():
-            x_up.copy_(xh_up, non_blocking=True)
-            x_dn.copy_(xh_dn, non_blocking=True)
+            for x, h in zip(x_in, hin):
+                x.copy_(h, non_blocking=True)
             step()
-            dh_up.copy_(d_up, non_blocking=True)
-            dh_dn.copy_(d_dn, non_blocking=True)
+            for d, h in zip(d_out, hout):
+                h.copy_(d, non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize(dev)
@@ -321,14 +425,15 @@ def main():
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             ems = float(t.item())
         result["e2e"] = {"value": world * flops_step * args.e2e_steps / (ems / 1e3) / 1e12, "unit": UNIT,
-                         "h2d_bytes_per_step": xh_up.numel() * 2 + xh_dn.numel() * 2,
-                         "d2h_bytes_per_step": dh_up.numel() * 2 + dh_dn.numel() * 2,
+                         "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h in hin),
+                         "d2h_bytes_per_step": sum(h.numel() * h.element_size() for h in hout),
                          "steps": args.e2e_steps}
 
-    if rank == 0 and not args.no_cpu_baseline:
-        rows = slice(0, CPU_SAMPLE_ROWS)
-        v, dt, cores = cpu_oracle_sample(x_up[rows].cpu(), x_dn[rows].cpu(), oracle_pack(w_up.cpu()),
-                                         oracle_pack(w_dn.cpu()))
+    if rank == 0 and not args.no_cpu_baseline and args.workload == "wan_ffn":
+        from mxfp4_block_scaled_mxq_b200 import inputs
+        x_up, w_up = inputs.wan_ffn(which="up", M=CPU_SAMPLE_ROWS)
+        x_dn, w_dn = inputs.wan_ffn(which="down", M=CPU_SAMPLE_ROWS)
+        v, dt, cores = cpu_oracle_sample(x_up, x_dn, oracle_pack(w_up), oracle_pack(w_dn))
         result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                                   "sample": f"{CPU_SAMPLE_ROWS} token rows of X_up and X_down (quantise + FP64 "
                                             f"GEMM vs all N), {dt:.1f} s"}
