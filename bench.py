@@ -40,6 +40,9 @@ FP8_PER_BF16 = 2.0                   # nominal FP8 : BF16 dense ratio (4.5 / 2.2
 # DRAM traffic per launch of the dominant kernel, from an ncu capture (see profiles/); None if
 # the kernel changed since the counters were taken.
 TRAFFIC = {}
+# Packed weight bytes per workload (MXFP4 codes + scales), for the L2-residency decision.
+W_BYTES = {"wan_ffn": 2 * 5120 * 13824 * 17 // 32, "wan_attn_hadamard": 4 * 5120 * 5120 * 17 // 32,
+           "flux_w4a8": (9216 + 12288) * 3072 * 17 // 32, "m_sweep": 13824 * 5120 * 17 // 32}
 WORKLOAD = "Wan2.2-A14B FFN W4A4 (up 32760x5120->13824, down 32760x13824->5120), dynamic MXFP4 acts, OCP rule"
 M_TOK, D_MODEL, D_FF = 32760, 5120, 13824
 
@@ -178,6 +181,25 @@ def run_reference(args, rank, world):
     }))
 
 
+# ------------------------------------------------------------------ multi-rank helpers
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own token batch (weak scaling over independent replicas)."""
+    return 2000 + 100 * rank
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The job's time is the slowest rank's (max over ranks, on the device for NCCL)."""
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """TFLOP/s of the whole job: every rank processes its own step of flops_per_step."""
+    return world * flops_per_step * steps / (max_ms / 1e3) / 1e12
+
+
 # ------------------------------------------------------------------ workloads
 class Part:
     """One kernel launch of the step: kind 'quant' (HBM-bound) or 'gemm' (tensor-bound)."""
@@ -298,16 +320,12 @@ def main():
     # Inputs (per rank its own token batch); weights packed once before timing.
     default_m = {"wan_ffn": M_TOK, "wan_attn_hadamard": M_TOK, "flux_w4a8": 3584, "m_sweep": 1024}[args.workload]
     M = args.m if args.m else default_m
-    desc, parts, x_in, d_out, flops_step = build_workload(args.workload, dev, M, 2000 + 100 * rank, args.rule)
+    desc, parts, x_in, d_out, flops_step = build_workload(args.workload, dev, M, rank_seed(rank), args.rule)
     stream = torch.cuda.current_stream(dev)
 
-    def step(ev=None):
-        for i, p in enumerate(parts):
-            if ev is not None:
-                ev[i].record(stream)
+    def step():
+        for p in parts:
             p.fn()
-        if ev is not None:
-            ev[len(parts)].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -315,33 +333,60 @@ def main():
     if mxq.mxq_debug_poll() != 0:
         raise RuntimeError("a kernel reported a timeout during warm-up")
 
-    # Whole-step timing (events only at the boundaries).
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # The step is captured once in a CUDA graph and replayed (no host launch overhead).
+    # Working sets that fit in L2 get an untimed L2 flush before every timed replay.
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    working_set = sum(t.numel() * t.element_size() for t in x_in + d_out) + W_BYTES.get(args.workload, 0)
+    flush = working_set < 4 * l2
+    scratch = torch.empty(2 * l2, dtype=torch.uint8, device=dev) if flush else None
+
+    def capture(fns):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for f in fns:
+                f()
+        return g
+
+    def time_graph(g, iters):
+        """Device time of `iters` replays (ms), flushed or back to back."""
+        if flush:
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+            for e0, e1 in evs:
+                scratch.zero_()
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+            torch.cuda.synchronize(dev)
+            return sum(e0.elapsed_time(e1) for e0, e1 in evs)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1)
+
+    step_graph = capture([p.fn for p in parts])
+    step_graph.replay()
+    torch.cuda.synchronize(dev)
+
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
-        start.record(stream)
-        for _ in range(args.steps):
-            step()
-        stop.record(stream)
-        torch.cuda.synchronize(dev)
+        ms = time_graph(step_graph, args.steps)
     if world > 1:
         dist.barrier()
-    ms = start.elapsed_time(stop)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * flops_step * args.steps / (ms / 1e3) / 1e12
+        ms = max_over_ranks(ms, dist, dev)
+    value = whole_job_rate(flops_step, args.steps, world, ms)
 
-    # Per-launch durations (a second, separately timed pass with events between launches).
+    # Per-launch durations: each part captured alone and timed the same way.
     n_prof = max(5, min(20, args.steps))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)] for _ in range(n_prof)]
-    for e in evs:
-        step(e)
-    torch.cuda.synchronize(dev)
-    part_ms = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(len(parts))]
+    part_ms = []
+    for p in parts:
+        g = capture([p.fn])
+        g.replay()
+        part_ms.append(time_graph(g, n_prof) / n_prof)
     if mxq.mxq_debug_poll() != 0:
         raise RuntimeError("a kernel reported a timeout during timing")
 
@@ -385,7 +430,9 @@ def main():
                  else "e4m3 x mxfp4 (e8m0 scales, fp32 accumulate)",
         "data": "synthetic",
         "config": {"workload": desc, "M": M, "parallelism": f"replicas x{world} (token batches, no collective)",
-                   "l2": "inputs larger than L2 (> 100 MB of traffic per step), no explicit flush"},
+                   "l2": (f"working set {working_set / 1e6:.0f} MB < 4x L2: L2 flushed (untimed) before every "
+                          f"timed step" if flush else f"working set {working_set / 1e9:.2f} GB > L2, steps back to back"),
+                   "timing": "step captured in one CUDA graph, replayed; CUDA events on the launching stream"},
         "pct_of_dense_peak": 100.0 * value / world / nominal,
         "roofline": roofline,
         "gemm": {"achieved": achieved_g, "unit": "TFLOP/s", "peak": peak_of[gemm_kind],
@@ -421,10 +468,8 @@ def main():
         torch.cuda.synchronize(dev)
         ems = e0.elapsed_time(e1)
         if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        result["e2e"] = {"value": world * flops_step * args.e2e_steps / (ems / 1e3) / 1e12, "unit": UNIT,
+            ems = max_over_ranks(ems, dist, dev)
+        result["e2e"] = {"value": whole_job_rate(flops_step, args.e2e_steps, world, ems), "unit": UNIT,
                          "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h in hin),
                          "d2h_bytes_per_step": sum(h.numel() * h.element_size() for h in hout),
                          "steps": args.e2e_steps}

@@ -236,7 +236,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mt = tile / n_tiles, nt = tile % n_tiles;
-      if (!mbar_wait(tmem_full, acc_phase)) break;
+      // warp-uniform wait: tcgen05.ld below is .sync.aligned
+      if (!__all_sync(0xffffffffu, mbar_wait(tmem_full, acc_phase))) break;
       tc_fence_after();
       uint32_t acc[4][32];
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + kAccCol + chalf * 128;

@@ -16,10 +16,18 @@
 //   MMA (warp 1, leader CTA only)  waits `full[s]`, copies the scale atoms of both
 //                                  CTAs into their TMEMs (tcgen05.cp.cta_group::2),
 //                                  issues 4 MMAs, commits to `empty[s]` of both CTAs;
-//                                  after the K loop commits to `tmem_full` of both.
+//                                  after the K loop commits to `acc_full[a]` of both.
 //   epilogue (warps 2..9, both)    drain their CTA's accumulator, arrive on the
-//                                  LEADER's `tmem_empty` (16 arrivals per tile), then
-//                                  scale / bias / round and TMA-store their 128 rows.
+//                                  LEADER's barriers, then scale / bias / round and
+//                                  store their 128 rows.
+//
+// Overlapping accumulators: a 256-column FP32 accumulator per tile leaves no room for
+// two disjoint buffers next to the scale columns, so tiles alternate between two
+// accumulators at TMEM columns 0 and 192 that share columns [192, 256).  The next
+// tile's MMAs need only (a) the previous tile's shared 64 columns drained -- the four
+// warps holding them load those first and arrive on `ovl_free` -- and (b) their own
+// accumulator fully drained two tiles ago (`acc_free[a]`).  The accumulator hand-off
+// then costs one 64-column TMEM load instead of the whole 256-column drain.
 // Every wait is bounded as in gemm.cuh; the CTAs leave only after a final cluster
 // barrier, so neither frees TMEM or shared memory the pair's MMAs may still use.
 #pragma once
@@ -28,7 +36,11 @@
 
 namespace mxq {
 
-constexpr int kPairStages = 5;
+constexpr int kPairStages = 6;
+// two 256-column accumulators sharing [192, 256)
+__device__ __forceinline__ constexpr uint32_t pair_acc_col(uint32_t a) { return a ? 192u : 0u; }
+constexpr uint32_t kPairSfa = 448;           // A scales: 2 parities x 2 atoms x 4 columns
+constexpr uint32_t kPairSfb = 464;           // B scales: 2 parities x 2 atoms x 8 columns (to 496)
 
 template <bool kW4A8>
 struct PairShape {
@@ -44,8 +56,7 @@ struct PairShape {
   static constexpr int kSfaConst = kW4A8 ? 512 : 0;
   static constexpr uint32_t kTxPerCta =
       128 * 128 + (kW4A8 ? 128 * 64 : 128 * 128) + kSfaStage + kSfbStage;  // unpacked FP4 counts packed bytes
-  static constexpr int kSmemBytes = 1024 + kPairStages * (kAStage + kBStage + kSfaStage + kSfbStage) + kSfaConst +
-                                    kEpiWarps * kEpiStageBytes + 256;
+  static constexpr int kSmemBytes = 1024 + kPairStages * (kAStage + kBStage + kSfaStage + kSfbStage) + kSfaConst + 256;
   static constexpr uint32_t kIdesc = (kW4A8 ? (0u << 7) | (5u << 10) : (1u << 7) | (1u << 10)) |
                                      (static_cast<uint32_t>(256 >> 3) << 17) | (1u << 23) |
                                      (static_cast<uint32_t>(256 >> 4) << 24);
@@ -55,21 +66,21 @@ template <bool kW4A8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                         const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
-                        const __grid_constant__ CUtensorMap tmap_d, const __nv_bfloat16* __restrict__ bias, int M,
-                        int N, int K, float alpha) {
+                        __nv_bfloat16* __restrict__ d, int64_t ldd, int d_vec32,
+                        const __nv_bfloat16* __restrict__ bias, int M, int N, int K, float alpha) {
   using S = PairShape<kW4A8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + kPairStages * S::kAStage;
-  uint8_t* sEpi = sB + kPairStages * S::kBStage;
-  uint8_t* sSfa = sEpi + kEpiWarps * kEpiStageBytes;
+  uint8_t* sSfa = sB + kPairStages * S::kBStage;
   uint8_t* sSfb = sSfa + kPairStages * S::kSfaStage + S::kSfaConst;
   uint64_t* full = reinterpret_cast<uint64_t*>(sSfb + kPairStages * S::kSfbStage);
   uint64_t* empty = full + kPairStages;
-  uint64_t* tmem_full = empty + kPairStages;
-  uint64_t* tmem_empty = tmem_full + 1;
-  uint64_t* drain = tmem_empty + 1;
+  uint64_t* acc_full = empty + kPairStages;  // [2]
+  uint64_t* acc_free = acc_full + 2;         // [2], leader's used
+  uint64_t* ovl_free = acc_free + 2;         // leader's used
+  uint64_t* drain = ovl_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -88,13 +99,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     prefetch_tmap(&tmap_b);
     prefetch_tmap(&tmap_sfa);
     prefetch_tmap(&tmap_sfb);
-    prefetch_tmap(&tmap_d);
     for (int s = 0; s < kPairStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(tmem_full, 1);
-    mbar_init(tmem_empty, 2 * kEpiWarps);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_free[a], 2 * kEpiWarps);  // every epilogue warp of both CTAs
+    }
+    mbar_init(ovl_free, kEpiWarps);  // the 4 warps per CTA that hold the shared columns
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -117,6 +130,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     if (elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
+      const uint64_t keep = l2_policy_evict_last();  // weights: reused by every row tile
       for (int tile = cluster; tile < num_tiles; tile += nclusters) {
         const int mt = tile / n_tiles, nt = tile % n_tiles;
         bool ok = true;
@@ -125,7 +139,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (leader) mbar_arrive_expect_tx(&full[stage], 2u * S::kTxPerCta);
           const uint32_t bar = map_to_rank(&full[stage], 0);
           tma_load_2d_pair(sA + stage * S::kAStage, &tmap_a, ks * 128, mt * 256 + rank * 128, bar);
-          tma_load_2d_pair(sB + stage * S::kBStage, &tmap_b, ks * 128, nt * 256 + rank * 128, bar);
+          tma_load_2d_pair_hint(sB + stage * S::kBStage, &tmap_b, ks * 128, nt * 256 + rank * 128, bar, keep);
           if (!kW4A8)
             tma_load_4d_pair(sSfa + stage * S::kSfaStage, &tmap_sfa, 0, 0, ks * S::kAtoms, 2 * mt + rank, bar);
           tma_load_4d_pair(sSfb + stage * S::kSfbStage, &tmap_sfb, 0, 0, ks * S::kAtoms, 2 * nt, bar);
@@ -138,17 +152,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------------ MMA issuer (leader CTA)
     if (leader && elect_one()) {
       int stage = 0;
-      uint32_t phase = 0, acc_phase = 0, sf_par = 0;
+      uint32_t phase = 0, sf_par = 0;
       bool ok = true;
       bool first = true;
-      for (int tile = cluster; ok && tile < num_tiles; tile += nclusters) {
-        if (!mbar_wait(tmem_empty, acc_phase ^ 1)) { ok = false; break; }
+      uint32_t it = 0;  // this cluster's tile count: accumulator it & 1, its use it >> 1
+      for (int tile = cluster; ok && tile < num_tiles; tile += nclusters, ++it) {
+        const uint32_t a_idx = it & 1u;
+        if (!mbar_wait(&acc_free[a_idx], ((it >> 1) & 1u) ^ 1u)) { ok = false; break; }  // drained 2 tiles ago
+        if (!mbar_wait(ovl_free, (it & 1u) ^ 1u)) { ok = false; break; }               // previous tile's shared cols
         tc_fence_after();
+        const uint32_t acc_col = pair_acc_col(a_idx);
         for (int ks = 0; ks < k_stages; ++ks) {
           if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sfa_base = kW4A8 ? kSfaCol : kSfaCol + sf_par * (S::kAtoms * 4);
-          const uint32_t sfb_base = kSfbCol + sf_par * (S::kAtoms * 8);
+          const uint32_t sfa_base = kW4A8 ? kPairSfa : kPairSfa + sf_par * (S::kAtoms * 4);
+          const uint32_t sfb_base = kPairSfb + sf_par * (S::kAtoms * 8);
           sf_par ^= 1u;
 #pragma unroll
           for (int a = 0; a < S::kAtoms; ++a) {
@@ -161,7 +179,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                                  smem_desc(smem_u32(sSfb + stage * S::kSfbStage + j * S::kAtoms * 512 + a * 512),
                                            0, 128, 0));
           }
-          if (kW4A8 && first) tc_cp_sf_atom_pair(tmem + kSfaCol, smem_desc(smem_u32(sSfa), 0, 128, 0));
+          if (kW4A8 && first) tc_cp_sf_atom_pair(tmem + kPairSfa, smem_desc(smem_u32(sSfa), 0, 128, 0));
           first = false;
           const uint32_t a_base = smem_u32(sA + stage * S::kAStage);
           const uint32_t b_base = smem_u32(sB + stage * S::kBStage);
@@ -173,19 +191,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const uint32_t idesc = S::kIdesc | (sf_id << 29) | (sf_id << 4);
             const uint64_t adesc = smem_desc(a_base + kk * 32, 16, 1024, 2);
             const uint64_t bdesc = smem_desc(b_base + kk * 32, 16, 1024, 2);
-            const uint32_t tsfa = kW4A8 ? tmem + kSfaCol : tmem + sfa_base + 4 * a;
+            const uint32_t tsfa = kW4A8 ? tmem + kPairSfa : tmem + sfa_base + 4 * a;
             const uint32_t tsfb = tmem + sfb_base + 8 * a;
             if (kW4A8)
-              tc_mma_mxf8f6f4_pair(tmem + kAccCol, adesc, bdesc, idesc, tsfa, tsfb, (ks | kk) != 0);
+              tc_mma_mxf8f6f4_pair(tmem + acc_col, adesc, bdesc, idesc, tsfa, tsfb, (ks | kk) != 0);
             else
-              tc_mma_mxf4_pair(tmem + kAccCol, adesc, bdesc, idesc, tsfa, tsfb, (ks | kk) != 0);
+              tc_mma_mxf4_pair(tmem + acc_col, adesc, bdesc, idesc, tsfa, tsfb, (ks | kk) != 0);
           }
           tc_commit_pair(&empty[stage], 0x3);
           if (++stage == kPairStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        tc_commit_pair(tmem_full, 0x3);
-        acc_phase ^= 1;
+        tc_commit_pair(&acc_full[a_idx], 0x3);
       }
       if (!ok) {
         tc_commit_pair(drain, 0x1);
@@ -194,33 +211,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
+    // Thread `lane` of warp (quad, chalf) owns output row 32*quad + lane of its CTA's
+    // 128 rows and columns [128*chalf, +128) of the tile.
     const int ew = warp - 2;
     const int quad = warp & 3;
     const int chalf = ew >> 2;
-    uint8_t* stage_buf = sEpi + ew * kEpiStageBytes;
-    const uint32_t stage_addr = smem_u32(stage_buf);
-    const uint32_t tmem_empty_leader = map_to_rank(tmem_empty, 0);
-    uint32_t acc_phase = 0;
-    for (int tile = cluster; tile < num_tiles; tile += nclusters) {
+    const uint32_t acc_free_leader0 = map_to_rank(&acc_free[0], 0);
+    const uint32_t acc_free_leader1 = map_to_rank(&acc_free[1], 0);
+    const uint32_t ovl_free_leader = map_to_rank(ovl_free, 0);
+    const uint64_t stream_out = l2_policy_evict_first();
+    uint32_t it = 0;
+    for (int tile = cluster; tile < num_tiles; tile += nclusters, ++it) {
       const int mt = tile / n_tiles, nt = tile % n_tiles;
-      if (!mbar_wait(tmem_full, acc_phase)) break;
+      const uint32_t a_idx = it & 1u;
+      // warp-uniform wait: tcgen05.ld below is .sync.aligned
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[a_idx], (it >> 1) & 1u))) break;
       tc_fence_after();
-      uint32_t acc[4][32];
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + kAccCol + chalf * 128;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(taddr + 32 * c, acc[c]);
+      // v[j] = accumulator column 128 * chalf + j of this warp's 32 lanes.  The shared
+      // columns [192, 256) are this warp's upper half (accumulator 0, chalf 1) or its
+      // lower half (accumulator 1, chalf 0): those four warps load them first.
+      uint32_t v[128];
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + pair_acc_col(a_idx) + chalf * 128;
+      if (a_idx == 0 && chalf == 1) {
+        tmem_ld64(taddr + 64, v + 64);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(ovl_free_leader);
+        tmem_ld64(taddr, v);
+      } else if (a_idx == 1 && chalf == 0) {
+        tmem_ld64(taddr, v);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(ovl_free_leader);
+        tmem_ld64(taddr + 64, v + 64);
+      } else {
+        tmem_ld64(taddr, v);
+        tmem_ld64(taddr + 64, v + 64);
+      }
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tmem_empty_leader);
-      acc_phase ^= 1;
+      if (lane == 0) mbar_arrive_cluster(a_idx ? acc_free_leader1 : acc_free_leader0);
 
-      const int row_base = mt * 256 + static_cast<int>(rank) * 128 + quad * 32;
+      const int row = mt * 256 + static_cast<int>(rank) * 128 + quad * 32 + lane;
+      __nv_bfloat16* drow = d + static_cast<int64_t>(row < M ? row : 0) * ldd;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int n0 = nt * 256 + chalf * 128 + 32 * c;
-        if (lane == 0) bulk_wait_read0();
-        __syncwarp();
+        if (row >= M || n0 >= N) continue;
         uint32_t packed[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -230,27 +270,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             if (n < N) b0 = __bfloat162float(bias[n]);
             if (n + 1 < N) b1 = __bfloat162float(bias[n + 1]);
           }
-          const float v0 = __fmaf_rn(alpha, __uint_as_float(acc[c][2 * j]), b0);
-          const float v1 = __fmaf_rn(alpha, __uint_as_float(acc[c][2 * j + 1]), b1);
+          const float v0 = __fmaf_rn(alpha, __uint_as_float(v[32 * c + 2 * j]), b0);
+          const float v1 = __fmaf_rn(alpha, __uint_as_float(v[32 * c + 2 * j + 1]), b1);
           packed[j] = pack_bf16x2(v0, v1);
         }
+        if (d_vec32 && n0 + 32 <= N) {
+          st_global_v8_hint(drow + n0, packed, stream_out);
+          st_global_v8_hint(drow + n0 + 16, packed + 8, stream_out);
+        } else {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t off = lane * 64 + ((q ^ ((lane >> 1) & 3)) * 16);
-          asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(stage_addr + off), "r"(packed[4 * q]),
-                       "r"(packed[4 * q + 1]), "r"(packed[4 * q + 2]), "r"(packed[4 * q + 3])
-                       : "memory");
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && n0 < N && row_base < M) {
-          tma_store_2d(&tmap_d, stage_buf, n0, row_base);
-          bulk_commit();
+          for (int j = 0; j < 16; ++j) {
+            const int n = n0 + 2 * j;
+            if (n + 1 < N)
+              *reinterpret_cast<uint32_t*>(drow + n) = packed[j];
+            else if (n < N)
+              *reinterpret_cast<uint16_t*>(drow + n) = static_cast<uint16_t>(packed[j] & 0xFFFFu);
+          }
         }
       }
     }
-    if (lane == 0) bulk_wait0();
-    __syncwarp();
   }
 
   tc_fence_before();

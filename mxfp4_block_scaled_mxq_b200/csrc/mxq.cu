@@ -115,7 +115,7 @@ mxq_status launch_gemm_pair(const void* a, const void* a_sf, const void* b, cons
   });
   if (attr_err != cudaSuccess || max_clusters < 1) return MXQ_ERR_CUDA;
 
-  CUtensorMap ta, tb, tsa, tsb, td;
+  CUtensorMap ta, tb, tsa, tsb;
   bool ok;
   if (kW4A8) {
     ok = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K, M, K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
@@ -127,14 +127,15 @@ mxq_status launch_gemm_pair(const void* a, const void* a_sf, const void* b, cons
          make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K / 2, N, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
          make_tmap_sf(&tsa, a_sf, M, K, S::kAtoms, 1);
   }
-  ok = ok && make_tmap_sf(&tsb, b_sf, N, K, S::kAtoms, 2) &&
-       make_tmap_2d(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, N, M, ldd * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  ok = ok && make_tmap_sf(&tsb, b_sf, N, K, S::kAtoms, 2);
   if (!ok) return MXQ_ERR_CUDA;
   const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
   const int clusters = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
+  // 32-byte output stores need 32-byte aligned rows
+  const int d_vec32 = (ldd % 16 == 0 && aligned(d, 32)) ? 1 : 0;
   kernel<<<2 * clusters, mxq::kGemmThreads, S::kSmemBytes, stream>>>(
-      ta, tb, tsa, tsb, td, static_cast<const __nv_bfloat16*>(bias), static_cast<int>(M), static_cast<int>(N),
-      static_cast<int>(K), alpha);
+      ta, tb, tsa, tsb, static_cast<__nv_bfloat16*>(d), ldd, d_vec32, static_cast<const __nv_bfloat16*>(bias),
+      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), alpha);
   return launch_status();
 }
 

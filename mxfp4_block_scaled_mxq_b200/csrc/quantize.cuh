@@ -103,42 +103,11 @@ __device__ __forceinline__ float exp2_neg(int e) {
   return e < 127 ? __uint_as_float(static_cast<uint32_t>(127 - e) << 23) : __uint_as_float(0x00400000u);
 }
 
-// 128-point normalised Sylvester-Hadamard across 8 consecutive lanes, each holding 16
-// consecutive elements (element j = 16 * (lane % 8) + i).  Butterfly strides 1, 2, 4,
-// 8 inside the thread, then 16, 32, 64 across lanes (xor 1, 2, 4); every stage is
-// (t_i, t_i+h) <- (t_i + t_i+h, t_i - t_i+h) in FP32 round-to-nearest, then one
-// multiply by fl32(1/sqrt(128)) -- the order of the definition, so the result is
-// bit-identical to the element-by-element butterfly.
-__device__ __forceinline__ void fwht128_8lanes(float (&f)[16], int l8) {
-#pragma unroll
-  for (int h = 1; h < 16; h *= 2) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if (i & h) continue;
-      const float a = f[i], b = f[i + h];
-      f[i] = __fadd_rn(a, b);
-      f[i + h] = __fsub_rn(a, b);
-    }
-  }
-#pragma unroll
-  for (int bit = 0; bit < 3; ++bit) {
-    const bool upper = (l8 >> bit) & 1;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float p = __shfl_xor_sync(0xffffffffu, f[i], 1 << bit);
-      f[i] = upper ? __fsub_rn(p, f[i]) : __fadd_rn(f[i], p);
-    }
-  }
-  const float c = __uint_as_float(kInvSqrt128Bits);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) f[i] = __fmul_rn(f[i], c);
-}
-
-// One CTA quantises rows [128*by, +128) x K columns [128*bx, +128) of x[rows][ld]:
-// codes [rows][K/2] and the tile's 512-byte scale atom (rows beyond `rows` and blocks
-// beyond K stay 0x00 padding).  Thread (warp w, lane l) owns, in iteration i, row
+// One CTA quantises rows [128*by, +128) x K columns [128*bx, +128) of x[rows][ld]
+// without rotation: codes [rows][K/2] and the tile's 512-byte scale atom (rows beyond
+// `rows` and blocks beyond K stay 0x00 padding).  Thread (warp w, lane l) owns, in iteration i, row
 // 16w + 4i + l/8 and elements [16 * (l%8), +16) of the tile's 128 columns.
-template <bool kHadamard, bool kUOS>
+template <bool kUOS>
 __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__ x, int64_t rows, int64_t K,
                                                     int64_t ld, uint8_t* __restrict__ codes,
                                                     uint8_t* __restrict__ sf) {
@@ -171,16 +140,7 @@ __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__
     const int64_t row = row0 + r;
     float f[16];
     bf16x16_to_float(w[i], f);
-    uint32_t amax;
-    if (kHadamard) {
-      fwht128_8lanes(f, l8);
-      float m = 0.f;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(f[j]));
-      amax = __float_as_uint(m);
-    } else {
-      amax = bf16x16_absmax(w[i]);
-    }
+    uint32_t amax = bf16x16_absmax(w[i]);
     amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));  // the other half of the block
     const int e = block_exponent<kUOS>(amax);
     const float s = exp2_neg(e);  // exact power of two
@@ -207,11 +167,124 @@ __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__
   }
 }
 
+// The rotated variant of the tile: two lanes per 128-element chunk, each holding 64
+// consecutive elements as 32 packed pairs P[i] = (t[i], t[i + 32]) -- so the pair's
+// halves are exactly the thread's two 32-element blocks.  Butterfly strides 1..16
+// run on packed pairs (FP32x2 add / fma with -1, both exact per half), stride 32 is
+// the within-pair butterfly, stride 64 is the one cross-lane exchange (xor 1); the
+// stage order and every rounding are those of the definition, so the rotated values
+// are bit-identical to the element-by-element butterfly.
+template <bool kUOS>
+__device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __restrict__ x, int64_t rows,
+                                                             int64_t K, int64_t ld, uint8_t* __restrict__ codes,
+                                                             uint8_t* __restrict__ sf) {
+  __shared__ __align__(16) uint8_t atom[512];
+  const int tid = threadIdx.x;
+  const int r = tid >> 1;   // row within the tile
+  const int half = tid & 1; // elements [64 * half, +64) of the tile's 128 columns
+  const int64_t row = static_cast<int64_t>(blockIdx.y) * 128 + r;
+  const int64_t k = static_cast<int64_t>(blockIdx.x) * 128 + 64 * half;  // K % 128 == 0
+  const bool ok = row < rows;
+
+  reinterpret_cast<uint32_t*>(atom)[tid & 127] = 0u;
+
+  float2 P[32];
+  {
+    uint32_t w[4][8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (ok) {
+        ld_stream_v8(x + row * ld + k + 16 * q, w[q]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[q][j] = 0u;
+      }
+    }
+    // element j = 16 q + 2 jj (+1) sits in w[q][jj] (low / high half)
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int jl = i, jh = i + 32;
+      const uint32_t wl = w[jl >> 4][(jl & 15) >> 1], wh = w[jh >> 4][(jh & 15) >> 1];
+      P[i].x = __uint_as_float((jl & 1) ? (wl & 0xFFFF0000u) : (wl << 16));
+      P[i].y = __uint_as_float((jh & 1) ? (wh & 0xFFFF0000u) : (wh << 16));
+    }
+  }
+  __syncthreads();  // atom zeroed
+
+  const float2 minus1 = make_float2(-1.f, -1.f);
+#pragma unroll
+  for (int h = 1; h < 32; h *= 2) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if (i & h) continue;
+      const float2 a = P[i], b = P[i + h];
+      P[i] = __fadd2_rn(a, b);
+      P[i + h] = __ffma2_rn(b, minus1, a);  // a - b, exactly rounded
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {  // stride 32: the two halves of each pair
+    const float a = P[i].x, b = P[i].y;
+    P[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+  }
+  {  // stride 64 across the lane pair: lower lane t + partner, upper lane partner - t
+    const float sgn = half ? -1.f : 1.f;
+    const float2 sg = make_float2(sgn, sgn);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float2 p = make_float2(__shfl_xor_sync(0xffffffffu, P[i].x, 1), __shfl_xor_sync(0xffffffffu, P[i].y, 1));
+      P[i] = __ffma2_rn(P[i], sg, p);
+    }
+  }
+  const float c = __uint_as_float(kInvSqrt128Bits);
+  const float2 cc = make_float2(c, c);
+  float m0 = 0.f, m1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    P[i] = __fmul2_rn(P[i], cc);
+    m0 = fmaxf(m0, fabsf(P[i].x));
+    m1 = fmaxf(m1, fabsf(P[i].y));
+  }
+  const int e0 = block_exponent<kUOS>(__float_as_uint(m0));
+  const int e1 = block_exponent<kUOS>(__float_as_uint(m1));
+  const float2 sc = make_float2(exp2_neg(e0), exp2_neg(e1));
+  uint32_t out[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 a = __fmul2_rn(P[8 * q + 2 * j], sc);
+      const float2 b = __fmul2_rn(P[8 * q + 2 * j + 1], sc);
+      lo |= e2m1x2(a.x, b.x) << (8 * j);  // block 0: elements 8q + 2j, 8q + 2j + 1
+      hi |= e2m1x2(a.y, b.y) << (8 * j);  // block 1: elements 32 + 8q + 2j, ...
+    }
+    out[q] = lo;
+    out[4 + q] = hi;
+  }
+  if (ok) {
+    uint4* dst = reinterpret_cast<uint4*>(codes + row * (K / 2) + k / 2);  // 16-byte aligned
+    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    *reinterpret_cast<uint16_t*>(atom + (r & 31) * 16 + (r >> 5) * 4 + 2 * half) =
+        static_cast<uint16_t>((e0 + 127) | ((e1 + 127) << 8));
+  }
+  __syncthreads();
+  if (tid < 32) {
+    const int64_t atoms_per_row_tile = K / 128;
+    const int64_t idx = static_cast<int64_t>(blockIdx.y) * atoms_per_row_tile + blockIdx.x;
+    reinterpret_cast<uint4*>(sf + idx * 512)[tid] = reinterpret_cast<const uint4*>(atom)[tid];
+  }
+}
+
 template <bool kHadamard, bool kUOS>
 __global__ void __launch_bounds__(kQuantThreads) quantize_act_mxfp4_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ldx, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ sf) {
-  quantize_mxfp4_tile<kHadamard, kUOS>(x, M, K, ldx, codes, sf);
+  if constexpr (kHadamard)
+    quantize_mxfp4_hadamard_tile<kUOS>(x, M, K, ldx, codes, sf);
+  else
+    quantize_mxfp4_tile<kUOS>(x, M, K, ldx, codes, sf);
 }
 
 // The offline weight packer: the same block arithmetic on W[N][K] rows.
@@ -219,7 +292,10 @@ template <bool kHadamard, bool kUOS>
 __global__ void __launch_bounds__(kQuantThreads) pack_weight_mxfp4_kernel(
     const uint16_t* __restrict__ w, int64_t N, int64_t K, int64_t ldw, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ sf) {
-  quantize_mxfp4_tile<kHadamard, kUOS>(w, N, K, ldw, codes, sf);
+  if constexpr (kHadamard)
+    quantize_mxfp4_hadamard_tile<kUOS>(w, N, K, ldw, codes, sf);
+  else
+    quantize_mxfp4_tile<kUOS>(w, N, K, ldw, codes, sf);
 }
 
 // Static FP8: q = E4M3_RNE_satfinite(fl32(x * inv_scale)), sign bit kept.  Each thread
