@@ -19,6 +19,8 @@ Parity status per function (what pins each one is in ``tests/test_oracle_*.py``)
   quantize_mxfp4 / _fp8       pinned: element-wise recomposition from the pinned codecs
   gemm                        pinned: exact-rational brute force on tiny shapes,
                               identities, error-quadrature property
+  bf16_rne / qdq_* /          pinned: torch's FP32->BF16 conversion, tie cases,
+  dequant_mxfp4_bf16          recomposition from the pinned codecs
 """
 
 from __future__ import annotations
@@ -89,6 +91,14 @@ def _load():
     lib.oracle_quantize_fp8.restype = None
     lib.oracle_dequant_mxfp4.argtypes = [P, P, I64, I64, P]
     lib.oracle_dequant_mxfp4.restype = None
+    lib.oracle_bf16_rne.argtypes = [ctypes.c_float]
+    lib.oracle_bf16_rne.restype = ctypes.c_uint16
+    lib.oracle_dequant_mxfp4_bf16.argtypes = [P, P, I64, I64, P]
+    lib.oracle_dequant_mxfp4_bf16.restype = None
+    lib.oracle_qdq_mxfp4.argtypes = [P, I64, I64, I64, ctypes.c_int, ctypes.c_int, P, ctypes.c_int]
+    lib.oracle_qdq_mxfp4.restype = None
+    lib.oracle_qdq_fp8.argtypes = [P, I64, I64, I64, ctypes.c_float, ctypes.c_float, P, ctypes.c_int]
+    lib.oracle_qdq_fp8.restype = None
     lib.oracle_gemm.argtypes = [ctypes.c_int, P, P, I64, P, P, I64, I64, ctypes.c_double, P, P, I64,
                                 P, ctypes.c_int]
     lib.oracle_gemm.restype = None
@@ -237,3 +247,34 @@ def gemm(a_codes: np.ndarray, a_sf: np.ndarray | None, b_codes: np.ndarray, b_sf
     _load().oracle_gemm(1 if a_fp8 else 0, _ptr(a_codes), _ptr(a_sf), M, _ptr(b_codes), _ptr(b_sf), N, K,
                         float(alpha), _ptr(bias_bits), _ptr(rows), rows.size, _ptr(y), _threads(nthreads))
     return y
+
+
+# ---------------------------------------------------------------- QDQ emulation / dequantisation
+def bf16_rne(v: float) -> int:
+    return int(_load().oracle_bf16_rne(ctypes.c_float(v)))
+
+
+def dequant_mxfp4_bf16(codes: np.ndarray, sf_physical: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """BF16 bit patterns [rows, K] of the dequantised MXFP4 values."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    sf_physical = np.ascontiguousarray(sf_physical, dtype=np.uint8)
+    out = np.empty((rows, K), np.uint16)
+    _load().oracle_dequant_mxfp4_bf16(_ptr(codes), _ptr(sf_physical), rows, K, _ptr(out))
+    return out
+
+
+def qdq_mxfp4(x, rule: int = RULE_OCP, hadamard: bool = False, nthreads: int | None = None) -> np.ndarray:
+    xb = _bf16_bits(x)
+    rows, K = xb.shape
+    out = np.empty((rows, K), np.uint16)
+    _load().oracle_qdq_mxfp4(_ptr(xb), rows, K, K, int(rule), int(bool(hadamard)), _ptr(out), _threads(nthreads))
+    return out
+
+
+def qdq_fp8(x, act_scale: float, nthreads: int | None = None) -> np.ndarray:
+    xb = _bf16_bits(x)
+    rows, K = xb.shape
+    out = np.empty((rows, K), np.uint16)
+    _load().oracle_qdq_fp8(_ptr(xb), rows, K, K, ctypes.c_float(fp8_inv_scale(act_scale)),
+                           ctypes.c_float(np.float32(act_scale)), _ptr(out), _threads(nthreads))
+    return out

@@ -36,6 +36,11 @@
 //      y[m][n] = alpha * sum_k deqA[m][k] * deqB[n][k] + bias[n]   (in FP64).
 //      [AMD Quark ... FLUX.1-dev MXFP4 -- "AMD Instinctプラットフォーム上の拡散
 //       モデル向けMXFP4量子化": the GEMM takes MXFP4 inputs with no dequant phase]
+//  * Quantise-dequantise (QDQ) emulation, the way the W4A8 results on the Wan2.2 page
+//    were obtained before native execution ("Native execution paths": QDQ emulation,
+//    quality only): out = BF16(dequant(quant(x))).  MXFP4: E2M1(code) * 2^e, exact in
+//    FP32 and in BF16 (overflow to Inf only for e = 127); FP8: fl32(E4M3(q) * s)
+//    rounded to BF16 (round to nearest even).
 //  * Scale-factor memory layout (not given by the pages; a reading): rows padded
 //    to a multiple of 128, scale columns to a multiple of 4, 512-byte atoms of
 //    128 rows x 4 scale columns, byte
@@ -297,6 +302,53 @@ void oracle_dequant_mxfp4(const uint8_t* codes, const uint8_t* sf_physical, int6
       const int sf = sf_physical[oracle_sf_offset(r, k / kBlock, K)];
       out[r * K + k] = std::ldexp(oracle_e2m1_decode(q), sf - 127);
     }
+}
+
+// ---------------------------------------------------------------- QDQ emulation
+
+// FP32 -> BF16, round to nearest, ties to even; NaN stays a (quiet) NaN.
+uint16_t oracle_bf16_rne(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, sizeof u);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) return static_cast<uint16_t>((u >> 16) | 0x40u);
+  const uint32_t lsb = (u >> 16) & 1u;
+  return static_cast<uint16_t>((u + 0x7FFFu + lsb) >> 16);
+}
+
+// BF16 of the dequantised MXFP4 values (scales from the swizzled buffer).
+void oracle_dequant_mxfp4_bf16(const uint8_t* codes, const uint8_t* sf_physical, int64_t rows, int64_t K,
+                               uint16_t* out) {
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t k = 0; k < K; ++k) {
+      const uint8_t byte = codes[r * (K / 2) + k / 2];
+      const uint8_t q = (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+      const int sf = sf_physical[oracle_sf_offset(r, k / kBlock, K)];
+      const double v = std::ldexp(oracle_e2m1_decode(q), sf - 127);  // exact, also as FP32 (or Inf)
+      out[r * K + k] = oracle_bf16_rne(static_cast<float>(v));
+    }
+  }
+}
+
+// out = BF16(dequant(quant(x))) for MXFP4 with the given rule / rotation.
+void oracle_qdq_mxfp4(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, int rule, int hadamard,
+                      uint16_t* out, int nthreads) {
+  std::vector<uint8_t> codes(static_cast<size_t>(rows * (K / 2)));
+  std::vector<uint8_t> sf_logical(static_cast<size_t>(rows * (K / kBlock)));
+  oracle_quantize_mxfp4(x, rows, K, ld, rule, hadamard, codes.data(), sf_logical.data(), nthreads);
+  std::vector<uint8_t> sf(static_cast<size_t>(oracle_sf_bytes(rows, K)));
+  oracle_sf_swizzle(sf_logical.data(), rows, K, sf.data());
+  oracle_dequant_mxfp4_bf16(codes.data(), sf.data(), rows, K, out);
+}
+
+// out = BF16(fl32(E4M3(fl32(x * inv_scale)) * scale)).
+void oracle_qdq_fp8(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, float inv_scale, float scale,
+                    uint16_t* out, int nthreads) {
+  std::vector<uint8_t> q(static_cast<size_t>(rows * K));
+  oracle_quantize_fp8(x, rows, K, ld, inv_scale, q.data(), nthreads);
+  for (int64_t i = 0; i < rows * K; ++i) {
+    const float v = static_cast<float>(oracle_e4m3_decode(q[i])) * scale;  // fl32 product
+    out[i] = oracle_bf16_rne(v);
+  }
 }
 
 // ---------------------------------------------------------------- GEMM
