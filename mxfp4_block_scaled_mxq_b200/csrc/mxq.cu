@@ -11,6 +11,7 @@
 #include "mxq.h"
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
+#include "gemm_swap.cuh"
 #include "quantize.cuh"
 
 namespace {
@@ -139,6 +140,46 @@ mxq_status launch_gemm_pair(const void* a, const void* a_sf, const void* b, cons
   return launch_status();
 }
 
+// Few tokens (M <= 128): D^T = W X^T with the weights on the MMA's 128-row side.
+template <bool kW4A8>
+mxq_status launch_gemm_swap(const DeviceInfo& dev, const void* a, const void* a_sf, const void* b, const void* b_sf,
+                            int64_t M, int64_t N, int64_t K, float alpha, const void* bias, void* d, int64_t ldd,
+                            cudaStream_t stream) {
+  using S = mxq::SwapShape<kW4A8>;
+  auto kernel = mxq::mx_gemm_swap_kernel<kW4A8>;
+  constexpr int kMaxSmem = 232448;  // opt-in shared memory per CTA on sm_100
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  });
+  if (attr_err != cudaSuccess) return MXQ_ERR_CUDA;
+  const int Mt = static_cast<int>((M + 15) / 16 * 16);
+  int stages = (kMaxSmem - S::kFixedBytes) / S::stage_bytes(Mt);
+  stages = stages > mxq::kSwapMaxStages ? mxq::kSwapMaxStages : stages;
+  const int smem = S::kFixedBytes + stages * S::stage_bytes(Mt);
+
+  CUtensorMap tw, tt, tsw, tst;
+  bool ok;
+  if (kW4A8) {
+    ok = make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, b, K, N, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_tmap_2d(&tt, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K, M, K, 128, Mt, CU_TENSOR_MAP_SWIZZLE_128B);
+    tst = tw;  // unused: E4M3 tokens carry unit scales
+  } else {
+    ok = make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K / 2, N, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_tmap_2d(&tt, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K / 2, M, K / 2, 128, Mt, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_tmap_sf(&tst, a_sf, M, K, S::kAtoms, 1);
+  }
+  ok = ok && make_tmap_sf(&tsw, b_sf, N, K, S::kAtoms, 1);
+  if (!ok) return MXQ_ERR_CUDA;
+  const int64_t tiles = (N + 127) / 128;
+  const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+  kernel<<<grid, mxq::kSwapThreads, smem, stream>>>(tw, tt, tsw, tst, static_cast<__nv_bfloat16*>(d), ldd,
+                                                    static_cast<const __nv_bfloat16*>(bias), static_cast<int>(M),
+                                                    static_cast<int>(N), static_cast<int>(K), alpha, stages);
+  return launch_status();
+}
+
 template <bool kW4A8>
 mxq_status launch_gemm(const void* a, const void* a_sf, const void* b, const void* b_sf, int64_t M, int64_t N,
                        int64_t K, float alpha, const void* bias, void* d, int64_t ldd, cudaStream_t stream) {
@@ -146,6 +187,7 @@ mxq_status launch_gemm(const void* a, const void* a_sf, const void* b, const voi
   mxq_status st = current_device(&dev);
   if (st != MXQ_OK) return st;
   if (M > mxq::kBM) return launch_gemm_pair<kW4A8>(a, a_sf, b, b_sf, M, N, K, alpha, bias, d, ldd, stream);
+  return launch_gemm_swap<kW4A8>(dev, a, a_sf, b, b_sf, M, N, K, alpha, bias, d, ldd, stream);
   CUtensorMap ta, tb, td;
   bool ok;
   if (kW4A8) {

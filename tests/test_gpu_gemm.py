@@ -83,6 +83,29 @@ def test_w4a8_cta_pair_edges():
     assert gemm_rel_err(d, rows, oracle_w4a8(x, w, s, rows)) <= GEMM_TOL
 
 
+@pytest.mark.parametrize("M", [1, 16, 48, 128])
+def test_w4a8_few_tokens(M):
+    """W4A8 in the few-token (weights as the MMA's 128-row side) path, with bias."""
+    x, w, x_cal = inputs.flux_w4a8(M=M)
+    w = w[:392].contiguous()
+    s = inputs.static_fp8_scale(x_cal)
+    bias = (torch.randn(392, generator=torch.Generator().manual_seed(M))).to(torch.bfloat16)
+    wc, wsf = mxq.pack_weight(w.cuda())
+    d = mxq.linear_w4a8(x.cuda(), s, wc, wsf, 392, bias=bias.cuda())
+    torch.cuda.synchronize()
+    rows = np.arange(M)
+    assert gemm_rel_err(d, rows, oracle_w4a8(x, w, s, rows, bias=bias)) <= GEMM_TOL
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 13824, 512), (7, 136, 384), (33, 1000, 1280), (100, 392, 640)])
+def test_few_token_shapes(M, N, K):
+    """Ragged M (rounded up to 16 for the MMA), N not a multiple of 128, K % 256 == 128."""
+    x = inputs.heavy_tailed_bf16(M, K, seed=3 * M + 1)
+    w = inputs.normal_bf16(N, K, 0.02, seed=N + 3)
+    bias = (torch.randn(N, generator=torch.Generator().manual_seed(N)) * 0.1).to(torch.bfloat16)
+    check_w4a4(x, w, bias=bias, alpha=0.5)
+
+
 def test_bias_and_alpha():
     x = inputs.normal_bf16(200, 512, 1.0, seed=1)
     w = inputs.normal_bf16(300, 512, 0.02, seed=2)
