@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MXFP4 W4A4 GEMM TFLOPS incl. act-quant and % of B200 dense FP4 peak"
 METRIC_W4A8 = "MXFP4 W4A8 GEMM TFLOPS incl. act-quant and % of B200 dense FP8 peak"
+METRIC_QDQ = "MXFP4 quantise-dequantise + weight dequantisation GB/s (HBM-bound)"
 UNIT = "TFLOP/s"
 NOMINAL_FP4_TFLOPS = 9000.0          # dense FP4, nominal
 NOMINAL_FP8_TFLOPS = 4500.0          # dense FP8, nominal (kind::mxf8f6f4 runs at the FP8 rate)
@@ -39,10 +40,11 @@ FP4_PER_BF16 = 4.0                   # nominal FP4 : BF16 dense ratio (9 / 2.25 
 FP8_PER_BF16 = 2.0                   # nominal FP8 : BF16 dense ratio (4.5 / 2.25 PFLOP/s)
 # DRAM traffic per launch of the dominant kernel, from an ncu capture (see profiles/); None if
 # the kernel changed since the counters were taken.
-TRAFFIC = {}
+# Wan FFN: mean of the up (241.4 + 867.0 MB) and down (345.3 + 314.8 MB) GEMM launches.
+TRAFFIC = {"wan_ffn": (241.4e6 + 867.0e6 + 345.3e6 + 314.8e6) / 2}
 # Packed weight bytes per workload (MXFP4 codes + scales), for the L2-residency decision.
 W_BYTES = {"wan_ffn": 2 * 5120 * 13824 * 17 // 32, "wan_attn_hadamard": 4 * 5120 * 5120 * 17 // 32,
-           "flux_w4a8": (9216 + 12288) * 3072 * 17 // 32, "m_sweep": 13824 * 5120 * 17 // 32}
+           "flux_w4a8": (9216 + 12288) * 3072 * 17 // 32, "m_sweep": 13824 * 5120 * 17 // 32, "qdq_wan_ffn": 0}
 WORKLOAD = "Wan2.2-A14B FFN W4A4 (up 32760x5120->13824, down 32760x13824->5120), dynamic MXFP4 acts, OCP rule"
 M_TOK, D_MODEL, D_FF = 32760, 5120, 13824
 
@@ -57,7 +59,7 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--m", type=int, default=0, help="token count (0: the workload's own)")
-    p.add_argument("--workload", choices=["wan_ffn", "wan_attn_hadamard", "flux_w4a8", "m_sweep"],
+    p.add_argument("--workload", choices=["wan_ffn", "wan_attn_hadamard", "flux_w4a8", "m_sweep", "qdq_wan_ffn"],
                    default="wan_ffn")
     p.add_argument("--rule", choices=["ocp", "uos"], default="ocp", help="activation scale rule")
     return p.parse_args()
@@ -292,6 +294,19 @@ def build_workload(name, dev, M, seed, rule_name):
         desc = f"M sweep W4A4: M={M}, 5120->13824, N(0,1) acts"
         return desc, p, [x], [d], sum(q.flops for q in p)
 
+    if name == "qdq_wan_ffn":
+        x, w = inputs.wan_ffn(seed=seed, which="up", device=dev, M=M)
+        rows, K = x.shape
+        N = w.shape[0]
+        wc, wsf = mxq.pack_weight(w)
+        d_x, d_w = out(rows, K), out(N, K)
+        parts = [Part("qdq_x_up", "quant", lambda: mxq.qdq_act(x, rule=rule, out=d_x), nbytes=4.0 * rows * K),
+                 Part("dequant_w_up", "quant", lambda: mxq.dequant_mxfp4(wc, wsf, K, out=d_w),
+                      nbytes=N * K / 2 + N * K / 32 + 2.0 * N * K)]
+        desc = (f"Wan2.2 FFN-up operands: fake-quantise X_up {rows}x{K} (MXFP4, {rule_name.upper()} rule) "
+                f"and expand packed W_up {N}x{K} to BF16")
+        return desc, parts, [x], [d_x, d_w], 0.0
+
     raise ValueError(f"unknown workload {name}")
 
 
@@ -318,7 +333,8 @@ def main():
     mxq.lib()
 
     # Inputs (per rank its own token batch); weights packed once before timing.
-    default_m = {"wan_ffn": M_TOK, "wan_attn_hadamard": M_TOK, "flux_w4a8": 3584, "m_sweep": 1024}[args.workload]
+    default_m = {"wan_ffn": M_TOK, "wan_attn_hadamard": M_TOK, "flux_w4a8": 3584, "m_sweep": 1024,
+                 "qdq_wan_ffn": M_TOK}[args.workload]
     M = args.m if args.m else default_m
     desc, parts, x_in, d_out, flops_step = build_workload(args.workload, dev, M, rank_seed(rank), args.rule)
     stream = torch.cuda.current_stream(dev)
@@ -378,7 +394,12 @@ def main():
     if world > 1:
         dist.barrier()
         ms = max_over_ranks(ms, dist, dev)
-    value = whole_job_rate(flops_step, args.steps, world, ms)
+    hbm_only = flops_step == 0.0
+    bytes_step = sum(p.nbytes for p in parts)
+    if hbm_only:  # GB/s: bytes per step instead of flops
+        value = whole_job_rate(bytes_step, args.steps, world, ms) * 1e3
+    else:
+        value = whole_job_rate(flops_step, args.steps, world, ms)
 
     # Per-launch durations: each part captured alone and timed the same way.
     n_prof = max(5, min(20, args.steps))
@@ -405,38 +426,47 @@ def main():
     quant_t = sum(t for p, t in zip(parts, part_ms) if p.kind == "quant")
     gemm_parts = [p for p in parts if p.kind == "gemm"]
     quant_parts = [p for p in parts if p.kind == "quant"]
-    gemm_kind = gemm_parts[0].peak_kind
-    achieved_g = sum(p.flops for p in gemm_parts) / (gemm_t / 1e3) / 1e12
+    gemm_kind = gemm_parts[0].peak_kind if gemm_parts else "fp4"
+    achieved_g = sum(p.flops for p in gemm_parts) / (gemm_t / 1e3) / 1e12 if gemm_parts else None
     achieved_q = sum(p.nbytes for p in quant_parts) / (quant_t / 1e3) / 1e9 if quant_parts else None
-    kernel_name = ("mx_gemm_pair_kernel" if M > 128 else "mx_gemm_kernel") + (
+    kernel_name = ("mx_gemm_pair_kernel" if M > 128 else "mx_gemm_swap_kernel") + (
         "<W4A8> (tcgen05 kind::mxf8f6f4)" if gemm_kind == "fp8" else "<W4A4> (tcgen05 kind::mxf4)")
-    if gemm_t >= quant_t:
+    if hbm_only:
+        top = max(zip(parts, part_ms), key=lambda pt: pt[1])
+        top_gbs = top[0].nbytes / (top[1] / 1e3) / 1e9
+        roofline = {"bound": "hbm", "kernel": top[0].label, "achieved": top_gbs, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": top_gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
+                    "traffic": None}
+    elif gemm_t >= quant_t:
         roofline = {"bound": "tensor", "kernel": kernel_name, "achieved": achieved_g, "peak": peak_of[gemm_kind],
                     "unit": "TFLOP/s", "frac": achieved_g / peak_of[gemm_kind],
                     "peak_source": f"{peak_kind} bf16_tflops (burst) x "
                                    f"{FP4_PER_BF16 if gemm_kind == 'fp4' else FP8_PER_BF16} (nominal ratio)",
-                    "traffic": TRAFFIC.get(args.workload)}
+                    "traffic": TRAFFIC.get(args.workload) if M == M_TOK else None,
+                    "traffic_note": "DRAM bytes per GEMM launch, mean over the step's launches (ncu)"}
     else:
         roofline = {"bound": "hbm", "kernel": "quantize_act", "achieved": achieved_q, "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": achieved_q / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
                     "traffic": None}
     nominal = NOMINAL_FP4_TFLOPS if gemm_kind == "fp4" else NOMINAL_FP8_TFLOPS
     result = {
-        "metric": METRIC if args.workload in ("wan_ffn", "m_sweep", "wan_attn_hadamard") else METRIC_W4A8,
-        "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": (METRIC_QDQ if hbm_only else
+                   METRIC if args.workload in ("wan_ffn", "m_sweep", "wan_attn_hadamard") else METRIC_W4A8),
+        "value": value, "unit": "GB/s" if hbm_only else UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "mxfp4 (e2m1 x e8m0, fp32 accumulate)" if gemm_kind == "fp4"
+        "dtype": "bf16 <-> mxfp4 (e2m1 x e8m0)" if hbm_only else "mxfp4 (e2m1 x e8m0, fp32 accumulate)"
+                 if gemm_kind == "fp4"
                  else "e4m3 x mxfp4 (e8m0 scales, fp32 accumulate)",
         "data": "synthetic",
         "config": {"workload": desc, "M": M, "parallelism": f"replicas x{world} (token batches, no collective)",
                    "l2": (f"working set {working_set / 1e6:.0f} MB < 4x L2: L2 flushed (untimed) before every "
                           f"timed step" if flush else f"working set {working_set / 1e9:.2f} GB > L2, steps back to back"),
                    "timing": "step captured in one CUDA graph, replayed; CUDA events on the launching stream"},
-        "pct_of_dense_peak": 100.0 * value / world / nominal,
+        "pct_of_dense_peak": None if hbm_only else 100.0 * value / world / nominal,
         "roofline": roofline,
-        "gemm": {"achieved": achieved_g, "unit": "TFLOP/s", "peak": peak_of[gemm_kind],
-                 "frac": achieved_g / peak_of[gemm_kind]},
+        "gemm": None if hbm_only else {"achieved": achieved_g, "unit": "TFLOP/s", "peak": peak_of[gemm_kind],
+                                       "frac": achieved_g / peak_of[gemm_kind]},
         "quantizer": ({"achieved": achieved_q, "unit": "GB/s", "peak": peaks["hbm_gbs"],
                        "frac": achieved_q / peaks["hbm_gbs"]} if quant_parts else None),
         "parts": parts_out,
@@ -469,7 +499,9 @@ def main():
         ems = e0.elapsed_time(e1)
         if world > 1:
             ems = max_over_ranks(ems, dist, dev)
-        result["e2e"] = {"value": whole_job_rate(flops_step, args.e2e_steps, world, ems), "unit": UNIT,
+        e2e_value = (whole_job_rate(bytes_step, args.e2e_steps, world, ems) * 1e3 if hbm_only
+                     else whole_job_rate(flops_step, args.e2e_steps, world, ems))
+        result["e2e"] = {"value": e2e_value, "unit": "GB/s" if hbm_only else UNIT,
                          "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h in hin),
                          "d2h_bytes_per_step": sum(h.numel() * h.element_size() for h in hout),
                          "steps": args.e2e_steps}

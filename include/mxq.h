@@ -158,6 +158,40 @@ MXQ_API mxq_status mxq_gemm_w4a8(const void* a_e4m3, float act_scale, const void
                          void* d_bf16, int64_t ldd, mxq_stream_t stream);
 
 /*
+ * mxq_dequant_mxfp4 -- out[r][k] = bf16(E2M1 value of code (r, k) * 2^(scale byte - 127)):
+ * the MXFP4 -> BF16 expansion of a tensor in the layout above (weights from
+ * mxq_pack_weight or activations from mxq_quantize_act).  Every product is a power of
+ * two times an E2M1 value, so it is exact in BF16 (or +-Inf past the BF16 range).
+ * Not on the W4A4 / W4A8 path (the GEMMs consume the MX operands directly); it serves
+ * layers kept in higher precision and checks of stored weights.
+ * [MXFP4 block structure and E8M0 scale: "MXFP4とは何か", AMD Instinct FP4 diffusion page]
+ *
+ * codes [rows][K/2] (16-byte aligned); sf as written by the quantiser
+ * (mxq_sf_bytes(rows, K) bytes; scale byte 0xFF, the E8M0 NaN, is outside the domain and
+ * its outputs are unspecified); out_bf16 [rows][ldo], 16-byte aligned, ldo >= K,
+ * ldo % 8 == 0, not overlapping the inputs.  1 <= rows <= 2^31, 32 <= K <= 2^22, K % 32 == 0.
+ */
+MXQ_API mxq_status mxq_dequant_mxfp4(const void* codes, const void* sf, int64_t rows, int64_t K,
+                                     void* out_bf16, int64_t ldo, mxq_stream_t stream);
+
+/*
+ * mxq_qdq_act -- quantise-dequantise ("fake quantisation") of activations in one pass:
+ * out = bf16(dequant(quant(x))) with exactly the arithmetic of mxq_quantize_act for the
+ * same (fmt, rule, hadamard128, act_scale), so that a BF16 layer fed `out` sees the values
+ * the W4A4 / W4A8 GEMM sees.  With hadamard128 the output stays in the rotated basis
+ * (x H/sqrt(128) quantised), as the GEMM's operand does.  FP8: out =
+ * bf16(fl32(E4M3 value * act_scale)).
+ * [Mixed-precision selection evaluates candidate precisions layer by layer: Wan2.2 page,
+ *  "Quark quantization pipeline and mixed-precision selection"]
+ *
+ * Arguments and limits as for mxq_quantize_act; out_bf16 [M][ldo], 16-byte aligned,
+ * ldo >= K, ldo % 8 == 0, not overlapping x.
+ */
+MXQ_API mxq_status mxq_qdq_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                               mxq_act_format fmt, mxq_scale_rule rule, int hadamard128,
+                               float act_scale, void* out_bf16, int64_t ldo, mxq_stream_t stream);
+
+/*
  * mxq_debug_poll -- reads and clears the library's device status word, written by a
  * kernel that gave up one of its bounded waits (each wait on a barrier or a copy is
  * capped at about a second, after which the kernel records MXQ_ERR_TIMEOUT, drains

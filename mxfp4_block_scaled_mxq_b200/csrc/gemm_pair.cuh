@@ -1,5 +1,5 @@
-// gemm_pair.cuh -- the block-scaled GEMM of gemm.cuh with a pair of CTAs (a
-// two-CTA thread-block cluster on two SMs) per 256 x 256 output tile.
+// gemm_pair.cuh -- the block-scaled GEMM (gemm_common.cuh) for M > 128 with a pair of
+// CTAs (a two-CTA thread-block cluster on two SMs) per 256 x 256 output tile.
 //
 // One tcgen05.mma.cta_group::2 of M = 256 spans both SMs: CTA r holds rows
 // [128r, 128r + 128) of the A tile and of the B tile (the N half), its own A-row
@@ -28,11 +28,11 @@
 // warps holding them load those first and arrive on `ovl_free` -- and (b) their own
 // accumulator fully drained two tiles ago (`acc_free[a]`).  The accumulator hand-off
 // then costs one 64-column TMEM load instead of the whole 256-column drain.
-// Every wait is bounded as in gemm.cuh; the CTAs leave only after a final cluster
+// Every wait is bounded (ptx.cuh); the CTAs leave only after a final cluster
 // barrier, so neither frees TMEM or shared memory the pair's MMAs may still use.
 #pragma once
 
-#include "gemm.cuh"
+#include "gemm_common.cuh"
 
 namespace mxq {
 

@@ -16,7 +16,7 @@
 //               one output row (64 contiguous bytes) per instruction.
 #pragma once
 
-#include "gemm.cuh"
+#include "gemm_common.cuh"
 
 namespace mxq {
 

@@ -1,5 +1,5 @@
 // mxq.cu -- libmxq: the C ABI of include/mxq.h (host-side validation, TMA tensor-map
-// encoding and launches) over the sm_100a kernels in quantize.cuh and gemm.cuh.
+// encoding and launches) over the sm_100a kernels in quantize.cuh, gemm_pair.cuh and gemm_swap.cuh.
 // One translation unit, so the library's device status word exists exactly once.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -9,7 +9,7 @@
 #include <mutex>
 
 #include "mxq.h"
-#include "gemm.cuh"
+#include "gemm_common.cuh"
 #include "gemm_pair.cuh"
 #include "gemm_swap.cuh"
 #include "quantize.cuh"
@@ -188,35 +188,6 @@ mxq_status launch_gemm(const void* a, const void* a_sf, const void* b, const voi
   if (st != MXQ_OK) return st;
   if (M > mxq::kBM) return launch_gemm_pair<kW4A8>(a, a_sf, b, b_sf, M, N, K, alpha, bias, d, ldd, stream);
   return launch_gemm_swap<kW4A8>(dev, a, a_sf, b, b_sf, M, N, K, alpha, bias, d, ldd, stream);
-  CUtensorMap ta, tb, td;
-  bool ok;
-  if (kW4A8) {
-    ok = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K, M, K, 128, mxq::kBM, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, b, K, N, K / 2, 128, mxq::kBN,
-                      CU_TENSOR_MAP_SWIZZLE_128B);
-  } else {
-    ok = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K / 2, M, K / 2, 128, mxq::kBM,
-                      CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K / 2, N, K / 2, 128, mxq::kBN,
-                      CU_TENSOR_MAP_SWIZZLE_128B);
-  }
-  ok = ok && make_tmap_2d(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, N, M, ldd * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
-  if (!ok) return MXQ_ERR_CUDA;
-
-  using S = mxq::GemmShape<kW4A8>;
-  auto kernel = mxq::mx_gemm_kernel<kW4A8>;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [&] {
-    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
-  });
-  if (attr_err != cudaSuccess) return MXQ_ERR_CUDA;
-  const int64_t tiles = ((M + mxq::kBM - 1) / mxq::kBM) * ((N + mxq::kBN - 1) / mxq::kBN);
-  const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-  kernel<<<grid, mxq::kGemmThreads, S::kSmemBytes, stream>>>(
-      ta, tb, td, static_cast<const uint8_t*>(a_sf), static_cast<const uint8_t*>(b_sf),
-      static_cast<const __nv_bfloat16*>(bias), static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), alpha);
-  return launch_status();
 }
 
 mxq_status check_gemm_shapes(const void* a, const void* b, const void* b_sf, const void* d, int64_t M, int64_t N,
@@ -355,6 +326,69 @@ mxq_status mxq_gemm_w4a8(const void* a_e4m3, float act_scale, const void* b_code
   if (st != MXQ_OK) return st;
   if (!aligned(b_codes, 32)) return MXQ_ERR_ALIGN;  // 16U4_ALIGN16B tensor maps need 32-byte bases
   return launch_gemm<true>(a_e4m3, nullptr, b_codes, b_sf, M, N, K, act_scale, bias_bf16, d_bf16, ldd, stream);
+}
+
+mxq_status mxq_dequant_mxfp4(const void* codes, const void* sf, int64_t rows, int64_t K, void* out_bf16,
+                             int64_t ldo, mxq_stream_t stream) {
+  if (!codes || !sf || !out_bf16) return MXQ_ERR_INVALID_ARG;
+  if (rows < 1 || rows > (int64_t(1) << 31) || K < 32 || K % 32 != 0 || K > (int64_t(1) << 22)) return MXQ_ERR_SHAPE;
+  if (ldo < K || ldo % 8 != 0) return MXQ_ERR_ALIGN;
+  if (!aligned(codes, 16) || !aligned(out_bf16, 16)) return MXQ_ERR_ALIGN;
+  DeviceInfo dev;
+  mxq_status st = current_device(&dev);
+  if (st != MXQ_OK) return st;
+  const int64_t units = rows * (K / 16);
+  const int64_t per_block = int64_t(mxq::kQuantThreads) * mxq::kDequantUnroll;
+  int64_t blocks = (units + per_block - 1) / per_block;
+  const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;
+  if (blocks > cap) blocks = cap;
+  mxq::dequant_mxfp4_kernel<<<static_cast<unsigned>(blocks), mxq::kQuantThreads, 0, stream>>>(
+      static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(sf), rows, K,
+      static_cast<uint16_t*>(out_bf16), ldo);
+  return launch_status();
+}
+
+mxq_status mxq_qdq_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, mxq_act_format fmt,
+                       mxq_scale_rule rule, int hadamard128, float act_scale, void* out_bf16, int64_t ldo,
+                       mxq_stream_t stream) {
+  if (!x_bf16 || !out_bf16) return MXQ_ERR_INVALID_ARG;
+  if (fmt != MXQ_ACT_MXFP4 && fmt != MXQ_ACT_FP8_E4M3) return MXQ_ERR_INVALID_ARG;
+  if (rule != MXQ_SCALE_OCP && rule != MXQ_SCALE_UOS) return MXQ_ERR_INVALID_ARG;
+  float inv = 0.f;
+  if (fmt == MXQ_ACT_FP8_E4M3) {
+    if (rule != MXQ_SCALE_OCP || hadamard128) return MXQ_ERR_INVALID_ARG;
+    if (!(act_scale > 0.f) || !std::isfinite(act_scale)) return MXQ_ERR_INVALID_ARG;
+    inv = 1.0f / act_scale;  // fl32(1 / s), as in the quantiser
+    if (!std::isfinite(inv)) return MXQ_ERR_INVALID_ARG;
+  }
+  const int64_t max_rows = fmt == MXQ_ACT_FP8_E4M3 ? (int64_t(1) << 31) : int64_t(65535) * 128;
+  if (M < 1 || M > max_rows || K < 32 || K % 32 != 0 || K > (int64_t(1) << 22)) return MXQ_ERR_SHAPE;
+  if (hadamard128 && K % 128 != 0) return MXQ_ERR_SHAPE;
+  if (ldx < K || ldx % 16 != 0 || ldo < K || ldo % 8 != 0) return MXQ_ERR_ALIGN;
+  if (!aligned(x_bf16, 32) || !aligned(out_bf16, 16)) return MXQ_ERR_ALIGN;
+  DeviceInfo dev;
+  mxq_status st = current_device(&dev);
+  if (st != MXQ_OK) return st;
+  const auto* xp = static_cast<const uint16_t*>(x_bf16);
+  auto* op = static_cast<uint16_t*>(out_bf16);
+  if (fmt == MXQ_ACT_FP8_E4M3) {
+    const int64_t chunks = M * (K / 16);
+    int64_t blocks = (chunks + mxq::kQuantThreads - 1) / mxq::kQuantThreads;
+    const int64_t cap = static_cast<int64_t>(dev.sm_count) * 16;
+    if (blocks > cap) blocks = cap;
+    mxq::qdq_act_fp8_kernel<<<static_cast<unsigned>(blocks), mxq::kQuantThreads, 0, stream>>>(xp, M, K, ldx, inv,
+                                                                                             act_scale, op, ldo);
+    return launch_status();
+  }
+  const dim3 grid(static_cast<unsigned>((K + 127) / 128), static_cast<unsigned>((M + 127) / 128));
+  const int sel = (hadamard128 ? 2 : 0) | (rule == MXQ_SCALE_UOS ? 1 : 0);
+  switch (sel) {
+    case 0: mxq::qdq_act_mxfp4_kernel<false, false><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, M, K, ldx, op, ldo); break;
+    case 1: mxq::qdq_act_mxfp4_kernel<false, true><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, M, K, ldx, op, ldo); break;
+    case 2: mxq::qdq_act_mxfp4_kernel<true, false><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, M, K, ldx, op, ldo); break;
+    default: mxq::qdq_act_mxfp4_kernel<true, true><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, M, K, ldx, op, ldo); break;
+  }
+  return launch_status();
 }
 
 mxq_status mxq_debug_poll(void) {

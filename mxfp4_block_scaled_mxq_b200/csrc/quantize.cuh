@@ -20,6 +20,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <cstdint>
 
@@ -56,6 +57,30 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\tcvt.u32.u16 %0, t;\n\t}"
       : "=r"(out)
       : "f"(hi), "f"(lo));
+  return out;
+}
+
+// One byte of two E2M1 codes -> two BF16 values code * scale (scale a power of two:
+// the product is exact in FP32, or overflows to Inf; BF16 holds it exactly): `lo`
+// nibble in bits 0-15.
+__device__ __forceinline__ uint32_t e2m1x2_to_bf16x2(uint32_t byte, float scale) {
+  uint32_t h;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h) : "r"(byte));
+  const float lo = __fmul_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xFFFFu))), scale);
+  const float hi = __fmul_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(h >> 16))), scale);
+  uint32_t out;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(hi), "f"(lo));
+  return out;
+}
+
+// Two E4M3 codes (bits 0-7, 8-15) -> two BF16 values bf16_rne(fl32(q * scale)).
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two, float scale) {
+  uint32_t h;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h) : "r"(two));
+  const float lo = __fmul_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xFFFFu))), scale);
+  const float hi = __fmul_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(h >> 16))), scale);
+  uint32_t out;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(hi), "f"(lo));
   return out;
 }
 
@@ -103,14 +128,20 @@ __device__ __forceinline__ float exp2_neg(int e) {
   return e < 127 ? __uint_as_float(static_cast<uint32_t>(127 - e) << 23) : __uint_as_float(0x00400000u);
 }
 
+// 2^e for e in [-127, 127].
+__device__ __forceinline__ float exp2_pos(int e) { return exp2_neg(-e); }
+
 // One CTA quantises rows [128*by, +128) x K columns [128*bx, +128) of x[rows][ld]
 // without rotation: codes [rows][K/2] and the tile's 512-byte scale atom (rows beyond
 // `rows` and blocks beyond K stay 0x00 padding).  Thread (warp w, lane l) owns, in iteration i, row
 // 16w + 4i + l/8 and elements [16 * (l%8), +16) of the tile's 128 columns.
-template <bool kUOS>
+// kQdq: instead of codes and scales, write BF16(dequant(quant(x))) to qdq[rows][ldq]
+// (the quantise-dequantise emulation; the same quantisation arithmetic).
+template <bool kUOS, bool kQdq = false>
 __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__ x, int64_t rows, int64_t K,
                                                     int64_t ld, uint8_t* __restrict__ codes,
-                                                    uint8_t* __restrict__ sf) {
+                                                    uint8_t* __restrict__ sf, uint16_t* __restrict__ qdq = nullptr,
+                                                    int64_t ldq = 0) {
   __shared__ __align__(16) uint8_t atom[512];  // byte (r%32)*16 + (r/32)*4 + block
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -154,11 +185,22 @@ __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__
         packed |= e2m1x2(__fmul_rn(f[8 * q + 2 * j], s), __fmul_rn(f[8 * q + 2 * j + 1], s)) << (8 * j);
       out[q] = packed;
     }
-    if (row < rows && k_ok) {
+    if (kQdq) {
+      if (row < rows && k_ok) {
+        const float up = exp2_pos(e);
+        uint32_t b[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) b[j] = e2m1x2_to_bf16x2((out[j >> 2] >> (8 * (j & 3))) & 0xFFu, up);
+        uint4* dst = reinterpret_cast<uint4*>(qdq + row * ldq + k);
+        dst[0] = make_uint4(b[0], b[1], b[2], b[3]);
+        dst[1] = make_uint4(b[4], b[5], b[6], b[7]);
+      }
+    } else if (row < rows && k_ok) {
       *reinterpret_cast<uint2*>(codes + row * (K / 2) + k / 2) = make_uint2(out[0], out[1]);
       if ((l8 & 1) == 0) atom[(r & 31) * 16 + (r >> 5) * 4 + (l8 >> 1)] = static_cast<uint8_t>(e + 127);
     }
   }
+  if (kQdq) return;  // uniform: no scale atom to write
   __syncthreads();
   if (tid < 32) {
     const int64_t atoms_per_row_tile = (K + 127) / 128;
@@ -174,10 +216,11 @@ __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__
 // the within-pair butterfly, stride 64 is the one cross-lane exchange (xor 1); the
 // stage order and every rounding are those of the definition, so the rotated values
 // are bit-identical to the element-by-element butterfly.
-template <bool kUOS>
+template <bool kUOS, bool kQdq = false>
 __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __restrict__ x, int64_t rows,
                                                              int64_t K, int64_t ld, uint8_t* __restrict__ codes,
-                                                             uint8_t* __restrict__ sf) {
+                                                             uint8_t* __restrict__ sf,
+                                                             uint16_t* __restrict__ qdq = nullptr, int64_t ldq = 0) {
   __shared__ __align__(16) uint8_t atom[512];
   const int tid = threadIdx.x;
   const int r = tid >> 1;   // row within the tile
@@ -262,6 +305,22 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
     out[q] = lo;
     out[4 + q] = hi;
   }
+  if (kQdq) {
+    if (ok) {  // block 0 = elements [k, k+32) (out[0..3]), block 1 = [k+32, k+64) (out[4..7])
+      const float up0 = exp2_pos(e0), up1 = exp2_pos(e1);
+#pragma unroll
+      for (int blk = 0; blk < 2; ++blk) {
+        uint32_t b[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          b[j] = e2m1x2_to_bf16x2((out[4 * blk + (j >> 2)] >> (8 * (j & 3))) & 0xFFu, blk ? up1 : up0);
+        uint4* dst = reinterpret_cast<uint4*>(qdq + row * ldq + k + 32 * blk);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(b[4 * q], b[4 * q + 1], b[4 * q + 2], b[4 * q + 3]);
+      }
+    }
+    return;  // uniform: no scale atom to write
+  }
   if (ok) {
     uint4* dst = reinterpret_cast<uint4*>(codes + row * (K / 2) + k / 2);  // 16-byte aligned
     dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
@@ -298,6 +357,82 @@ __global__ void __launch_bounds__(kQuantThreads) pack_weight_mxfp4_kernel(
     quantize_mxfp4_tile<kUOS>(w, N, K, ldw, codes, sf);
 }
 
+// Quantise-dequantise emulation of the MXFP4 activation quantiser (BF16 out).
+template <bool kHadamard, bool kUOS>
+__global__ void __launch_bounds__(kQuantThreads) qdq_act_mxfp4_kernel(const uint16_t* __restrict__ x, int64_t M,
+                                                                       int64_t K, int64_t ldx,
+                                                                       uint16_t* __restrict__ out, int64_t ldo) {
+  if constexpr (kHadamard)
+    quantize_mxfp4_hadamard_tile<kUOS, true>(x, M, K, ldx, nullptr, nullptr, out, ldo);
+  else
+    quantize_mxfp4_tile<kUOS, true>(x, M, K, ldx, nullptr, nullptr, out, ldo);
+}
+
+// MXFP4 -> BF16: a unit of work is 16 elements (8 code bytes + their scale byte from the
+// swizzled buffer) expanded into 32 contiguous output bytes, so a warp reads 256 and writes
+// 1024 contiguous bytes per unit.  Each thread takes kDequantUnroll units spaced one grid
+// apart per pass, loading all of them before converting any (independent loads in flight),
+// grid-stride over the [rows][K/16] units with (row, unit) advanced incrementally (no
+// 64-bit division inside the loop).
+constexpr int kDequantUnroll = 4;
+
+__global__ void __launch_bounds__(kQuantThreads) dequant_mxfp4_kernel(const uint8_t* __restrict__ codes,
+                                                                       const uint8_t* __restrict__ sf, int64_t rows,
+                                                                       int64_t K, uint16_t* __restrict__ out,
+                                                                       int64_t ldo) {
+  const int64_t cpr = K / 16;  // units per row
+  const int64_t atoms_per_row_tile = (K / 32 + 3) / 4;
+  const int64_t S = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t start = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t dr1 = S / cpr, dc1 = S - dr1 * cpr;  // one grid of units
+  const int64_t step = S * kDequantUnroll;
+  const int64_t drU = step / cpr, dcU = step - drU * cpr;
+  int64_t r[kDequantUnroll], c[kDequantUnroll];
+  r[0] = start / cpr;
+  c[0] = start - r[0] * cpr;
+#pragma unroll
+  for (int u = 1; u < kDequantUnroll; ++u) {
+    r[u] = r[u - 1] + dr1;
+    c[u] = c[u - 1] + dc1;
+    if (c[u] >= cpr) {
+      c[u] -= cpr;
+      ++r[u];
+    }
+  }
+  while (r[0] < rows) {  // r[0] <= r[1] <= ...: later units may already be past the end
+    uint2 cw[kDequantUnroll];
+    uint32_t sb[kDequantUnroll];
+#pragma unroll
+    for (int u = 0; u < kDequantUnroll; ++u) {
+      if (r[u] < rows) {
+        cw[u] = *reinterpret_cast<const uint2*>(codes + r[u] * (K / 2) + c[u] * 8);
+        const int64_t blk = c[u] >> 1;
+        sb[u] = sf[((r[u] >> 7) * atoms_per_row_tile + (blk >> 2)) * 512 + (r[u] & 31) * 16 +
+                   ((r[u] & 127) >> 5) * 4 + (blk & 3)];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kDequantUnroll; ++u) {
+      if (r[u] < rows) {
+        const float up = exp2_pos(static_cast<int>(sb[u]) - 127);
+        uint32_t b[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          b[j] = e2m1x2_to_bf16x2((((j < 4) ? cw[u].x : cw[u].y) >> (8 * (j & 3))) & 0xFFu, up);
+        uint4* dst = reinterpret_cast<uint4*>(out + r[u] * ldo + c[u] * 16);
+        dst[0] = make_uint4(b[0], b[1], b[2], b[3]);
+        dst[1] = make_uint4(b[4], b[5], b[6], b[7]);
+      }
+      r[u] += drU;
+      c[u] += dcU;
+      if (c[u] >= cpr) {
+        c[u] -= cpr;
+        ++r[u];
+      }
+    }
+  }
+}
+
 // Static FP8: q = E4M3_RNE_satfinite(fl32(x * inv_scale)), sign bit kept.  Each thread
 // converts 16-element chunks (32 bytes in, 16 bytes out) in a grid-stride loop.
 __global__ void __launch_bounds__(kQuantThreads) quantize_act_fp8_kernel(const uint16_t* __restrict__ x, int64_t M,
@@ -321,6 +456,36 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_act_fp8_kernel(const u
       o[j] = lo | (hi << 16);
     }
     *reinterpret_cast<uint4*>(q + row * K + k) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace mxq
+
+namespace mxq {
+
+// Quantise-dequantise emulation of the static FP8 activations:
+// out = bf16_rne(fl32(E4M3(fl32(x * inv_scale)) * scale)).
+__global__ void __launch_bounds__(kQuantThreads) qdq_act_fp8_kernel(const uint16_t* __restrict__ x, int64_t M,
+                                                                     int64_t K, int64_t ldx, float inv_scale,
+                                                                     float scale, uint16_t* __restrict__ out,
+                                                                     int64_t ldo) {
+  const int64_t chunks_per_row = K / 16;
+  const int64_t total = M * chunks_per_row;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < total; c += stride) {
+    const int64_t row = c / chunks_per_row;
+    const int64_t k = (c - row * chunks_per_row) * 16;
+    uint32_t w[8];
+    ld_stream_v8(x + row * ldx + k, w);
+    float f[16];
+    bf16x16_to_float(w, f);
+    uint32_t b[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      b[j] = e4m3x2_to_bf16x2(e4m3x2(__fmul_rn(f[2 * j], inv_scale), __fmul_rn(f[2 * j + 1], inv_scale)), scale);
+    uint4* dst = reinterpret_cast<uint4*>(out + row * ldo + k);
+    dst[0] = make_uint4(b[0], b[1], b[2], b[3]);
+    dst[1] = make_uint4(b[4], b[5], b[6], b[7]);
   }
 }
 

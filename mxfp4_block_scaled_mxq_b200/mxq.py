@@ -24,7 +24,7 @@ MXQ_SCALE_OCP, MXQ_SCALE_UOS = 0, 1
 MXQ_ACT_MXFP4, MXQ_ACT_FP8_E4M3 = 0, 1
 
 EXPORTED = ("mxq_status_string", "mxq_sf_bytes", "mxq_quantize_act", "mxq_pack_weight", "mxq_gemm_w4a4",
-            "mxq_gemm_w4a8", "mxq_debug_poll")
+            "mxq_gemm_w4a8", "mxq_dequant_mxfp4", "mxq_qdq_act", "mxq_debug_poll")
 
 
 class MxqError(RuntimeError):
@@ -57,6 +57,10 @@ def lib() -> ctypes.CDLL:
     L.mxq_gemm_w4a4.restype = I32
     L.mxq_gemm_w4a8.argtypes = [P, F32, P, P, I64, I64, I64, P, P, I64, P]
     L.mxq_gemm_w4a8.restype = I32
+    L.mxq_dequant_mxfp4.argtypes = [P, P, I64, I64, P, I64, P]
+    L.mxq_dequant_mxfp4.restype = I32
+    L.mxq_qdq_act.argtypes = [P, I64, I64, I64, I32, I32, I32, F32, P, I64, P]
+    L.mxq_qdq_act.restype = I32
     L.mxq_debug_poll.argtypes = []
     L.mxq_debug_poll.restype = I32
     _lib = L
@@ -115,6 +119,16 @@ def mxq_gemm_w4a4(a_codes, a_sf, b_codes, b_sf, M, N, K, alpha, bias, d, ldd, st
 def mxq_gemm_w4a8(a_e4m3, act_scale, b_codes, b_sf, M, N, K, bias, d, ldd, stream=None) -> None:
     _check(lib().mxq_gemm_w4a8(_ptr(a_e4m3), float(act_scale), _ptr(b_codes), _ptr(b_sf), int(M), int(N), int(K),
                                _ptr(bias), _ptr(d), int(ldd), _stream(stream)), "mxq_gemm_w4a8")
+
+
+def mxq_dequant_mxfp4(codes, sf, rows, K, out, ldo, stream=None) -> None:
+    _check(lib().mxq_dequant_mxfp4(_ptr(codes), _ptr(sf), int(rows), int(K), _ptr(out), int(ldo), _stream(stream)),
+           "mxq_dequant_mxfp4")
+
+
+def mxq_qdq_act(x, M, K, ldx, fmt, rule, hadamard128, act_scale, out, ldo, stream=None) -> None:
+    _check(lib().mxq_qdq_act(_ptr(x), int(M), int(K), int(ldx), int(fmt), int(rule), int(bool(hadamard128)),
+                             float(act_scale), _ptr(out), int(ldo), _stream(stream)), "mxq_qdq_act")
 
 
 def mxq_debug_poll() -> int:
@@ -181,6 +195,25 @@ def gemm_w4a8(a_e4m3, act_scale, b_codes, b_sf, M, N, K, bias=None, out=None, st
     d = _out_bf16(M, N, a_e4m3.device) if out is None else out
     mxq_gemm_w4a8(a_e4m3, act_scale, b_codes, b_sf, M, N, K, bias, d.data_ptr(), d.stride(0), stream)
     return d
+
+
+def dequant_mxfp4(codes: torch.Tensor, sf: torch.Tensor, K: int, out=None, stream=None) -> torch.Tensor:
+    """MXFP4 codes [rows][K/2] + swizzled scales -> BF16 [rows][K] (exact values)."""
+    rows = codes.shape[0]
+    o = _out_bf16(rows, K, codes.device) if out is None else out
+    mxq_dequant_mxfp4(codes, sf, rows, K, o.data_ptr(), o.stride(0), stream)
+    return o
+
+
+def qdq_act(x: torch.Tensor, fmt: int = MXQ_ACT_MXFP4, rule: int = MXQ_SCALE_OCP, hadamard128: bool = False,
+            act_scale: float = 1.0, out=None, stream=None) -> torch.Tensor:
+    """BF16 dequant(quant(X)) with the activation quantiser's arithmetic (fake quantisation)."""
+    x = _bf16_2d(x, "x")
+    M, K = x.shape
+    o = _out_bf16(M, K, x.device) if out is None else out
+    mxq_qdq_act(x.data_ptr(), M, K, x.stride(0), fmt, rule, hadamard128, act_scale, o.data_ptr(), o.stride(0),
+                stream)
+    return o
 
 
 def linear_w4a4(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE_OCP, hadamard128: bool = False,

@@ -104,6 +104,32 @@ def test_gemm_validation_happens_before_any_launch(L):
     assert g8(FAKE, 1.0, FAKE + 16, FAKE, 128, 256, 256, None, FAKE, 256, None) == ALIGN  # B needs 32 B
 
 
+def test_dequant_and_qdq_validation_happens_before_any_launch(L):
+    INV, SHAPE, ALIGN = 1, 2, 3
+    dq = lambda *a: L.mxq_dequant_mxfp4(*a)
+    assert dq(None, FAKE, 4, 64, FAKE, 64, None) == INV
+    assert dq(FAKE, None, 4, 64, FAKE, 64, None) == INV
+    assert dq(FAKE, FAKE, 0, 64, FAKE, 64, None) == SHAPE
+    assert dq(FAKE, FAKE, 4, 48, FAKE, 48, None) == SHAPE                    # K % 32
+    assert dq(FAKE, FAKE, 4, 64, FAKE, 60, None) == ALIGN                    # ldo < K
+    assert dq(FAKE, FAKE, 4, 64, FAKE, 68, None) == ALIGN                    # ldo % 8
+    assert dq(FAKE + 8, FAKE, 4, 64, FAKE, 64, None) == ALIGN                # codes 16-byte aligned
+    assert dq(FAKE, FAKE, 4, 64, FAKE + 8, 64, None) == ALIGN
+    qq = lambda *a: L.mxq_qdq_act(*a)
+    assert qq(None, 4, 64, 64, 0, 0, 0, 1.0, FAKE, 64, None) == INV
+    assert qq(FAKE, 4, 64, 64, 0, 0, 0, 1.0, None, 64, None) == INV
+    assert qq(FAKE, 4, 64, 64, 5, 0, 0, 1.0, FAKE, 64, None) == INV          # bad format
+    assert qq(FAKE, 4, 64, 64, 0, 3, 0, 1.0, FAKE, 64, None) == INV          # bad rule
+    assert qq(FAKE, 4, 64, 64, 1, 0, 0, -1.0, FAKE, 64, None) == INV         # FP8 scale <= 0
+    assert qq(FAKE, 4, 64, 64, 1, 1, 0, 1.0, FAKE, 64, None) == INV          # FP8 with UOS
+    assert qq(FAKE, 4, 64, 64, 1, 0, 1, 1.0, FAKE, 64, None) == INV          # FP8 with hadamard
+    assert qq(FAKE, 4, 96, 96, 0, 0, 1, 1.0, FAKE, 96, None) == SHAPE        # hadamard needs K % 128
+    assert qq(FAKE, 0, 64, 64, 0, 0, 0, 1.0, FAKE, 64, None) == SHAPE
+    assert qq(FAKE + 16, 4, 64, 64, 0, 0, 0, 1.0, FAKE, 64, None) == ALIGN   # x needs 32 bytes
+    assert qq(FAKE, 4, 64, 64, 0, 0, 0, 1.0, FAKE + 8, 64, None) == ALIGN    # out needs 16 bytes
+    assert qq(FAKE, 4, 64, 64, 0, 0, 0, 1.0, FAKE, 68, None) == ALIGN        # ldo % 8
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):

@@ -216,3 +216,25 @@ def test_m_sweep_largest():
     rows = sample_rows(65536, 64)
     d = run_w4a4(x, w)
     assert gemm_rel_err(d, rows, oracle_w4a4(x, w, rows)) <= GEMM_TOL
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("which", ["up", "down"])
+def test_full_output_against_fp32_matmul_of_expanded_operands(which):
+    """Supplement to the sampled oracle rows: every element of D at the full Wan FFN size
+    against an FP32 (no TF32) matmul of the operands expanded to BF16 by the dequantiser,
+    whose output is itself bit-exact against the oracle."""
+    x, w = inputs.wan_ffn(which=which, device="cuda")
+    M, K = x.shape
+    N = w.shape[0]
+    wc, wsf = mxq.pack_weight(w)
+    q, sf = mxq.quantize_act(x)
+    d = mxq.gemm_w4a4(q, sf, wc, wsf, M, N, K)
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        ref = mxq.dequant_mxfp4(q, sf, K).float() @ mxq.dequant_mxfp4(wc, wsf, K).float().T
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
+    err = ((d.float() - ref).abs().max() / ref.abs().max()).item()
+    assert err <= GEMM_TOL, err
