@@ -99,6 +99,13 @@ def _load():
     lib.oracle_qdq_mxfp4.restype = None
     lib.oracle_qdq_fp8.argtypes = [P, I64, I64, I64, ctypes.c_float, ctypes.c_float, P, ctypes.c_int]
     lib.oracle_qdq_fp8.restype = None
+    lib.oracle_quantize_mxfp4_smooth.argtypes = [P, I64, I64, I64, ctypes.c_int, ctypes.c_int, P, P, P,
+                                                 ctypes.c_int]
+    lib.oracle_quantize_mxfp4_smooth.restype = None
+    lib.oracle_channel_absmax.argtypes = [P, I64, I64, I64, ctypes.c_int, P]
+    lib.oracle_channel_absmax.restype = None
+    lib.oracle_smooth_factors.argtypes = [P, P, I64, ctypes.c_double, P, P]
+    lib.oracle_smooth_factors.restype = None
     lib.oracle_gemm.argtypes = [ctypes.c_int, P, P, I64, P, P, I64, I64, ctypes.c_double, P, P, I64,
                                 P, ctypes.c_int]
     lib.oracle_gemm.restype = None
@@ -278,3 +285,38 @@ def qdq_fp8(x, act_scale: float, nthreads: int | None = None) -> np.ndarray:
     _load().oracle_qdq_fp8(_ptr(xb), rows, K, K, ctypes.c_float(fp8_inv_scale(act_scale)),
                            ctypes.c_float(np.float32(act_scale)), _ptr(out), _threads(nthreads))
     return out
+
+
+# ---------------------------------------------------------------- SmoothQuant after the rotation
+def quantize_mxfp4_smooth(x, chan_scale: np.ndarray, rule: int = RULE_OCP, hadamard: bool = False,
+                          nthreads: int | None = None):
+    """MXFP4 quantisation of (x R) * chan_scale (per channel, FP32).  Returns (codes, sf_logical)."""
+    xb = _bf16_bits(x)
+    rows, K = xb.shape
+    c = np.ascontiguousarray(chan_scale, dtype=np.float32)
+    assert c.shape == (K,) and K % 32 == 0 and (not hadamard or K % 128 == 0)
+    codes = np.zeros((rows, K // 2), np.uint8)
+    sf = np.zeros((rows, K // 32), np.uint8)
+    _load().oracle_quantize_mxfp4_smooth(_ptr(xb), rows, K, K, int(rule), int(bool(hadamard)), _ptr(c),
+                                         _ptr(codes), _ptr(sf), _threads(nthreads))
+    return codes, sf
+
+
+def channel_absmax(x, hadamard: bool = False) -> np.ndarray:
+    """max over rows of |(x R)[r][k]| per channel k (FP32)."""
+    xb = _bf16_bits(x)
+    rows, K = xb.shape
+    out = np.empty(K, np.float32)
+    _load().oracle_channel_absmax(_ptr(xb), rows, K, K, int(bool(hadamard)), _ptr(out))
+    return out
+
+
+def smooth_factors(ax: np.ndarray, aw: np.ndarray, alpha: float = 0.5):
+    """SmoothQuant migration factors (lambda, fl32(1/lambda)) from the channel maxima."""
+    ax = np.ascontiguousarray(ax, dtype=np.float32)
+    aw = np.ascontiguousarray(aw, dtype=np.float32)
+    K = ax.size
+    lam = np.empty(K, np.float32)
+    inv = np.empty(K, np.float32)
+    _load().oracle_smooth_factors(_ptr(ax), _ptr(aw), K, float(alpha), _ptr(lam), _ptr(inv))
+    return lam, inv

@@ -41,6 +41,16 @@
 //    quality only): out = BF16(dequant(quant(x))).  MXFP4: E2M1(code) * 2^e, exact in
 //    FP32 and in BF16 (overflow to Inf only for e = 127); FP8: fl32(E4M3(q) * s)
 //    rounded to BF16 (round to nearest even).
+//  * SmoothQuant after the fixed rotation: the block-selection transform is a fixed
+//    Hadamard rotation followed by SmoothQuant [AMD Quark adds native W4A8 ... Wan2.2 --
+//    "Fixed rotation selector" and "Block-level SQNR calibration"].  Per channel k of
+//    the (rotated) values y: activations y_k * (1/lambda_k), weight rows y_k * lambda_k,
+//    so that the product is unchanged.  lambda is the SmoothQuant migration factor
+//    (the pages give no formula; the published SmoothQuant definition is used):
+//      lambda_k = max(ax_k^a / max(aw_k, 1e-5)^(1-a), 1e-5),
+//    ax_k / aw_k = max over rows of |y_k| of the calibration activations / weights,
+//    a = the migration strength.  The multiply is one FP32 product per element,
+//    before the block maximum.
 //  * Scale-factor memory layout (not given by the pages; a reading): rows padded
 //    to a multiple of 128, scale columns to a multiple of 4, 512-byte atoms of
 //    128 rows x 4 scale columns, byte
@@ -245,15 +255,18 @@ static void row_to_float(const uint16_t* xrow, int64_t K, int hadamard, float* y
   }
 }
 
-// MXFP4 quantisation of rows x K BF16 values (row stride ld elements).
+// MXFP4 quantisation of rows x K BF16 values (row stride ld elements), with an optional
+// per-channel multiplier applied after the rotation (chan_scale == nullptr: none).
 // codes: [rows][K/2] bytes, element k in byte k/2, low nibble when k is even.
 // sf_logical: [rows][K/32] E8M0 bytes.
-void oracle_quantize_mxfp4(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, int rule,
-                           int hadamard, uint8_t* codes, uint8_t* sf_logical, int nthreads) {
+static void quantize_rows(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, int rule, int hadamard,
+                          const float* chan_scale, uint8_t* codes, uint8_t* sf_logical, int nthreads) {
   parallel_rows(rows, nthreads, [&](int64_t r0, int64_t r1) {
     std::vector<float> y(static_cast<size_t>(K));
     for (int64_t r = r0; r < r1; ++r) {
       row_to_float(x + r * ld, K, hadamard, y.data());
+      if (chan_scale)
+        for (int64_t k = 0; k < K; ++k) y[k] = y[k] * chan_scale[k];  // fl32 product
       for (int64_t b = 0; b < K / kBlock; ++b) {
         const float* blk = y.data() + b * kBlock;
         double amax = 0.0;
@@ -270,6 +283,42 @@ void oracle_quantize_mxfp4(const uint16_t* x, int64_t rows, int64_t K, int64_t l
       }
     }
   });
+}
+
+void oracle_quantize_mxfp4(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, int rule,
+                           int hadamard, uint8_t* codes, uint8_t* sf_logical, int nthreads) {
+  quantize_rows(x, rows, K, ld, rule, hadamard, nullptr, codes, sf_logical, nthreads);
+}
+
+// The same with SmoothQuant's per-channel multiplier (1/lambda for activations, lambda
+// for weights) applied to the rotated values.
+void oracle_quantize_mxfp4_smooth(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, int rule,
+                                  int hadamard, const float* chan_scale, uint8_t* codes,
+                                  uint8_t* sf_logical, int nthreads) {
+  quantize_rows(x, rows, K, ld, rule, hadamard, chan_scale, codes, sf_logical, nthreads);
+}
+
+// Calibration statistic: amax[k] = max over rows of |y[r][k]| (y rotated or not).
+void oracle_channel_absmax(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, int hadamard,
+                           float* amax) {
+  std::vector<float> y(static_cast<size_t>(K));
+  for (int64_t k = 0; k < K; ++k) amax[k] = 0.0f;
+  for (int64_t r = 0; r < rows; ++r) {
+    row_to_float(x + r * ld, K, hadamard, y.data());
+    for (int64_t k = 0; k < K; ++k) amax[k] = std::max(amax[k], std::fabs(y[k]));
+  }
+}
+
+// SmoothQuant migration factors: lambda[k] = max(ax^a / max(aw, 1e-5)^(1 - a), 1e-5),
+// evaluated in FP64 and rounded once to FP32; inv_lambda[k] = fl32(1 / lambda[k]).
+void oracle_smooth_factors(const float* ax, const float* aw, int64_t K, double alpha, float* lambda,
+                           float* inv_lambda) {
+  for (int64_t k = 0; k < K; ++k) {
+    const double w = std::max(static_cast<double>(aw[k]), 1e-5);
+    const double l = std::max(std::pow(static_cast<double>(ax[k]), alpha) / std::pow(w, 1.0 - alpha), 1e-5);
+    lambda[k] = static_cast<float>(l);
+    inv_lambda[k] = 1.0f / lambda[k];
+  }
 }
 
 // Returns the rotated FP32 values the quantiser sees (for tests).
