@@ -62,6 +62,8 @@ def parse():
     p.add_argument("--workload", choices=["wan_ffn", "wan_attn_hadamard", "flux_w4a8", "m_sweep", "qdq_wan_ffn"],
                    default="wan_ffn")
     p.add_argument("--rule", choices=["ocp", "uos"], default="ocp", help="activation scale rule")
+    p.add_argument("--smooth", action="store_true",
+                   help="SmoothQuant after the rotation (W4A4 workloads; factors calibrated before timing)")
     return p.parse_args()
 
 
@@ -215,7 +217,7 @@ def quant_bytes(M, K, fp8=False):
     return M * K * 2 + (M * K if fp8 else M * K // 2 + M * K // 32)
 
 
-def build_workload(name, dev, M, seed, rule_name):
+def build_workload(name, dev, M, seed, rule_name, smooth=False):
     """Returns (description, parts, inputs [(device tensor)], outputs [(device tensor)], flops per step)."""
     import torch
     from mxfp4_block_scaled_mxq_b200 import inputs, mxq
@@ -229,17 +231,25 @@ def build_workload(name, dev, M, seed, rule_name):
     def out(rows, N):
         return torch.empty(rows, N, dtype=torch.bfloat16, device=dev)
 
-    def w4a4_layer(label, x, w, hadamard, qb=None, share_quant=False):
-        """Parts for quantise(x) (unless shared) + GEMM against packed w."""
+    def w4a4_layer(label, x, w, hadamard, qb=None, share_quant=False, factors=None):
+        """Parts for quantise(x) (unless shared) + GEMM against packed w.  With `smooth`,
+        SmoothQuant factors (lambda, 1/lambda) -- given, or from the channel maxima of x and
+        w (offline calibration) -- are applied after the rotation on both sides."""
         rows, K = x.shape
         N = w.shape[0]
-        wc, wsf = mxq.pack_weight(w, mxq.MXQ_SCALE_OCP, hadamard)
+        if smooth:
+            lam, inv = factors if factors is not None else mxq.smooth_factors(
+                mxq.channel_absmax(x, hadamard), mxq.channel_absmax(w, hadamard), 0.5)
+            wc, wsf = mxq.quantize_smooth(w, lam, mxq.MXQ_SCALE_OCP, hadamard)
+            quant = lambda: mxq.quantize_smooth(x, inv, rule, hadamard, out=qb)
+        else:
+            wc, wsf = mxq.pack_weight(w, mxq.MXQ_SCALE_OCP, hadamard)
+            quant = lambda: mxq.quantize_act(x, rule, hadamard, out=qb)
         qb = qb if qb is not None else qbufs(rows, K)
         d = out(rows, N)
         parts = []
         if not share_quant:
-            parts.append(Part(f"quant_{label}", "quant",
-                              lambda: mxq.quantize_act(x, rule, hadamard, out=qb), nbytes=quant_bytes(rows, K)))
+            parts.append(Part(f"quant_{label}", "quant", quant, nbytes=quant_bytes(rows, K)))
         parts.append(Part(f"gemm_{label}", "gemm",
                           lambda: mxq.gemm_w4a4(qb[0], qb[1], wc, wsf, rows, N, K, out=d),
                           flops=2.0 * rows * N * K))
@@ -259,12 +269,18 @@ def build_workload(name, dev, M, seed, rule_name):
     if name == "wan_attn_hadamard":
         x, ws = inputs.wan_attn(seed=4000 + seed - 2000, device=dev, M=M)
         x_o = inputs.heavy_tailed_bf16(x.shape[0], x.shape[1], seed + 77, device=dev)
-        pq, qb, dq = w4a4_layer("q", x, ws[0], True)
-        pk, _, dk = w4a4_layer("k", x, ws[1], True, qb=qb, share_quant=True)
-        pv, _, dv = w4a4_layer("v", x, ws[2], True, qb=qb, share_quant=True)
+        f_qkv = None
+        if smooth:  # Q, K and V share one quantised X: one lambda from the three weights' maxima
+            aw = torch.maximum(torch.maximum(mxq.channel_absmax(ws[0], True), mxq.channel_absmax(ws[1], True)),
+                               mxq.channel_absmax(ws[2], True))
+            f_qkv = mxq.smooth_factors(mxq.channel_absmax(x, True), aw.contiguous(), 0.5)
+        pq, qb, dq = w4a4_layer("q", x, ws[0], True, factors=f_qkv)
+        pk, _, dk = w4a4_layer("k", x, ws[1], True, qb=qb, share_quant=True, factors=f_qkv)
+        pv, _, dv = w4a4_layer("v", x, ws[2], True, qb=qb, share_quant=True, factors=f_qkv)
         po, _, do = w4a4_layer("o", x_o, ws[3], True)
         parts = pq + pk + pv + po
-        desc = (f"Wan2.2 attention projections W4A4 with 128-point block-Hadamard, Q/K/V/O "
+        desc = (f"Wan2.2 attention projections W4A4 with 128-point block-Hadamard"
+                f"{' + SmoothQuant (alpha 0.5)' if smooth else ''}, Q/K/V/O "
                 f"{x.shape[0]}x5120->5120, {rule_name.upper()} rule")
         return desc, parts, [x, x_o], [dq, dk, dv, do], sum(p.flops for p in parts)
 
@@ -336,7 +352,8 @@ def main():
     default_m = {"wan_ffn": M_TOK, "wan_attn_hadamard": M_TOK, "flux_w4a8": 3584, "m_sweep": 1024,
                  "qdq_wan_ffn": M_TOK}[args.workload]
     M = args.m if args.m else default_m
-    desc, parts, x_in, d_out, flops_step = build_workload(args.workload, dev, M, rank_seed(rank), args.rule)
+    desc, parts, x_in, d_out, flops_step = build_workload(args.workload, dev, M, rank_seed(rank), args.rule,
+                                                          args.smooth)
     stream = torch.cuda.current_stream(dev)
 
     def step():

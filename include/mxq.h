@@ -192,6 +192,48 @@ MXQ_API mxq_status mxq_qdq_act(const void* x_bf16, int64_t M, int64_t K, int64_t
                                float act_scale, void* out_bf16, int64_t ldo, mxq_stream_t stream);
 
 /*
+ * SmoothQuant after the fixed rotation.  The selection transform on the Wan2.2 page is
+ * a fixed Hadamard rotation followed by SmoothQuant (no learned parameters):
+ * [AMD Quark adds native W4A8 ... Wan2.2 -- "Fixed rotation selector" and "Block-level
+ *  SQNR calibration"].  Per channel k of the (rotated) values, activations are
+ * multiplied by 1/lambda_k and weight rows by lambda_k, so X W^T is unchanged while
+ * activation outliers migrate into the weights.  The pages give no formula for lambda;
+ * mxq_smooth_factors uses the published SmoothQuant one (migration strength alpha).
+ *
+ * mxq_channel_absmax -- calibration statistic: amax_out[k] = max over rows of |y[r][k]|
+ * with y = x, or y = x H/sqrt(128) per 128-column chunk when hadamard128 (the rotation
+ * of mxq_quantize_act).  accumulate = 0: amax_out is cleared first (on `stream`);
+ * accumulate != 0: the maxima merge into amax_out's current values (non-negative
+ * FP32), so several calibration batches can be folded in.
+ * x_bf16 / rows / K / ldx as for mxq_quantize_act; amax_out: device [K] FP32, 16-byte
+ * aligned.
+ */
+MXQ_API mxq_status mxq_channel_absmax(const void* x_bf16, int64_t rows, int64_t K, int64_t ldx,
+                                      int hadamard128, int accumulate, float* amax_out,
+                                      mxq_stream_t stream);
+
+/*
+ * mxq_smooth_factors -- lambda[k] = max(amax_x[k]^alpha / max(amax_w[k], 1e-5)^(1-alpha), 1e-5)
+ * in FP32 (powf), inv_lambda[k] = 1 / lambda[k] (IEEE division), for 0 <= alpha <= 1.
+ * amax_x / amax_w: device [K] FP32 channel maxima of the calibration activations and of the
+ * weights (both from mxq_channel_absmax with the same hadamard128).  1 <= K <= 2^22.
+ */
+MXQ_API mxq_status mxq_smooth_factors(const float* amax_x, const float* amax_w, int64_t K, float alpha,
+                                      float* lambda_out, float* inv_lambda_out, mxq_stream_t stream);
+
+/*
+ * mxq_quantize_smooth -- the MXFP4 quantiser of mxq_quantize_act / mxq_pack_weight with one
+ * FP32 multiply per value by chan_scale[k] after the optional rotation and before the
+ * block maximum: codes of (x R)[r][k] * chan_scale[k].  Pass inv_lambda for activations
+ * (every call) and lambda for the weights (offline packing); the W4A4 GEMM then runs
+ * unchanged on the two outputs.  chan_scale: device [K] FP32, 16-byte aligned, finite.
+ * Other arguments, layouts and limits as for mxq_quantize_act (MXFP4).
+ */
+MXQ_API mxq_status mxq_quantize_smooth(const void* x_bf16, int64_t rows, int64_t K, int64_t ldx,
+                                       mxq_scale_rule rule, int hadamard128, const float* chan_scale,
+                                       void* codes_out, void* sf_out, mxq_stream_t stream);
+
+/*
  * mxq_debug_poll -- reads and clears the library's device status word, written by a
  * kernel that gave up one of its bounded waits (each wait on a barrier or a copy is
  * capped at about a second, after which the kernel records MXQ_ERR_TIMEOUT, drains

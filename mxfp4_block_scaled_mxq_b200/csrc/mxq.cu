@@ -391,6 +391,63 @@ mxq_status mxq_qdq_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, mx
   return launch_status();
 }
 
+mxq_status mxq_channel_absmax(const void* x_bf16, int64_t rows, int64_t K, int64_t ldx, int hadamard128,
+                              int accumulate, float* amax_out, mxq_stream_t stream) {
+  if (!amax_out) return MXQ_ERR_INVALID_ARG;
+  // same tiling and limits as the quantiser (the scale pointers are not used)
+  mxq_status st = check_quant_args(x_bf16, rows, K, ldx, MXQ_SCALE_OCP, hadamard128, amax_out, amax_out);
+  if (st != MXQ_OK) return st;
+  DeviceInfo dev;
+  st = current_device(&dev);
+  if (st != MXQ_OK) return st;
+  if (!accumulate && cudaMemsetAsync(amax_out, 0, static_cast<size_t>(K) * sizeof(float), stream) != cudaSuccess)
+    return MXQ_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>((K + 127) / 128), static_cast<unsigned>((rows + 127) / 128));
+  const auto* xp = static_cast<const uint16_t*>(x_bf16);
+  if (hadamard128)
+    mxq::channel_absmax_kernel<true><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ldx, amax_out);
+  else
+    mxq::channel_absmax_kernel<false><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ldx, amax_out);
+  return launch_status();
+}
+
+mxq_status mxq_smooth_factors(const float* amax_x, const float* amax_w, int64_t K, float alpha, float* lambda_out,
+                              float* inv_lambda_out, mxq_stream_t stream) {
+  if (!amax_x || !amax_w || !lambda_out || !inv_lambda_out) return MXQ_ERR_INVALID_ARG;
+  if (!(alpha >= 0.f && alpha <= 1.f)) return MXQ_ERR_INVALID_ARG;
+  if (K < 1 || K > (int64_t(1) << 22)) return MXQ_ERR_SHAPE;
+  DeviceInfo dev;
+  mxq_status st = current_device(&dev);
+  if (st != MXQ_OK) return st;
+  const unsigned blocks = static_cast<unsigned>((K + 255) / 256);
+  mxq::smooth_factors_kernel<<<blocks, 256, 0, stream>>>(amax_x, amax_w, K, alpha, lambda_out, inv_lambda_out);
+  return launch_status();
+}
+
+mxq_status mxq_quantize_smooth(const void* x_bf16, int64_t rows, int64_t K, int64_t ldx, mxq_scale_rule rule,
+                               int hadamard128, const float* chan_scale, void* codes_out, void* sf_out,
+                               mxq_stream_t stream) {
+  if (!chan_scale) return MXQ_ERR_INVALID_ARG;
+  mxq_status st = check_quant_args(x_bf16, rows, K, ldx, rule, hadamard128, codes_out, sf_out);
+  if (st != MXQ_OK) return st;
+  if (!aligned(chan_scale, 16)) return MXQ_ERR_ALIGN;
+  DeviceInfo dev;
+  st = current_device(&dev);
+  if (st != MXQ_OK) return st;
+  const dim3 grid(static_cast<unsigned>((K + 127) / 128), static_cast<unsigned>((rows + 127) / 128));
+  const auto* xp = static_cast<const uint16_t*>(x_bf16);
+  auto* cp = static_cast<uint8_t*>(codes_out);
+  auto* sp = static_cast<uint8_t*>(sf_out);
+  const int sel = (hadamard128 ? 2 : 0) | (rule == MXQ_SCALE_UOS ? 1 : 0);
+  switch (sel) {
+    case 0: mxq::quantize_smooth_mxfp4_kernel<false, false><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ldx, chan_scale, cp, sp); break;
+    case 1: mxq::quantize_smooth_mxfp4_kernel<false, true><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ldx, chan_scale, cp, sp); break;
+    case 2: mxq::quantize_smooth_mxfp4_kernel<true, false><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ldx, chan_scale, cp, sp); break;
+    default: mxq::quantize_smooth_mxfp4_kernel<true, true><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ldx, chan_scale, cp, sp); break;
+  }
+  return launch_status();
+}
+
 mxq_status mxq_debug_poll(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return MXQ_ERR_CUDA;
   unsigned int v = 0;

@@ -131,18 +131,33 @@ __device__ __forceinline__ float exp2_neg(int e) {
 // 2^e for e in [-127, 127].
 __device__ __forceinline__ float exp2_pos(int e) { return exp2_neg(-e); }
 
+// What a quantiser tile produces.
+enum TileOut : int {
+  kOutCodes = 0,   // MXFP4 codes + the tile's 512-byte scale atom
+  kOutQdq = 1,     // BF16(dequant(quant(x))): the quantise-dequantise emulation
+  kOutAbsmax = 2,  // per-channel max |y| over the tile's rows (calibration statistic)
+};
+
+struct TileArgs {
+  uint8_t* codes = nullptr;      // kOutCodes: [rows][K/2]
+  uint8_t* sf = nullptr;         // kOutCodes: swizzled scale bytes
+  uint16_t* qdq = nullptr;       // kOutQdq: BF16 [rows][ldq]
+  int64_t ldq = 0;
+  const float* chan = nullptr;   // kSmooth: per-channel multiplier applied after the rotation
+  float* chan_amax = nullptr;    // kOutAbsmax: FP32 maxima, merged with atomicMax on the bits
+};
+
 // One CTA quantises rows [128*by, +128) x K columns [128*bx, +128) of x[rows][ld]
 // without rotation: codes [rows][K/2] and the tile's 512-byte scale atom (rows beyond
 // `rows` and blocks beyond K stay 0x00 padding).  Thread (warp w, lane l) owns, in iteration i, row
 // 16w + 4i + l/8 and elements [16 * (l%8), +16) of the tile's 128 columns.
-// kQdq: instead of codes and scales, write BF16(dequant(quant(x))) to qdq[rows][ldq]
-// (the quantise-dequantise emulation; the same quantisation arithmetic).
-template <bool kUOS, bool kQdq = false>
+// kOut selects what is written (TileOut); kSmooth multiplies each value by the channel's
+// factor o.chan[k] (one FP32 product) before the block maximum, as SmoothQuant does.
+template <bool kUOS, int kOut = kOutCodes, bool kSmooth = false>
 __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__ x, int64_t rows, int64_t K,
-                                                    int64_t ld, uint8_t* __restrict__ codes,
-                                                    uint8_t* __restrict__ sf, uint16_t* __restrict__ qdq = nullptr,
-                                                    int64_t ldq = 0) {
-  __shared__ __align__(16) uint8_t atom[512];  // byte (r%32)*16 + (r/32)*4 + block
+                                                    int64_t ld, const TileArgs& o) {
+  constexpr bool kQdq = kOut == kOutQdq;
+  __shared__ __align__(16) uint8_t atom[512];  // byte (r%32)*16 + (r/32)*4 + block; column maxima
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int l8 = lane & 7;
@@ -165,13 +180,63 @@ __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__
   }
   __syncthreads();  // atom zeroed
 
+  if constexpr (kOut == kOutAbsmax) {
+    // lanes l, l^8, l^16, l^24 of a warp own the same 16 columns (rows beyond `rows` are 0)
+    uint32_t* cmax = reinterpret_cast<uint32_t*>(atom);  // 128 columns, FP32 bits
+    float cm[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) cm[j] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float f[16];
+      bf16x16_to_float(w[i], f);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) cm[j] = fmaxf(cm[j], fabsf(f[j]));
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      cm[j] = fmaxf(cm[j], __shfl_xor_sync(0xffffffffu, cm[j], 8));
+      cm[j] = fmaxf(cm[j], __shfl_xor_sync(0xffffffffu, cm[j], 16));
+    }
+    if (lane < 8 && k_ok)
+#pragma unroll
+      for (int j = 0; j < 16; ++j) atomicMax(cmax + 16 * l8 + j, __float_as_uint(cm[j]));
+    __syncthreads();
+    const int64_t col = static_cast<int64_t>(blockIdx.x) * 128 + tid;
+    if (tid < 128 && col < K) atomicMax(reinterpret_cast<unsigned int*>(o.chan_amax) + col, cmax[tid]);
+    return;
+  }
+
+  float cm[16];  // kSmooth: this thread's 16 channel factors (the same for all its rows)
+  if constexpr (kSmooth) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = k_ok ? *reinterpret_cast<const float4*>(o.chan + k + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      cm[4 * q] = v.x;
+      cm[4 * q + 1] = v.y;
+      cm[4 * q + 2] = v.z;
+      cm[4 * q + 3] = v.w;
+    }
+  }
+
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = 16 * warp + 4 * i + (lane >> 3);  // row within the tile
     const int64_t row = row0 + r;
     float f[16];
     bf16x16_to_float(w[i], f);
-    uint32_t amax = bf16x16_absmax(w[i]);
+    uint32_t amax;
+    if constexpr (kSmooth) {
+      float m = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        f[j] = __fmul_rn(f[j], cm[j]);
+        m = fmaxf(m, fabsf(f[j]));
+      }
+      amax = __float_as_uint(m);
+    } else {
+      amax = bf16x16_absmax(w[i]);
+    }
     amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));  // the other half of the block
     const int e = block_exponent<kUOS>(amax);
     const float s = exp2_neg(e);  // exact power of two
@@ -191,12 +256,12 @@ __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__
         uint32_t b[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) b[j] = e2m1x2_to_bf16x2((out[j >> 2] >> (8 * (j & 3))) & 0xFFu, up);
-        uint4* dst = reinterpret_cast<uint4*>(qdq + row * ldq + k);
+        uint4* dst = reinterpret_cast<uint4*>(o.qdq + row * o.ldq + k);
         dst[0] = make_uint4(b[0], b[1], b[2], b[3]);
         dst[1] = make_uint4(b[4], b[5], b[6], b[7]);
       }
     } else if (row < rows && k_ok) {
-      *reinterpret_cast<uint2*>(codes + row * (K / 2) + k / 2) = make_uint2(out[0], out[1]);
+      *reinterpret_cast<uint2*>(o.codes + row * (K / 2) + k / 2) = make_uint2(out[0], out[1]);
       if ((l8 & 1) == 0) atom[(r & 31) * 16 + (r >> 5) * 4 + (l8 >> 1)] = static_cast<uint8_t>(e + 127);
     }
   }
@@ -205,7 +270,7 @@ __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__
   if (tid < 32) {
     const int64_t atoms_per_row_tile = (K + 127) / 128;
     const int64_t idx = static_cast<int64_t>(blockIdx.y) * atoms_per_row_tile + blockIdx.x;
-    reinterpret_cast<uint4*>(sf + idx * 512)[tid] = reinterpret_cast<const uint4*>(atom)[tid];
+    reinterpret_cast<uint4*>(o.sf + idx * 512)[tid] = reinterpret_cast<const uint4*>(atom)[tid];
   }
 }
 
@@ -216,12 +281,12 @@ __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__
 // the within-pair butterfly, stride 64 is the one cross-lane exchange (xor 1); the
 // stage order and every rounding are those of the definition, so the rotated values
 // are bit-identical to the element-by-element butterfly.
-template <bool kUOS, bool kQdq = false>
+template <bool kUOS, int kOut = kOutCodes, bool kSmooth = false>
 __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __restrict__ x, int64_t rows,
-                                                             int64_t K, int64_t ld, uint8_t* __restrict__ codes,
-                                                             uint8_t* __restrict__ sf,
-                                                             uint16_t* __restrict__ qdq = nullptr, int64_t ldq = 0) {
+                                                             int64_t K, int64_t ld, const TileArgs& o) {
+  constexpr bool kQdq = kOut == kOutQdq;
   __shared__ __align__(16) uint8_t atom[512];
+  __shared__ __align__(16) float s_chan[kSmooth ? 128 : 1];  // the tile's 128 channel factors
   const int tid = threadIdx.x;
   const int r = tid >> 1;   // row within the tile
   const int half = tid & 1; // elements [64 * half, +64) of the tile's 128 columns
@@ -230,6 +295,11 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
   const bool ok = row < rows;
 
   reinterpret_cast<uint32_t*>(atom)[tid & 127] = 0u;
+  if constexpr (kSmooth) {
+    if (tid < 32)
+      reinterpret_cast<float4*>(s_chan)[tid] =
+          reinterpret_cast<const float4*>(o.chan + static_cast<int64_t>(blockIdx.x) * 128)[tid];
+  }
 
   float2 P[32];
   {
@@ -252,7 +322,7 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
       P[i].y = __uint_as_float((jh & 1) ? (wh & 0xFFFF0000u) : (wh << 16));
     }
   }
-  __syncthreads();  // atom zeroed
+  __syncthreads();  // atom zeroed, channel factors staged
 
   const float2 minus1 = make_float2(-1.f, -1.f);
 #pragma unroll
@@ -281,10 +351,34 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
   }
   const float c = __uint_as_float(kInvSqrt128Bits);
   const float2 cc = make_float2(c, c);
+  if constexpr (kOut == kOutAbsmax) {
+    // column maxima over the 16 rows of this warp with the same `half` (lanes of one
+    // parity), then over the warps in shared memory, then into the global maxima
+    uint32_t* cmax = reinterpret_cast<uint32_t*>(atom);  // 128 columns, FP32 bits
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float a = fabsf(__fmul_rn(P[i].x, c)), b = fabsf(__fmul_rn(P[i].y, c));
+#pragma unroll
+      for (int sh = 2; sh < 32; sh *= 2) {
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, sh));
+        b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, sh));
+      }
+      if ((tid & 31) < 2) {
+        atomicMax(cmax + 64 * half + i, __float_as_uint(a));
+        atomicMax(cmax + 64 * half + 32 + i, __float_as_uint(b));
+      }
+    }
+    __syncthreads();
+    if (tid < 128)
+      atomicMax(reinterpret_cast<unsigned int*>(o.chan_amax) + static_cast<int64_t>(blockIdx.x) * 128 + tid,
+                cmax[tid]);
+    return;
+  }
   float m0 = 0.f, m1 = 0.f;
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     P[i] = __fmul2_rn(P[i], cc);
+    if constexpr (kSmooth) P[i] = __fmul2_rn(P[i], make_float2(s_chan[64 * half + i], s_chan[64 * half + 32 + i]));
     m0 = fmaxf(m0, fabsf(P[i].x));
     m1 = fmaxf(m1, fabsf(P[i].y));
   }
@@ -314,7 +408,7 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           b[j] = e2m1x2_to_bf16x2((out[4 * blk + (j >> 2)] >> (8 * (j & 3))) & 0xFFu, blk ? up1 : up0);
-        uint4* dst = reinterpret_cast<uint4*>(qdq + row * ldq + k + 32 * blk);
+        uint4* dst = reinterpret_cast<uint4*>(o.qdq + row * o.ldq + k + 32 * blk);
 #pragma unroll
         for (int q = 0; q < 4; ++q) dst[q] = make_uint4(b[4 * q], b[4 * q + 1], b[4 * q + 2], b[4 * q + 3]);
       }
@@ -322,7 +416,7 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
     return;  // uniform: no scale atom to write
   }
   if (ok) {
-    uint4* dst = reinterpret_cast<uint4*>(codes + row * (K / 2) + k / 2);  // 16-byte aligned
+    uint4* dst = reinterpret_cast<uint4*>(o.codes + row * (K / 2) + k / 2);  // 16-byte aligned
     dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
     dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
     *reinterpret_cast<uint16_t*>(atom + (r & 31) * 16 + (r >> 5) * 4 + 2 * half) =
@@ -332,18 +426,27 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
   if (tid < 32) {
     const int64_t atoms_per_row_tile = K / 128;
     const int64_t idx = static_cast<int64_t>(blockIdx.y) * atoms_per_row_tile + blockIdx.x;
-    reinterpret_cast<uint4*>(sf + idx * 512)[tid] = reinterpret_cast<const uint4*>(atom)[tid];
+    reinterpret_cast<uint4*>(o.sf + idx * 512)[tid] = reinterpret_cast<const uint4*>(atom)[tid];
   }
+}
+
+template <bool kHadamard, bool kUOS, int kOut, bool kSmooth>
+__device__ __forceinline__ void mxfp4_tile(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ld,
+                                           const TileArgs& o) {
+  if constexpr (kHadamard)
+    quantize_mxfp4_hadamard_tile<kUOS, kOut, kSmooth>(x, rows, K, ld, o);
+  else
+    quantize_mxfp4_tile<kUOS, kOut, kSmooth>(x, rows, K, ld, o);
 }
 
 template <bool kHadamard, bool kUOS>
 __global__ void __launch_bounds__(kQuantThreads) quantize_act_mxfp4_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ldx, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ sf) {
-  if constexpr (kHadamard)
-    quantize_mxfp4_hadamard_tile<kUOS>(x, M, K, ldx, codes, sf);
-  else
-    quantize_mxfp4_tile<kUOS>(x, M, K, ldx, codes, sf);
+  TileArgs o;
+  o.codes = codes;
+  o.sf = sf;
+  mxfp4_tile<kHadamard, kUOS, kOutCodes, false>(x, M, K, ldx, o);
 }
 
 // The offline weight packer: the same block arithmetic on W[N][K] rows.
@@ -351,10 +454,10 @@ template <bool kHadamard, bool kUOS>
 __global__ void __launch_bounds__(kQuantThreads) pack_weight_mxfp4_kernel(
     const uint16_t* __restrict__ w, int64_t N, int64_t K, int64_t ldw, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ sf) {
-  if constexpr (kHadamard)
-    quantize_mxfp4_hadamard_tile<kUOS>(w, N, K, ldw, codes, sf);
-  else
-    quantize_mxfp4_tile<kUOS>(w, N, K, ldw, codes, sf);
+  TileArgs o;
+  o.codes = codes;
+  o.sf = sf;
+  mxfp4_tile<kHadamard, kUOS, kOutCodes, false>(w, N, K, ldw, o);
 }
 
 // Quantise-dequantise emulation of the MXFP4 activation quantiser (BF16 out).
@@ -362,10 +465,44 @@ template <bool kHadamard, bool kUOS>
 __global__ void __launch_bounds__(kQuantThreads) qdq_act_mxfp4_kernel(const uint16_t* __restrict__ x, int64_t M,
                                                                        int64_t K, int64_t ldx,
                                                                        uint16_t* __restrict__ out, int64_t ldo) {
-  if constexpr (kHadamard)
-    quantize_mxfp4_hadamard_tile<kUOS, true>(x, M, K, ldx, nullptr, nullptr, out, ldo);
-  else
-    quantize_mxfp4_tile<kUOS, true>(x, M, K, ldx, nullptr, nullptr, out, ldo);
+  TileArgs o;
+  o.qdq = out;
+  o.ldq = ldo;
+  mxfp4_tile<kHadamard, kUOS, kOutQdq, false>(x, M, K, ldx, o);
+}
+
+// SmoothQuant after the (optional) rotation: codes of (x R) * chan per channel.  Serves
+// activations (chan = 1/lambda) and the offline weight packer (chan = lambda).
+template <bool kHadamard, bool kUOS>
+__global__ void __launch_bounds__(kQuantThreads) quantize_smooth_mxfp4_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ld, const float* __restrict__ chan,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  TileArgs o;
+  o.codes = codes;
+  o.sf = sf;
+  o.chan = chan;
+  mxfp4_tile<kHadamard, kUOS, kOutCodes, true>(x, rows, K, ld, o);
+}
+
+// Calibration statistic: amax[k] = max(amax[k], max over rows of |(x R)[r][k]|).
+template <bool kHadamard>
+__global__ void __launch_bounds__(kQuantThreads) channel_absmax_kernel(const uint16_t* __restrict__ x,
+                                                                        int64_t rows, int64_t K, int64_t ld,
+                                                                        float* __restrict__ amax) {
+  TileArgs o;
+  o.chan_amax = amax;
+  mxfp4_tile<kHadamard, false, kOutAbsmax, false>(x, rows, K, ld, o);
+}
+
+// SmoothQuant migration factors, one thread per channel:
+// lambda = max(ax^a / max(aw, 1e-5)^(1-a), 1e-5), inv_lambda = 1 / lambda (IEEE division).
+__global__ void smooth_factors_kernel(const float* __restrict__ ax, const float* __restrict__ aw, int64_t K,
+                                      float alpha, float* __restrict__ lambda, float* __restrict__ inv_lambda) {
+  const int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (k >= K) return;
+  const float l = fmaxf(__fdiv_rn(powf(ax[k], alpha), powf(fmaxf(aw[k], 1e-5f), 1.0f - alpha)), 1e-5f);
+  lambda[k] = l;
+  inv_lambda[k] = __fdiv_rn(1.0f, l);
 }
 
 // MXFP4 -> BF16: a unit of work is 16 elements (8 code bytes + their scale byte from the

@@ -24,7 +24,8 @@ MXQ_SCALE_OCP, MXQ_SCALE_UOS = 0, 1
 MXQ_ACT_MXFP4, MXQ_ACT_FP8_E4M3 = 0, 1
 
 EXPORTED = ("mxq_status_string", "mxq_sf_bytes", "mxq_quantize_act", "mxq_pack_weight", "mxq_gemm_w4a4",
-            "mxq_gemm_w4a8", "mxq_dequant_mxfp4", "mxq_qdq_act", "mxq_debug_poll")
+            "mxq_gemm_w4a8", "mxq_dequant_mxfp4", "mxq_qdq_act", "mxq_channel_absmax", "mxq_smooth_factors",
+            "mxq_quantize_smooth", "mxq_debug_poll")
 
 
 class MxqError(RuntimeError):
@@ -61,6 +62,12 @@ def lib() -> ctypes.CDLL:
     L.mxq_dequant_mxfp4.restype = I32
     L.mxq_qdq_act.argtypes = [P, I64, I64, I64, I32, I32, I32, F32, P, I64, P]
     L.mxq_qdq_act.restype = I32
+    L.mxq_channel_absmax.argtypes = [P, I64, I64, I64, I32, I32, P, P]
+    L.mxq_channel_absmax.restype = I32
+    L.mxq_smooth_factors.argtypes = [P, P, I64, F32, P, P, P]
+    L.mxq_smooth_factors.restype = I32
+    L.mxq_quantize_smooth.argtypes = [P, I64, I64, I64, I32, I32, P, P, P, P]
+    L.mxq_quantize_smooth.restype = I32
     L.mxq_debug_poll.argtypes = []
     L.mxq_debug_poll.restype = I32
     _lib = L
@@ -129,6 +136,22 @@ def mxq_dequant_mxfp4(codes, sf, rows, K, out, ldo, stream=None) -> None:
 def mxq_qdq_act(x, M, K, ldx, fmt, rule, hadamard128, act_scale, out, ldo, stream=None) -> None:
     _check(lib().mxq_qdq_act(_ptr(x), int(M), int(K), int(ldx), int(fmt), int(rule), int(bool(hadamard128)),
                              float(act_scale), _ptr(out), int(ldo), _stream(stream)), "mxq_qdq_act")
+
+
+def mxq_channel_absmax(x, rows, K, ldx, hadamard128, accumulate, amax_out, stream=None) -> None:
+    _check(lib().mxq_channel_absmax(_ptr(x), int(rows), int(K), int(ldx), int(bool(hadamard128)),
+                                    int(bool(accumulate)), _ptr(amax_out), _stream(stream)), "mxq_channel_absmax")
+
+
+def mxq_smooth_factors(amax_x, amax_w, K, alpha, lambda_out, inv_lambda_out, stream=None) -> None:
+    _check(lib().mxq_smooth_factors(_ptr(amax_x), _ptr(amax_w), int(K), float(alpha), _ptr(lambda_out),
+                                    _ptr(inv_lambda_out), _stream(stream)), "mxq_smooth_factors")
+
+
+def mxq_quantize_smooth(x, rows, K, ldx, rule, hadamard128, chan_scale, codes_out, sf_out, stream=None) -> None:
+    _check(lib().mxq_quantize_smooth(_ptr(x), int(rows), int(K), int(ldx), int(rule), int(bool(hadamard128)),
+                                     _ptr(chan_scale), _ptr(codes_out), _ptr(sf_out), _stream(stream)),
+           "mxq_quantize_smooth")
 
 
 def mxq_debug_poll() -> int:
@@ -214,6 +237,39 @@ def qdq_act(x: torch.Tensor, fmt: int = MXQ_ACT_MXFP4, rule: int = MXQ_SCALE_OCP
     mxq_qdq_act(x.data_ptr(), M, K, x.stride(0), fmt, rule, hadamard128, act_scale, o.data_ptr(), o.stride(0),
                 stream)
     return o
+
+
+def channel_absmax(x: torch.Tensor, hadamard128: bool = False, out=None, accumulate: bool = False,
+                   stream=None) -> torch.Tensor:
+    """Per-channel max |x R| over the rows (FP32 [K]); accumulate merges into `out`."""
+    x = _bf16_2d(x, "x")
+    rows, K = x.shape
+    o = torch.empty(K, dtype=torch.float32, device=x.device) if out is None else out
+    mxq_channel_absmax(x.data_ptr(), rows, K, x.stride(0), hadamard128, accumulate, o, stream)
+    return o
+
+
+def smooth_factors(amax_x: torch.Tensor, amax_w: torch.Tensor, alpha: float = 0.5, stream=None):
+    """SmoothQuant (lambda, 1/lambda) from the channel maxima of activations and weights."""
+    K = amax_x.numel()
+    lam = torch.empty(K, dtype=torch.float32, device=amax_x.device)
+    inv = torch.empty_like(lam)
+    mxq_smooth_factors(amax_x, amax_w, K, alpha, lam, inv, stream)
+    return lam, inv
+
+
+def quantize_smooth(x: torch.Tensor, chan_scale: torch.Tensor, rule: int = MXQ_SCALE_OCP,
+                    hadamard128: bool = False, out=None, stream=None):
+    """MXFP4 codes + scales of (x R) * chan_scale (per channel): 1/lambda for activations,
+    lambda for weights."""
+    x = _bf16_2d(x, "x")
+    rows, K = x.shape
+    if out is None:
+        out = (torch.empty(rows, K // 2, dtype=torch.uint8, device=x.device),
+               torch.empty(mxq_sf_bytes(rows, K), dtype=torch.uint8, device=x.device))
+    q, sf = out
+    mxq_quantize_smooth(x.data_ptr(), rows, K, x.stride(0), rule, hadamard128, chan_scale, q, sf, stream)
+    return q, sf
 
 
 def linear_w4a4(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE_OCP, hadamard128: bool = False,

@@ -130,6 +130,25 @@ def test_dequant_and_qdq_validation_happens_before_any_launch(L):
     assert qq(FAKE, 4, 64, 64, 0, 0, 0, 1.0, FAKE, 68, None) == ALIGN        # ldo % 8
 
 
+def test_smoothing_validation_happens_before_any_launch(L):
+    INV, SHAPE, ALIGN = 1, 2, 3
+    ca = lambda *a: L.mxq_channel_absmax(*a)
+    assert ca(FAKE, 4, 64, 64, 0, 0, None, None) == INV                      # null output
+    assert ca(None, 4, 64, 64, 0, 0, FAKE, None) == INV
+    assert ca(FAKE, 4, 96, 96, 1, 0, FAKE, None) == SHAPE                    # hadamard needs K % 128
+    assert ca(FAKE, 4, 64, 64, 0, 0, FAKE + 4, None) == ALIGN
+    sf = lambda *a: L.mxq_smooth_factors(*a)
+    assert sf(FAKE, FAKE, 64, 1.5, FAKE, FAKE, None) == INV                  # alpha outside [0, 1]
+    assert sf(FAKE, FAKE, 64, float("nan"), FAKE, FAKE, None) == INV
+    assert sf(FAKE, None, 64, 0.5, FAKE, FAKE, None) == INV
+    assert sf(FAKE, FAKE, 0, 0.5, FAKE, FAKE, None) == SHAPE
+    qs = lambda *a: L.mxq_quantize_smooth(*a)
+    assert qs(FAKE, 4, 64, 64, 0, 0, None, FAKE, FAKE, None) == INV          # null factors
+    assert qs(FAKE, 4, 64, 64, 0, 0, FAKE + 8, FAKE, FAKE, None) == ALIGN    # factors 16-byte aligned
+    assert qs(FAKE, 4, 64, 64, 2, 0, FAKE, FAKE, FAKE, None) == INV          # bad rule
+    assert qs(FAKE, 4, 48, 48, 0, 0, FAKE, FAKE, FAKE, None) == SHAPE
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
