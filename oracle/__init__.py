@@ -106,6 +106,12 @@ def _load():
     lib.oracle_channel_absmax.restype = None
     lib.oracle_smooth_factors.argtypes = [P, P, I64, ctypes.c_double, P, P]
     lib.oracle_smooth_factors.restype = None
+    lib.oracle_sqnr_sums.argtypes = [P, P, I64, P]
+    lib.oracle_sqnr_sums.restype = None
+    lib.oracle_sqnr_db.argtypes = [ctypes.c_double, ctypes.c_double]
+    lib.oracle_sqnr_db.restype = ctypes.c_double
+    lib.oracle_select_precision.argtypes = [ctypes.c_double] * 4
+    lib.oracle_select_precision.restype = ctypes.c_int
     lib.oracle_gemm.argtypes = [ctypes.c_int, P, P, I64, P, P, I64, I64, ctypes.c_double, P, P, I64,
                                 P, ctypes.c_int]
     lib.oracle_gemm.restype = None
@@ -320,3 +326,26 @@ def smooth_factors(ax: np.ndarray, aw: np.ndarray, alpha: float = 0.5):
     inv = np.empty(K, np.float32)
     _load().oracle_smooth_factors(_ptr(ax), _ptr(aw), K, float(alpha), _ptr(lam), _ptr(inv))
     return lam, inv
+
+
+# ---------------------------------------------------------------- precision selection
+PREC_W4A4, PREC_W4A4_TRANSFORM, PREC_W4A8, PREC_BF16 = 0, 1, 2, 3
+
+
+def sqnr_sums(y: np.ndarray, ref: np.ndarray):
+    """(sum ref^2, sum (y - ref)^2) in FP64."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    ref = np.ascontiguousarray(ref, dtype=np.float64)
+    assert y.shape == ref.shape
+    out = np.empty(2, np.float64)
+    _load().oracle_sqnr_sums(_ptr(y), _ptr(ref), y.size, _ptr(out))
+    return float(out[0]), float(out[1])
+
+
+def sqnr_db(signal: float, noise: float) -> float:
+    return float(_load().oracle_sqnr_db(float(signal), float(noise)))
+
+
+def select_precision(sqnr_plain_db: float, sqnr_transform_db: float, high_db: float, low_db: float) -> int:
+    return int(_load().oracle_select_precision(float(sqnr_plain_db), float(sqnr_transform_db), float(high_db),
+                                               float(low_db)))

@@ -51,6 +51,13 @@
 //    ax_k / aw_k = max over rows of |y_k| of the calibration activations / weights,
 //    a = the migration strength.  The multiply is one FP32 product per element,
 //    before the block maximum.
+//  * Per-layer precision selection [AMD Quark adds native W4A8 ... Wan2.2 -- "Block-level
+//    SQNR calibration"]: the output SQNR against the BF16 layer,
+//      SQNR = 10 log10( sum ref^2 / sum (y - ref)^2 )  dB,
+//    measured with plain MXFP4 and with the transform (rotation + SmoothQuant), then
+//    tiered thresholds (values not on the pages; parameters): plain >= high -> plain W4A4;
+//    else transform >= high -> transform-enabled W4A4; else the better of the two >= low
+//    -> W4A8 promotion; else BF16 fallback.
 //  * Scale-factor memory layout (not given by the pages; a reading): rows padded
 //    to a multiple of 128, scale columns to a multiple of 4, 512-byte atoms of
 //    128 rows x 4 scale columns, byte
@@ -437,6 +444,34 @@ void oracle_gemm(int a_kind, const uint8_t* a_codes, const uint8_t* a_sf, int64_
     }
   });
   (void)M;
+}
+
+// ---------------------------------------------------------------- precision selection
+
+// signal_noise[0] = sum ref^2, signal_noise[1] = sum (y - ref)^2 over n values (FP64).
+void oracle_sqnr_sums(const double* y, const double* ref, int64_t n, double* signal_noise) {
+  double s = 0.0, e = 0.0;
+  for (int64_t i = 0; i < n; ++i) {
+    s += ref[i] * ref[i];
+    const double d = y[i] - ref[i];
+    e += d * d;
+  }
+  signal_noise[0] = s;
+  signal_noise[1] = e;
+}
+
+double oracle_sqnr_db(double signal, double noise) {
+  if (noise <= 0.0) return HUGE_VAL;
+  if (signal <= 0.0) return -HUGE_VAL;
+  return 10.0 * std::log10(signal / noise);
+}
+
+// 0 = plain W4A4, 1 = transform-enabled W4A4 (rotation + SmoothQuant), 2 = W4A8, 3 = BF16.
+int oracle_select_precision(double sqnr_plain_db, double sqnr_transform_db, double high_db, double low_db) {
+  if (sqnr_plain_db >= high_db) return 0;
+  if (sqnr_transform_db >= high_db) return 1;
+  if (std::max(sqnr_plain_db, sqnr_transform_db) >= low_db) return 2;
+  return 3;
 }
 
 }  // extern "C"
