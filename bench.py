@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 METRIC = "MXFP4 W4A4 GEMM TFLOPS incl. act-quant and % of B200 dense FP4 peak"
 METRIC_W4A8 = "MXFP4 W4A8 GEMM TFLOPS incl. act-quant and % of B200 dense FP8 peak"
 METRIC_QDQ = "MXFP4 quantise-dequantise + weight dequantisation GB/s (HBM-bound)"
+METRIC_POLICY = "precision-selection pass (plain + rotation/SmoothQuant W4A4 vs BF16 SQNR), ms per Wan FFN block"
 UNIT = "TFLOP/s"
 NOMINAL_FP4_TFLOPS = 9000.0          # dense FP4, nominal
 NOMINAL_FP8_TFLOPS = 4500.0          # dense FP8, nominal (kind::mxf8f6f4 runs at the FP8 rate)
@@ -44,7 +45,8 @@ FP8_PER_BF16 = 2.0                   # nominal FP8 : BF16 dense ratio (4.5 / 2.2
 TRAFFIC = {"wan_ffn": (241.4e6 + 867.0e6 + 345.3e6 + 314.8e6) / 2}
 # Packed weight bytes per workload (MXFP4 codes + scales), for the L2-residency decision.
 W_BYTES = {"wan_ffn": 2 * 5120 * 13824 * 17 // 32, "wan_attn_hadamard": 4 * 5120 * 5120 * 17 // 32,
-           "flux_w4a8": (9216 + 12288) * 3072 * 17 // 32, "m_sweep": 13824 * 5120 * 17 // 32, "qdq_wan_ffn": 0}
+           "flux_w4a8": (9216 + 12288) * 3072 * 17 // 32, "m_sweep": 13824 * 5120 * 17 // 32, "qdq_wan_ffn": 0,
+           "policy_wan_ffn": 0}
 WORKLOAD = "Wan2.2-A14B FFN W4A4 (up 32760x5120->13824, down 32760x13824->5120), dynamic MXFP4 acts, OCP rule"
 M_TOK, D_MODEL, D_FF = 32760, 5120, 13824
 
@@ -59,7 +61,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--m", type=int, default=0, help="token count (0: the workload's own)")
-    p.add_argument("--workload", choices=["wan_ffn", "wan_attn_hadamard", "flux_w4a8", "m_sweep", "qdq_wan_ffn"],
+    p.add_argument("--workload", choices=["wan_ffn", "wan_attn_hadamard", "flux_w4a8", "m_sweep", "qdq_wan_ffn",
+                                          "policy_wan_ffn"],
                    default="wan_ffn")
     p.add_argument("--rule", choices=["ocp", "uos"], default="ocp", help="activation scale rule")
     p.add_argument("--smooth", action="store_true",
@@ -206,10 +209,13 @@ def whole_job_rate(flops_per_step: float, steps: int, world: int, max_ms: float)
 
 # ------------------------------------------------------------------ workloads
 class Part:
-    """One kernel launch of the step: kind 'quant' (HBM-bound) or 'gemm' (tensor-bound)."""
+    """One launch of the step: kind 'quant' (HBM-bound), 'gemm' (tensor-bound), 'lib' (a library
+    kernel, e.g. the cuBLAS BF16 reference) or 'other' (small reductions)."""
 
-    def __init__(self, label, kind, fn, flops=0.0, nbytes=0.0, peak_kind="fp4"):
+    def __init__(self, label, kind, fn, flops=0.0, nbytes=0.0, peak_kind="fp4", launches=None):
         self.label, self.kind, self.fn, self.flops, self.nbytes, self.peak_kind = label, kind, fn, flops, nbytes, peak_kind
+        # kernels of this library the part launches ("lib" parts run a library kernel)
+        self.launches = launches if launches is not None else (0 if kind == "lib" else 1)
 
 
 def quant_bytes(M, K, fp8=False):
@@ -323,6 +329,55 @@ def build_workload(name, dev, M, seed, rule_name, smooth=False):
                 f"and expand packed W_up {N}x{K} to BF16")
         return desc, parts, [x], [d_x, d_w], 0.0
 
+    if name == "policy_wan_ffn":
+        # One selection pass over the FFN block on a calibration batch: the BF16 layers
+        # (cuBLAS), both conditions' weight packing, quantisation and W4A4 GEMMs, the
+        # SmoothQuant calibration, and the SQNR sums.
+        parts, xs, outs = [], [], []
+        acc = torch.zeros(4, dtype=torch.float64, device=dev)
+        flops = 0.0
+        for label in ("up", "down"):
+            x, w = inputs.wan_ffn(seed=seed, which=label, device=dev, M=M)
+            rows, K = x.shape
+            N = w.shape[0]
+            xs.append(x)
+            ref, y1, y2 = out(rows, N), out(rows, N), out(rows, N)
+            outs += [ref, y1, y2]
+            wq, q1, wq2, q2 = qbufs(N, K), qbufs(rows, K), qbufs(N, K), qbufs(rows, K)
+            ax = torch.empty(K, dtype=torch.float32, device=dev)
+            aw = torch.empty_like(ax)
+            lam, inv = torch.empty_like(ax), torch.empty_like(ax)
+            f = 2.0 * rows * N * K
+            flops += 2 * f
+
+            def sq(y, a):
+                return lambda: mxq.mxq_sqnr_accumulate(y.data_ptr(), y.stride(0), ref.data_ptr(), ref.stride(0),
+                                                       rows, N, True, a)
+            parts += [
+                Part(f"bf16_ref_{label}", "lib", lambda x=x, w=w, ref=ref: torch.matmul(x, w.t(), out=ref), flops=f),
+                Part(f"pack_{label}", "quant", lambda w=w, wq=wq: mxq.mxq_pack_weight(
+                    w.data_ptr(), N, K, K, mxq.MXQ_SCALE_OCP, False, wq[0], wq[1]), nbytes=quant_bytes(N, K)),
+                Part(f"quant_{label}", "quant", lambda x=x, q1=q1: mxq.quantize_act(x, rule, out=q1),
+                     nbytes=quant_bytes(rows, K)),
+                Part(f"gemm_{label}", "gemm", lambda q1=q1, wq=wq, y1=y1: mxq.gemm_w4a4(
+                    q1[0], q1[1], wq[0], wq[1], rows, N, K, out=y1), flops=f),
+                Part(f"sqnr_plain_{label}", "other", sq(y1, acc[0:2])),
+                Part(f"absmax_{label}", "other", lambda x=x, w=w, ax=ax, aw=aw: (
+                    mxq.channel_absmax(x, True, out=ax), mxq.channel_absmax(w, True, out=aw)), launches=2),
+                Part(f"factors_{label}", "other", lambda ax=ax, aw=aw, lam=lam, inv=inv: mxq.mxq_smooth_factors(
+                    ax, aw, K, 0.5, lam, inv)),
+                Part(f"pack_smooth_{label}", "quant", lambda w=w, lam=lam, wq2=wq2: mxq.quantize_smooth(
+                    w, lam, mxq.MXQ_SCALE_OCP, True, out=wq2), nbytes=quant_bytes(N, K)),
+                Part(f"quant_smooth_{label}", "quant", lambda x=x, inv=inv, q2=q2: mxq.quantize_smooth(
+                    x, inv, rule, True, out=q2), nbytes=quant_bytes(rows, K)),
+                Part(f"gemm_smooth_{label}", "gemm", lambda q2=q2, wq2=wq2, y2=y2: mxq.gemm_w4a4(
+                    q2[0], q2[1], wq2[0], wq2[1], rows, N, K, out=y2), flops=f),
+                Part(f"sqnr_transform_{label}", "other", sq(y2, acc[2:4])),
+            ]
+        desc = (f"selection pass on the Wan2.2 FFN block (up 5120->13824, down 13824->5120), calibration batch "
+                f"M={M}: BF16 reference, plain and rotation+SmoothQuant W4A4, SQNR sums")
+        return desc, parts, xs, outs, flops
+
     raise ValueError(f"unknown workload {name}")
 
 
@@ -350,7 +405,7 @@ def main():
 
     # Inputs (per rank its own token batch); weights packed once before timing.
     default_m = {"wan_ffn": M_TOK, "wan_attn_hadamard": M_TOK, "flux_w4a8": 3584, "m_sweep": 1024,
-                 "qdq_wan_ffn": M_TOK}[args.workload]
+                 "qdq_wan_ffn": M_TOK, "policy_wan_ffn": 4096}[args.workload]
     M = args.m if args.m else default_m
     desc, parts, x_in, d_out, flops_step = build_workload(args.workload, dev, M, rank_seed(rank), args.rule,
                                                           args.smooth)
@@ -412,8 +467,11 @@ def main():
         dist.barrier()
         ms = max_over_ranks(ms, dist, dev)
     hbm_only = flops_step == 0.0
+    time_metric = args.workload == "policy_wan_ffn"
     bytes_step = sum(p.nbytes for p in parts)
-    if hbm_only:  # GB/s: bytes per step instead of flops
+    if time_metric:  # ms per step (per block), the slowest rank's
+        value = ms / args.steps
+    elif hbm_only:  # GB/s: bytes per step instead of flops
         value = whole_job_rate(bytes_step, args.steps, world, ms) * 1e3
     else:
         value = whole_job_rate(flops_step, args.steps, world, ms)
@@ -435,10 +493,12 @@ def main():
     peak_of = {"fp4": peaks["bf16_tflops"] * FP4_PER_BF16, "fp8": peaks["bf16_tflops"] * FP8_PER_BF16}
     parts_out = {}
     for p, t in zip(parts, part_ms):
-        if p.kind == "gemm":
+        if p.kind in ("gemm", "lib"):
             parts_out[p.label] = {"ms": t, "tflops": p.flops / (t / 1e3) / 1e12}
-        else:
+        elif p.kind == "quant":
             parts_out[p.label] = {"ms": t, "gbs": p.nbytes / (t / 1e3) / 1e9}
+        else:
+            parts_out[p.label] = {"ms": t}
     gemm_t = sum(t for p, t in zip(parts, part_ms) if p.kind == "gemm")
     quant_t = sum(t for p, t in zip(parts, part_ms) if p.kind == "quant")
     gemm_parts = [p for p in parts if p.kind == "gemm"]
@@ -467,10 +527,11 @@ def main():
                     "traffic": None}
     nominal = NOMINAL_FP4_TFLOPS if gemm_kind == "fp4" else NOMINAL_FP8_TFLOPS
     result = {
-        "metric": (METRIC_QDQ if hbm_only else
+        "metric": (METRIC_POLICY if time_metric else METRIC_QDQ if hbm_only else
                    METRIC if args.workload in ("wan_ffn", "m_sweep", "wan_attn_hadamard") else METRIC_W4A8),
-        "value": value, "unit": "GB/s" if hbm_only else UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "value": value, "unit": "ms" if time_metric else "GB/s" if hbm_only else UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": not time_metric, "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16 <-> mxfp4 (e2m1 x e8m0)" if hbm_only else "mxfp4 (e2m1 x e8m0, fp32 accumulate)"
                  if gemm_kind == "fp4"
@@ -480,14 +541,14 @@ def main():
                    "l2": (f"working set {working_set / 1e6:.0f} MB < 4x L2: L2 flushed (untimed) before every "
                           f"timed step" if flush else f"working set {working_set / 1e9:.2f} GB > L2, steps back to back"),
                    "timing": "step captured in one CUDA graph, replayed; CUDA events on the launching stream"},
-        "pct_of_dense_peak": None if hbm_only else 100.0 * value / world / nominal,
+        "pct_of_dense_peak": None if hbm_only or time_metric else 100.0 * value / world / nominal,
         "roofline": roofline,
         "gemm": None if hbm_only else {"achieved": achieved_g, "unit": "TFLOP/s", "peak": peak_of[gemm_kind],
                                        "frac": achieved_g / peak_of[gemm_kind]},
         "quantizer": ({"achieved": achieved_q, "unit": "GB/s", "peak": peaks["hbm_gbs"],
                        "frac": achieved_q / peaks["hbm_gbs"]} if quant_parts else None),
         "parts": parts_out,
-        "gpu_launches": len(parts) * args.steps,
+        "gpu_launches": sum(p.launches for p in parts) * args.steps,
         "clocks": clocks.summary(),
     }
 
@@ -516,9 +577,10 @@ def main():
         ems = e0.elapsed_time(e1)
         if world > 1:
             ems = max_over_ranks(ems, dist, dev)
-        e2e_value = (whole_job_rate(bytes_step, args.e2e_steps, world, ems) * 1e3 if hbm_only
+        e2e_value = (ems / args.e2e_steps if time_metric else
+                     whole_job_rate(bytes_step, args.e2e_steps, world, ems) * 1e3 if hbm_only
                      else whole_job_rate(flops_step, args.e2e_steps, world, ems))
-        result["e2e"] = {"value": e2e_value, "unit": "GB/s" if hbm_only else UNIT,
+        result["e2e"] = {"value": e2e_value, "unit": "ms" if time_metric else "GB/s" if hbm_only else UNIT,
                          "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h in hin),
                          "d2h_bytes_per_step": sum(h.numel() * h.element_size() for h in hout),
                          "steps": args.e2e_steps}

@@ -84,6 +84,13 @@ typedef enum {
   MXQ_ACT_FP8_E4M3 = 1 /* static per-tensor FP8 E4M3 activations (W4A8) */
 } mxq_act_format;
 
+typedef enum {
+  MXQ_PREC_W4A4 = 0,           /* plain MXFP4 weights and activations                  */
+  MXQ_PREC_W4A4_TRANSFORM = 1, /* W4A4 with the fixed rotation + SmoothQuant            */
+  MXQ_PREC_W4A8 = 2,           /* promotion: MXFP4 weights, static FP8 E4M3 activations */
+  MXQ_PREC_BF16 = 3            /* fallback: the layer stays in BF16                     */
+} mxq_precision;
+
 /* Human-readable name of a status code (static string, never NULL). */
 MXQ_API const char* mxq_status_string(mxq_status status);
 
@@ -232,6 +239,35 @@ MXQ_API mxq_status mxq_smooth_factors(const float* amax_x, const float* amax_w, 
 MXQ_API mxq_status mxq_quantize_smooth(const void* x_bf16, int64_t rows, int64_t K, int64_t ldx,
                                        mxq_scale_rule rule, int hadamard128, const float* chan_scale,
                                        void* codes_out, void* sf_out, mxq_stream_t stream);
+
+/*
+ * Per-layer precision selection.  The Wan2.2 page selects each block's precision from its
+ * whole-block output SQNR against BF16, measured with plain MXFP4 and with the transform
+ * (fixed rotation + SmoothQuant), through tiered thresholds: plain W4A4, W4A8 promotion,
+ * transform-enabled W4A4 or BF16 fallback.  [AMD Quark adds native W4A8 ... Wan2.2 --
+ * "Block-level SQNR calibration"]  The threshold values are not on the pages: they are
+ * parameters.
+ *
+ * mxq_sqnr_accumulate -- acc[0] += sum ref^2, acc[1] += sum (y - ref)^2 over M x N BF16
+ * values (y: the quantised layer's output, ref: the BF16 layer's), in FP64 on the device.
+ * accumulate = 0 clears acc first (on `stream`); != 0 adds to it, so the layers of a block
+ * sum into one SQNR.  y_bf16 / ref_bf16: device [M][ldy] / [M][ldr], 16-byte aligned,
+ * ldy, ldr >= N and multiples of 8; acc: device double[2].  The FP64 addition order varies
+ * between runs (atomics), so the sums do in their last bits.
+ */
+MXQ_API mxq_status mxq_sqnr_accumulate(const void* y_bf16, int64_t ldy, const void* ref_bf16,
+                                       int64_t ldr, int64_t M, int64_t N, int accumulate, double* acc,
+                                       mxq_stream_t stream);
+
+/* 10 log10(signal / noise) dB; +HUGE_VAL when noise == 0, -HUGE_VAL when signal == 0.
+ * Host-only (no device access). */
+MXQ_API double mxq_sqnr_db(double signal, double noise);
+
+/* The tier decision, host-only: plain >= high_db -> MXQ_PREC_W4A4; else transform >= high_db
+ * -> MXQ_PREC_W4A4_TRANSFORM; else max(plain, transform) >= low_db -> MXQ_PREC_W4A8; else
+ * MXQ_PREC_BF16 (SQNRs in dB, ties pass). */
+MXQ_API mxq_precision mxq_select_precision(double sqnr_plain_db, double sqnr_transform_db,
+                                           double high_db, double low_db);
 
 /*
  * mxq_debug_poll -- reads and clears the library's device status word, written by a

@@ -12,6 +12,7 @@
 #include "gemm_common.cuh"
 #include "gemm_pair.cuh"
 #include "gemm_swap.cuh"
+#include "policy.cuh"
 #include "quantize.cuh"
 
 namespace {
@@ -446,6 +447,39 @@ mxq_status mxq_quantize_smooth(const void* x_bf16, int64_t rows, int64_t K, int6
     default: mxq::quantize_smooth_mxfp4_kernel<true, true><<<grid, mxq::kQuantThreads, 0, stream>>>(xp, rows, K, ldx, chan_scale, cp, sp); break;
   }
   return launch_status();
+}
+
+mxq_status mxq_sqnr_accumulate(const void* y_bf16, int64_t ldy, const void* ref_bf16, int64_t ldr, int64_t M,
+                               int64_t N, int accumulate, double* acc, mxq_stream_t stream) {
+  if (!y_bf16 || !ref_bf16 || !acc) return MXQ_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || M > (int64_t(1) << 31) || N > (int64_t(1) << 31)) return MXQ_ERR_SHAPE;
+  if (ldy < N || ldr < N || ldy % 8 != 0 || ldr % 8 != 0) return MXQ_ERR_ALIGN;
+  if (!aligned(y_bf16, 16) || !aligned(ref_bf16, 16) || !aligned(acc, 8)) return MXQ_ERR_ALIGN;
+  DeviceInfo dev;
+  mxq_status st = current_device(&dev);
+  if (st != MXQ_OK) return st;
+  if (!accumulate && cudaMemsetAsync(acc, 0, 2 * sizeof(double), stream) != cudaSuccess) return MXQ_ERR_CUDA;
+  const int64_t chunks = M * ((N + 7) / 8);
+  int64_t blocks = (chunks + mxq::kSqnrThreads - 1) / mxq::kSqnrThreads;
+  const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;
+  if (blocks > cap) blocks = cap;
+  mxq::sqnr_sums_kernel<<<static_cast<unsigned>(blocks), mxq::kSqnrThreads, 0, stream>>>(
+      static_cast<const uint16_t*>(y_bf16), ldy, static_cast<const uint16_t*>(ref_bf16), ldr, M, N, acc);
+  return launch_status();
+}
+
+double mxq_sqnr_db(double signal, double noise) {
+  if (!(noise > 0.0)) return HUGE_VAL;
+  if (!(signal > 0.0)) return -HUGE_VAL;
+  return 10.0 * std::log10(signal / noise);
+}
+
+mxq_precision mxq_select_precision(double sqnr_plain_db, double sqnr_transform_db, double high_db,
+                                   double low_db) {
+  if (sqnr_plain_db >= high_db) return MXQ_PREC_W4A4;
+  if (sqnr_transform_db >= high_db) return MXQ_PREC_W4A4_TRANSFORM;
+  if ((sqnr_plain_db > sqnr_transform_db ? sqnr_plain_db : sqnr_transform_db) >= low_db) return MXQ_PREC_W4A8;
+  return MXQ_PREC_BF16;
 }
 
 mxq_status mxq_debug_poll(void) {

@@ -22,10 +22,11 @@ STATUS_NAMES = {0: "MXQ_OK", 1: "MXQ_ERR_INVALID_ARG", 2: "MXQ_ERR_SHAPE", 3: "M
                 4: "MXQ_ERR_UNSUPPORTED", 5: "MXQ_ERR_CUDA", 6: "MXQ_ERR_TIMEOUT"}
 MXQ_SCALE_OCP, MXQ_SCALE_UOS = 0, 1
 MXQ_ACT_MXFP4, MXQ_ACT_FP8_E4M3 = 0, 1
+MXQ_PREC_W4A4, MXQ_PREC_W4A4_TRANSFORM, MXQ_PREC_W4A8, MXQ_PREC_BF16 = 0, 1, 2, 3
 
 EXPORTED = ("mxq_status_string", "mxq_sf_bytes", "mxq_quantize_act", "mxq_pack_weight", "mxq_gemm_w4a4",
             "mxq_gemm_w4a8", "mxq_dequant_mxfp4", "mxq_qdq_act", "mxq_channel_absmax", "mxq_smooth_factors",
-            "mxq_quantize_smooth", "mxq_debug_poll")
+            "mxq_quantize_smooth", "mxq_sqnr_accumulate", "mxq_sqnr_db", "mxq_select_precision", "mxq_debug_poll")
 
 
 class MxqError(RuntimeError):
@@ -68,6 +69,12 @@ def lib() -> ctypes.CDLL:
     L.mxq_smooth_factors.restype = I32
     L.mxq_quantize_smooth.argtypes = [P, I64, I64, I64, I32, I32, P, P, P, P]
     L.mxq_quantize_smooth.restype = I32
+    L.mxq_sqnr_accumulate.argtypes = [P, I64, P, I64, I64, I64, I32, P, P]
+    L.mxq_sqnr_accumulate.restype = I32
+    L.mxq_sqnr_db.argtypes = [ctypes.c_double, ctypes.c_double]
+    L.mxq_sqnr_db.restype = ctypes.c_double
+    L.mxq_select_precision.argtypes = [ctypes.c_double] * 4
+    L.mxq_select_precision.restype = I32
     L.mxq_debug_poll.argtypes = []
     L.mxq_debug_poll.restype = I32
     _lib = L
@@ -152,6 +159,20 @@ def mxq_quantize_smooth(x, rows, K, ldx, rule, hadamard128, chan_scale, codes_ou
     _check(lib().mxq_quantize_smooth(_ptr(x), int(rows), int(K), int(ldx), int(rule), int(bool(hadamard128)),
                                      _ptr(chan_scale), _ptr(codes_out), _ptr(sf_out), _stream(stream)),
            "mxq_quantize_smooth")
+
+
+def mxq_sqnr_accumulate(y, ldy, ref, ldr, M, N, accumulate, acc, stream=None) -> None:
+    _check(lib().mxq_sqnr_accumulate(_ptr(y), int(ldy), _ptr(ref), int(ldr), int(M), int(N), int(bool(accumulate)),
+                                     _ptr(acc), _stream(stream)), "mxq_sqnr_accumulate")
+
+
+def mxq_sqnr_db(signal: float, noise: float) -> float:
+    return float(lib().mxq_sqnr_db(float(signal), float(noise)))
+
+
+def mxq_select_precision(sqnr_plain_db: float, sqnr_transform_db: float, high_db: float, low_db: float) -> int:
+    return int(lib().mxq_select_precision(float(sqnr_plain_db), float(sqnr_transform_db), float(high_db),
+                                          float(low_db)))
 
 
 def mxq_debug_poll() -> int:

@@ -149,6 +149,31 @@ def test_smoothing_validation_happens_before_any_launch(L):
     assert qs(FAKE, 4, 48, 48, 0, 0, FAKE, FAKE, FAKE, None) == SHAPE
 
 
+def test_host_side_precision_selection_matches_the_oracle(L):
+    """The tier decision and the dB conversion are host-only C functions: compared with
+    the oracle's on a grid around both thresholds and on random values."""
+    import math
+    import random
+    vals = [-math.inf, 0.0, 9.99, 10.0, 10.01, 14.99, 15.0, 15.01, 30.0, math.inf]
+    rng = random.Random(3)
+    pairs = [(a, b) for a in vals for b in vals] + [(rng.uniform(0, 30), rng.uniform(0, 30)) for _ in range(200)]
+    for a, b in pairs:
+        assert mxq.mxq_select_precision(a, b, 15.0, 10.0) == oracle.select_precision(a, b, 15.0, 10.0), (a, b)
+    for s, n in [(26.0, 5.0), (1.0, 0.0), (0.0, 1.0), (3.5e7, 2.25e-3)]:
+        assert mxq.mxq_sqnr_db(s, n) == oracle.sqnr_db(s, n)
+
+
+def test_sqnr_validation_happens_before_any_launch(L):
+    INV, SHAPE, ALIGN = 1, 2, 3
+    sq = lambda *a: L.mxq_sqnr_accumulate(*a)
+    assert sq(None, 8, FAKE, 8, 4, 8, 0, FAKE, None) == INV
+    assert sq(FAKE, 8, FAKE, 8, 4, 8, 0, None, None) == INV
+    assert sq(FAKE, 8, FAKE, 8, 0, 8, 0, FAKE, None) == SHAPE
+    assert sq(FAKE, 4, FAKE, 8, 4, 8, 0, FAKE, None) == ALIGN                # ldy < N
+    assert sq(FAKE, 12, FAKE, 16, 4, 8, 0, FAKE, None) == ALIGN              # ldy % 8
+    assert sq(FAKE + 8, 8, FAKE, 8, 4, 8, 0, FAKE, None) == ALIGN
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
