@@ -112,6 +112,11 @@ def _load():
     lib.oracle_sqnr_db.restype = ctypes.c_double
     lib.oracle_select_precision.argtypes = [ctypes.c_double] * 4
     lib.oracle_select_precision.restype = ctypes.c_int
+    lib.oracle_pnq_exp2.argtypes = [ctypes.c_float, ctypes.c_int]
+    lib.oracle_pnq_exp2.restype = ctypes.c_float
+    lib.oracle_attention_mxfp4.argtypes = [P, P, P, I64, I64, I64, I64, I64, ctypes.c_int, ctypes.c_int, P, I64,
+                                           P, P, ctypes.c_int]
+    lib.oracle_attention_mxfp4.restype = None
     lib.oracle_gemm.argtypes = [ctypes.c_int, P, P, I64, P, P, I64, I64, ctypes.c_double, P, P, I64,
                                 P, ctypes.c_int]
     lib.oracle_gemm.restype = None
@@ -349,3 +354,28 @@ def sqnr_db(signal: float, noise: float) -> float:
 def select_precision(sqnr_plain_db: float, sqnr_transform_db: float, high_db: float, low_db: float) -> int:
     return int(_load().oracle_select_precision(float(sqnr_plain_db), float(sqnr_transform_db), float(high_db),
                                                float(low_db)))
+
+
+# ---------------------------------------------------------------- MXFP4 attention (UOS + PNQ)
+ATTN_PNQ, ATTN_NORMALISE_THEN_QUANTISE, ATTN_UNQUANTISED_P = 0, 1, 2
+
+
+def pnq_exp2(t: float, chat: int) -> float:
+    """2^(t - chat) by the attention numerators' polynomial definition (FP32)."""
+    return float(_load().oracle_pnq_exp2(ctypes.c_float(t), int(chat)))
+
+
+def attention_mxfp4(q, k, v, H: int, d: int, rows=None, rule: int = RULE_UOS, mode: int = ATTN_PNQ,
+                    nthreads: int | None = None):
+    """MXFP4 attention of query rows `rows` (default all) for every head.
+    q [Sq][H*d], k, v [Skv][H*d] BF16.  Returns (out [len(rows)][H][d] FP64,
+    weight sums [len(rows)][H])."""
+    qb, kb, vb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
+    Sq, Skv = qb.shape[0], kb.shape[0]
+    assert qb.shape[1] == kb.shape[1] == vb.shape[1] == H * d and d % 32 == 0
+    rows = np.arange(Sq, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    out = np.empty((rows.size, H, d), np.float64)
+    ws = np.empty((rows.size, H), np.float64)
+    _load().oracle_attention_mxfp4(_ptr(qb), _ptr(kb), _ptr(vb), Sq, Skv, H, d, H * d, int(rule), int(mode),
+                                   _ptr(rows), rows.size, _ptr(out), _ptr(ws), _threads(nthreads))
+    return out, ws

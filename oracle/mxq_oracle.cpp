@@ -58,6 +58,21 @@
 //    tiered thresholds (values not on the pages; parameters): plain >= high -> plain W4A4;
 //    else transform >= high -> transform-enabled W4A4; else the better of the two >= low
 //    -> W4A8 promotion; else BF16 fallback.
+//  * MXFP4 attention with UOS and PNQ [MXAttention: Data-Free Optimal Scaling and
+//    Pre-Normalization Quantization for MXFP4 Attention -- TL;DR, "Architecture" and
+//    "What it actually does"]: Q, K and V in MXFP4 (Q, K in 32-blocks along the head
+//    dimension, V in 32-blocks along the keys), scores S = deq(Q) deq(K)^T, the
+//    unnormalised exponentials quantised to MXFP4 in 32-key blocks BEFORE the row sum
+//    (PNQ), the row sum l taken over the quantised values, O = (deq(P) deq(V)) / l.
+//    Readings (the pages fix none of these): the numerators are taken in base 2,
+//    t = fl32(fl32(S) * fl32(log2(e) / sqrt(d))), relative to an integer offset
+//    c = ceil(max_j t_j) -- a power-of-two offset, under which E8M0 block scaling is
+//    exactly equivariant, so the codes do not depend on it; the exponential is
+//    2^(t - c) = p(g) * 2^(n - c) with n = floor(t), g = t - n - 1/2 and p the degree-7
+//    Taylor polynomial of 2^(g + 1/2) (coefficients a_0 = sqrt(2), a_k = a_(k-1) * ln 2 / k
+//    in FP64, rounded to FP32; Horner with FP32 fused multiply-adds), and numerators
+//    below 2^-126 are 0.  These FP32 steps decide the quantised codes, so they are
+//    taken in the kernel's precision; the rest is FP64.
 //  * Scale-factor memory layout (not given by the pages; a reading): rows padded
 //    to a multiple of 128, scale columns to a multiple of 4, 512-byte atoms of
 //    128 rows x 4 scale columns, byte
@@ -444,6 +459,122 @@ void oracle_gemm(int a_kind, const uint8_t* a_codes, const uint8_t* a_sf, int64_
     }
   });
   (void)M;
+}
+
+// ---------------------------------------------------------------- MXFP4 attention
+
+// Coefficients of the degree-7 Taylor polynomial of 2^(g + 1/2) around g = 0.
+static void pnq_exp2_coefficients(float* a) {
+  double c = std::sqrt(2.0);
+  const double ln2 = std::log(2.0);
+  for (int k = 0; k < 8; ++k) {
+    a[k] = static_cast<float>(c);
+    c = c * ln2 / static_cast<double>(k + 1);
+  }
+}
+
+// 2^(t - chat) by the definition above (t finite, chat an integer).
+float oracle_pnq_exp2(float t, int chat) {
+  float a[8];
+  pnq_exp2_coefficients(a);
+  const float n = std::floor(t);
+  const float g = (t - n) - 0.5f;  // both steps exact
+  float p = a[7];
+  for (int k = 6; k >= 0; --k) p = std::fmaf(p, g, a[k]);
+  const long e = static_cast<long>(n) - chat;
+  if (e < -126) return 0.0f;
+  return p * std::ldexp(1.0f, static_cast<int>(e));
+}
+
+// Attention of the sampled query rows q_rows[0..n_rows) for every head.
+//   q: [Sq][ld], k, v: [Skv][ld] BF16, head h in columns [h*d, (h+1)*d), d % 32 == 0.
+//   mode 0: PNQ (quantise the numerators, then the row sum); 1: the conventional order
+//   (row-normalise in FP32, quantise the probabilities, no further division); 2: no
+//   quantisation of P (FP64 softmax of the quantised-operand scores).
+//   out: [n_rows][H][d] FP64; wsum: [n_rows][H] sum of the implied attention weights.
+void oracle_attention_mxfp4(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t Sq, int64_t Skv,
+                            int64_t H, int64_t d, int64_t ld, int rule, int mode, const int64_t* q_rows,
+                            int64_t n_rows, double* out, double* wsum, int nthreads) {
+  const int64_t HD = H * d;
+  // K codes / scales for all rows (blocks along the head dimension).
+  std::vector<uint8_t> kc(static_cast<size_t>(Skv * HD / 2)), ks(static_cast<size_t>(Skv * HD / kBlock));
+  oracle_quantize_mxfp4(k, Skv, HD, ld, rule, 0, kc.data(), ks.data(), nthreads);
+  // V^T per head and channel, blocks along the keys, zero-padded to a whole block.
+  const int64_t Sp = (Skv + kBlock - 1) / kBlock * kBlock;
+  std::vector<uint16_t> vt(static_cast<size_t>(HD * Sp), 0);
+  for (int64_t j = 0; j < Skv; ++j)
+    for (int64_t c = 0; c < HD; ++c) vt[c * Sp + j] = v[j * ld + c];
+  std::vector<uint8_t> vc(static_cast<size_t>(HD * Sp / 2)), vs(static_cast<size_t>(HD * Sp / kBlock));
+  oracle_quantize_mxfp4(vt.data(), HD, Sp, Sp, rule, 0, vc.data(), vs.data(), nthreads);
+  auto deq = [](const uint8_t* codes, const uint8_t* sf, int64_t rowlen, int64_t r, int64_t i) {
+    const uint8_t byte = codes[r * (rowlen / 2) + i / 2];
+    const uint8_t c = (i % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+    return std::ldexp(oracle_e2m1_decode(c), static_cast<int>(sf[r * (rowlen / kBlock) + i / kBlock]) - 127);
+  };
+  std::vector<double> K(static_cast<size_t>(Skv * HD)), VT(static_cast<size_t>(HD * Sp));
+  for (int64_t j = 0; j < Skv; ++j)
+    for (int64_t c = 0; c < HD; ++c) K[j * HD + c] = deq(kc.data(), ks.data(), HD, j, c);
+  for (int64_t c = 0; c < HD; ++c)
+    for (int64_t j = 0; j < Sp; ++j) VT[c * Sp + j] = deq(vc.data(), vs.data(), Sp, c, j);
+  const float scale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+
+  parallel_rows(n_rows, nthreads, [&](int64_t i0, int64_t i1) {
+    std::vector<uint8_t> qc(static_cast<size_t>(HD / 2)), qs(static_cast<size_t>(HD / kBlock));
+    std::vector<double> Q(static_cast<size_t>(HD)), P(static_cast<size_t>(Sp));
+    std::vector<float> t(static_cast<size_t>(Skv)), pt(static_cast<size_t>(Sp));
+    for (int64_t i = i0; i < i1; ++i) {
+      const int64_t row = q_rows[i];
+      oracle_quantize_mxfp4(q + row * ld, 1, HD, ld, rule, 0, qc.data(), qs.data(), 1);
+      for (int64_t c = 0; c < HD; ++c) Q[c] = deq(qc.data(), qs.data(), HD, 0, c);
+      for (int64_t h = 0; h < H; ++h) {
+        float tmax = -INFINITY;
+        for (int64_t j = 0; j < Skv; ++j) {
+          double s = 0.0;
+          for (int64_t c = 0; c < d; ++c) s += Q[h * d + c] * K[j * HD + h * d + c];
+          t[j] = static_cast<float>(s) * scale;  // fl32(fl32(S) * scale)
+          tmax = std::max(tmax, t[j]);
+        }
+        if (mode == 2) {  // FP64 softmax, no quantisation of P
+          double l = 0.0;
+          for (int64_t j = 0; j < Skv; ++j) l += (P[j] = std::exp2(static_cast<double>(t[j]) - tmax));
+          for (int64_t j = Skv; j < Sp; ++j) P[j] = 0.0;
+          for (int64_t j = 0; j < Sp; ++j) P[j] /= l;
+        } else {
+          const int chat = static_cast<int>(std::ceil(tmax));
+          for (int64_t j = 0; j < Sp; ++j) pt[j] = j < Skv ? oracle_pnq_exp2(t[j], chat) : 0.0f;
+          if (mode == 1) {  // conventional: normalise, then quantise
+            double l = 0.0;
+            for (int64_t j = 0; j < Sp; ++j) l += pt[j];
+            for (int64_t j = 0; j < Sp; ++j) pt[j] = static_cast<float>(pt[j] / l);
+          }
+          for (int64_t b = 0; b < Sp / kBlock; ++b) {  // MXFP4 of the numerators, 32-key blocks
+            double amax = 0.0;
+            for (int u = 0; u < kBlock; ++u) amax = std::max(amax, static_cast<double>(pt[b * kBlock + u]));
+            const int e = oracle_block_exponent(amax, rule);
+            for (int u = 0; u < kBlock; ++u) {
+              const double x = std::ldexp(static_cast<double>(pt[b * kBlock + u]), -e);
+              P[b * kBlock + u] = std::ldexp(oracle_e2m1_decode(oracle_e2m1_encode(x)), e);
+            }
+          }
+          if (mode == 0) {  // PNQ: the row sum over the quantised numerators
+            double l = 0.0;
+            for (int64_t j = 0; j < Sp; ++j) l += P[j];
+            for (int64_t j = 0; j < Sp; ++j) P[j] /= l;
+          }
+        }
+        double ws = 0.0;
+        for (int64_t j = 0; j < Sp; ++j) ws += P[j];
+        if (wsum) wsum[i * H + h] = ws;
+        for (int64_t c = 0; c < d; ++c) {
+          double acc = 0.0;
+          const double* vrow = VT.data() + (h * d + c) * Sp;
+          for (int64_t j = 0; j < Sp; ++j) acc += P[j] * vrow[j];
+          out[(i * H + h) * d + c] = acc;
+        }
+      }
+    }
+  });
+  (void)Sq;
 }
 
 // ---------------------------------------------------------------- precision selection

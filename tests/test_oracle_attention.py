@@ -1,0 +1,110 @@
+"""Pins of the oracle's MXFP4 attention (UOS + PNQ): its exponential, closed-form
+outputs, and the properties the MXAttention page states.
+
+[MXAttention: Data-Free Optimal Scaling and Pre-Normalization Quantization for MXFP4
+ Attention -- TL;DR, "What it actually does"]
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mxfp4_block_scaled_mxq_b200 import inputs
+
+
+def _f32(x):
+    return float(np.float32(x))
+
+
+def test_pnq_exp2_accuracy():
+    """Within 4e-7 relative of 2^(t - c) over the range softmax numerators use."""
+    ts = np.float32(np.linspace(-40.0, 8.0, 20011))
+    worst = 0.0
+    for t in ts:
+        want = 2.0 ** (float(t) - 3)
+        worst = max(worst, abs(oracle.pnq_exp2(float(t), 3) - want) / want)
+    assert worst < 4e-7, worst
+
+
+@pytest.mark.parametrize("t", [-17.37, -0.001, 0.0, 2.5, 7.99])
+def test_pnq_exp2_offset_is_an_exact_power_of_two(t):
+    """Changing the integer offset scales the numerator by exactly a power of two (the
+    property that makes the MXFP4 codes independent of the offset)."""
+    t = _f32(t)
+    a, b = oracle.pnq_exp2(t, 0), oracle.pnq_exp2(t, 5)
+    assert a == b * 32.0
+
+
+def test_pnq_exp2_flushes_below_2_to_minus_126():
+    assert oracle.pnq_exp2(-127.5, 0) == 0.0
+    assert oracle.pnq_exp2(-126.0, 0) > 0.0
+
+
+def test_equal_scores_average_the_values():
+    """Identical keys: every score is equal, every numerator is equal, so O is the
+    plain mean of the dequantised values over the keys (PNQ's l cancels exactly)."""
+    H, d, S = 1, 64, 96
+    q = inputs.normal_bf16(4, H * d, 1.0, seed=1)
+    k = inputs.normal_bf16(1, H * d, 1.0, seed=2).repeat(S, 1)
+    v = inputs.normal_bf16(S, H * d, 1.0, seed=3)
+    out, ws = oracle.attention_mxfp4(q, k, v, H, d)
+    codes, sl = oracle.quantize_mxfp4(v.t().contiguous(), rule=oracle.RULE_UOS)   # V^T, blocks along keys
+    deq_vt = oracle.dequant_mxfp4(codes, oracle.sf_swizzle(sl, H * d, S), H * d, S)
+    want = deq_vt.mean(axis=1)
+    np.testing.assert_allclose(out[:, 0, :], np.broadcast_to(want, (4, d)), rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(ws, 1.0, rtol=1e-14)
+
+
+def test_one_dominant_key_returns_its_value():
+    """One key's score exceeds the others' by more than 126 in base 2: every other
+    numerator flushes to 0, so O is exactly that key's dequantised value row."""
+    H, d, S = 1, 32, 64
+    q = torch.zeros(1, d, dtype=torch.bfloat16)
+    q[0, 0] = 24.0
+    k = torch.zeros(S, d, dtype=torch.bfloat16)
+    k[17, 0] = 24.0            # S = 576, t = 576 * log2(e) / sqrt(32) = 147 vs 0
+    v = inputs.normal_bf16(S, d, 1.0, seed=4)
+    out, _ = oracle.attention_mxfp4(q, k, v, H, d)
+    codes, sl = oracle.quantize_mxfp4(v.t().contiguous(), rule=oracle.RULE_UOS)
+    deq_vt = oracle.dequant_mxfp4(codes, oracle.sf_swizzle(sl, d, S), d, S)
+    np.testing.assert_array_equal(out[0, 0], deq_vt[:, 17])
+
+
+def _three_modes(scale, rule=oracle.RULE_UOS):
+    H, d, S = 2, 128, 300
+    q = inputs.normal_bf16(S, H * d, scale, seed=1)
+    k = inputs.normal_bf16(S, H * d, scale, seed=2)
+    v = inputs.normal_bf16(S, H * d, 1.0, seed=3)
+    rows = np.arange(0, S, 7)
+    return [oracle.attention_mxfp4(q, k, v, H, d, rows, rule=rule, mode=m) for m in (0, 1, 2)]
+
+
+def test_pnq_preserves_normalisation_and_the_conventional_order_does_not():
+    """PNQ: the implied attention weights of every row sum to 1 (by construction).
+    Quantising after the row normalisation leaves rows whose weights do not."""
+    (o0, w0), (o1, w1), _ = _three_modes(1.0)
+    assert np.abs(w0 - 1.0).max() < 1e-12
+    assert np.abs(w1 - 1.0).max() > 1e-3
+
+
+def test_pnq_beats_the_conventional_order_on_peaked_attention():
+    """Peaked score distributions (Q, K ~ N(0, 4)): PNQ's output is closer to the
+    unquantised-P attention than quantise-after-normalise's (0.067 vs 0.101 here)."""
+    (o0, _), (o1, _), (o2, _) = _three_modes(2.0)
+    err = lambda o: np.linalg.norm(o - o2) / np.linalg.norm(o2)
+    assert err(o0) < 0.8 * err(o1), (err(o0), err(o1))
+
+
+@pytest.mark.parametrize("scale", [2.0, 3.0])
+def test_uos_beats_ocp(scale):
+    """UOS (Qmax = 7.25) against the stock OCP rule, both with PNQ, on peaked scores:
+    the quantised P moves the output less from the unquantised-P attention (each rule
+    against its own unquantised-P output, so only the numerators' quantisation differs;
+    0.067 vs 0.081 and 0.040 vs 0.047 here -- on diffuse scores the two are within 2 %)."""
+    (u, _), _, (u_ref, _) = _three_modes(scale, oracle.RULE_UOS)
+    (o, _), _, (o_ref, _) = _three_modes(scale, oracle.RULE_OCP)
+    err = lambda a, r: np.linalg.norm(a - r) / np.linalg.norm(r)
+    assert err(u, u_ref) < err(o, o_ref), (err(u, u_ref), err(o, o_ref))
