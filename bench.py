@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 METRIC = "MXFP4 W4A4 GEMM TFLOPS incl. act-quant and % of B200 dense FP4 peak"
 METRIC_W4A8 = "MXFP4 W4A8 GEMM TFLOPS incl. act-quant and % of B200 dense FP8 peak"
 METRIC_QDQ = "MXFP4 quantise-dequantise + weight dequantisation GB/s (HBM-bound)"
+METRIC_ATTN = "MXFP4 attention (UOS + PNQ) TFLOPS incl. Q/K/V quantisation and % of B200 dense FP4 peak"
 METRIC_POLICY = "precision-selection pass (plain + rotation/SmoothQuant W4A4 vs BF16 SQNR), ms per Wan FFN block"
 UNIT = "TFLOP/s"
 NOMINAL_FP4_TFLOPS = 9000.0          # dense FP4, nominal
@@ -46,7 +47,7 @@ TRAFFIC = {"wan_ffn": (241.4e6 + 867.0e6 + 345.3e6 + 314.8e6) / 2}
 # Packed weight bytes per workload (MXFP4 codes + scales), for the L2-residency decision.
 W_BYTES = {"wan_ffn": 2 * 5120 * 13824 * 17 // 32, "wan_attn_hadamard": 4 * 5120 * 5120 * 17 // 32,
            "flux_w4a8": (9216 + 12288) * 3072 * 17 // 32, "m_sweep": 13824 * 5120 * 17 // 32, "qdq_wan_ffn": 0,
-           "policy_wan_ffn": 0}
+           "policy_wan_ffn": 0, "attn_wan": 0}
 WORKLOAD = "Wan2.2-A14B FFN W4A4 (up 32760x5120->13824, down 32760x13824->5120), dynamic MXFP4 acts, OCP rule"
 M_TOK, D_MODEL, D_FF = 32760, 5120, 13824
 
@@ -62,9 +63,10 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--m", type=int, default=0, help="token count (0: the workload's own)")
     p.add_argument("--workload", choices=["wan_ffn", "wan_attn_hadamard", "flux_w4a8", "m_sweep", "qdq_wan_ffn",
-                                          "policy_wan_ffn"],
+                                          "policy_wan_ffn", "attn_wan"],
                    default="wan_ffn")
-    p.add_argument("--rule", choices=["ocp", "uos"], default="ocp", help="activation scale rule")
+    p.add_argument("--rule", choices=["ocp", "uos"], default=None,
+                   help="activation scale rule (default: ocp; uos for the attention workload)")
     p.add_argument("--smooth", action="store_true",
                    help="SmoothQuant after the rotation (W4A4 workloads; factors calibrated before timing)")
     return p.parse_args()
@@ -378,6 +380,32 @@ def build_workload(name, dev, M, seed, rule_name, smooth=False):
                 f"M={M}: BF16 reference, plain and rotation+SmoothQuant W4A4, SQNR sums")
         return desc, parts, xs, outs, flops
 
+    if name == "attn_wan":
+        # Wan2.2 self-attention: 40 heads of 128 over the video tokens; Q, K, V quantised
+        # (UOS by default), then one attention launch over all heads.
+        H, d = 40, 128
+        q = inputs.normal_bf16(M, H * d, 1.0, seed, device=dev)
+        k = inputs.normal_bf16(M, H * d, 1.0, seed + 1, device=dev)
+        v = inputs.heavy_tailed_bf16(M, H * d, seed + 2, device=dev)
+        arule = mxq.MXQ_SCALE_OCP if rule_name == "ocp" else mxq.MXQ_SCALE_UOS
+        qb, kb = qbufs(M, H * d), qbufs(M, H * d)
+        Sp = mxq.mxq_attn_padded_keys(M)
+        vb = (torch.empty(H * d, Sp // 2, dtype=torch.uint8, device=dev),
+              torch.empty(mxq.mxq_sf_bytes(H * d, Sp), dtype=torch.uint8, device=dev))
+        o = out(M, H * d)
+        flops = 4.0 * M * M * d * H
+        parts = [
+            Part("quant_q", "quant", lambda: mxq.quantize_act(q, arule, out=qb), nbytes=quant_bytes(M, H * d)),
+            Part("quant_k", "quant", lambda: mxq.quantize_act(k, arule, out=kb), nbytes=quant_bytes(M, H * d)),
+            Part("quant_vt", "quant", lambda: mxq.quantize_vt(v, arule, out=vb), nbytes=quant_bytes(M, H * d)),
+            Part("attention", "gemm", lambda: mxq.mxq_attention_mxfp4(qb[0], qb[1], kb[0], kb[1], vb[0], vb[1], M, M,
+                                                                      H, d, arule, o.data_ptr(), o.stride(0)),
+                 flops=flops),
+        ]
+        desc = (f"Wan2.2 self-attention, {M} tokens x {H} heads x d={d}, MXFP4 Q/K/V/P with "
+                f"{'UOS' if arule == mxq.MXQ_SCALE_UOS else 'OCP'} scales and PNQ")
+        return desc, parts, [q, k, v], [o], flops
+
     raise ValueError(f"unknown workload {name}")
 
 
@@ -405,9 +433,10 @@ def main():
 
     # Inputs (per rank its own token batch); weights packed once before timing.
     default_m = {"wan_ffn": M_TOK, "wan_attn_hadamard": M_TOK, "flux_w4a8": 3584, "m_sweep": 1024,
-                 "qdq_wan_ffn": M_TOK, "policy_wan_ffn": 4096}[args.workload]
+                 "qdq_wan_ffn": M_TOK, "policy_wan_ffn": 4096, "attn_wan": M_TOK}[args.workload]
     M = args.m if args.m else default_m
-    desc, parts, x_in, d_out, flops_step = build_workload(args.workload, dev, M, rank_seed(rank), args.rule,
+    rule = args.rule or ("uos" if args.workload == "attn_wan" else "ocp")
+    desc, parts, x_in, d_out, flops_step = build_workload(args.workload, dev, M, rank_seed(rank), rule,
                                                           args.smooth)
     stream = torch.cuda.current_stream(dev)
 
@@ -508,6 +537,8 @@ def main():
     achieved_q = sum(p.nbytes for p in quant_parts) / (quant_t / 1e3) / 1e9 if quant_parts else None
     kernel_name = ("mx_gemm_pair_kernel" if M > 128 else "mx_gemm_swap_kernel") + (
         "<W4A8> (tcgen05 kind::mxf8f6f4)" if gemm_kind == "fp8" else "<W4A4> (tcgen05 kind::mxf4)")
+    if args.workload == "attn_wan":
+        kernel_name = "mx_attention_kernel (tcgen05 kind::mxf4 Q K^T and P V, PNQ softmax on the CUDA cores)"
     if hbm_only:
         top = max(zip(parts, part_ms), key=lambda pt: pt[1])
         top_gbs = top[0].nbytes / (top[1] / 1e3) / 1e9
@@ -527,7 +558,8 @@ def main():
                     "traffic": None}
     nominal = NOMINAL_FP4_TFLOPS if gemm_kind == "fp4" else NOMINAL_FP8_TFLOPS
     result = {
-        "metric": (METRIC_POLICY if time_metric else METRIC_QDQ if hbm_only else
+        "metric": (METRIC_POLICY if time_metric else METRIC_QDQ if hbm_only else METRIC_ATTN
+                   if args.workload == "attn_wan" else
                    METRIC if args.workload in ("wan_ffn", "m_sweep", "wan_attn_hadamard") else METRIC_W4A8),
         "value": value, "unit": "ms" if time_metric else "GB/s" if hbm_only else UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,

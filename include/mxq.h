@@ -270,6 +270,48 @@ MXQ_API mxq_precision mxq_select_precision(double sqnr_plain_db, double sqnr_tra
                                            double high_db, double low_db);
 
 /*
+ * MXFP4 attention with UOS and pre-normalisation quantisation (PNQ).
+ * [MXAttention: Data-Free Optimal Scaling and Pre-Normalization Quantization for MXFP4
+ *  Attention -- TL;DR, "Architecture", "What it actually does"]
+ * Per head h (columns [h d, (h+1) d) of the [S][H d] activations):
+ *   S = deq(Q) deq(K)^T, t = fl32(S * fl32(log2(e) / sqrt(d))),
+ *   P = MXFP4(2^(t - c)) in 32-key blocks -- the unnormalised numerators quantised BEFORE
+ *       the row sum, with the block-scale rule `rule` (UOS: Qmax = 7.25),
+ *   l = sum_j deq(P)_j,  O = deq(P) deq(V) / l.
+ * c is an integer offset (at least the row maximum of t minus 8); since E8M0 block scaling
+ * is exactly equivariant under powers of two, the codes of P do not depend on which such c
+ * is used.  2^(t - c) is evaluated as p(g) * 2^(n - c) with n = rint(t) (ties to even),
+ * g = t - n and p the degree-7 Taylor polynomial of 2^g (a_0 = 1, a_k = a_(k-1) ln 2 / k in
+ * FP64, rounded to FP32; Horner with FP32 fused multiply-adds); numerators with n - c < -126
+ * are 0.  Scores must satisfy |t| < 2^22.
+ *
+ * mxq_attn_padded_keys -- Sp = S_kv rounded up to the kernel's 256-key tile (-1 if S_kv is
+ * outside [1, 2^23]).
+ *
+ * mxq_quantize_vt -- V [S][ldv] BF16 -> V^T in MXFP4 with 32-key blocks (the layout the P V
+ * product consumes): codes_out [HD][Sp/2] (keys in [S, Sp) are zero), sf_out
+ * mxq_sf_bytes(HD, Sp) bytes in the layout of the other scale buffers (rows = channels).
+ * HD % 128 == 0, HD <= 2^16, ldv >= HD, ldv % 16 == 0, v 32-byte aligned.
+ *
+ * mxq_attention_mxfp4 -- q_codes / q_sf: Q [S_q][H d] quantised by mxq_quantize_act (MXFP4,
+ * the same rule, no rotation); k_codes / k_sf: K [S_kv][H d] likewise; vt_codes / vt_sf:
+ * from mxq_quantize_vt.  out_bf16: O [S_q][ldo] BF16 (head h in columns [h d, (h+1) d)),
+ * ldo >= H d, ldo % 8 == 0.  d must be 128 (MXQ_ERR_UNSUPPORTED otherwise); H d <= 2^16;
+ * 1 <= S_q <= 8388480; all buffers 16-byte aligned.  One sequence per call.
+ */
+MXQ_API int64_t mxq_attn_padded_keys(int64_t S_kv);
+
+MXQ_API mxq_status mxq_quantize_vt(const void* v_bf16, int64_t S, int64_t HD, int64_t ldv,
+                                   mxq_scale_rule rule, void* codes_out, void* sf_out,
+                                   mxq_stream_t stream);
+
+MXQ_API mxq_status mxq_attention_mxfp4(const void* q_codes, const void* q_sf, const void* k_codes,
+                                       const void* k_sf, const void* vt_codes, const void* vt_sf,
+                                       int64_t S_q, int64_t S_kv, int64_t H, int64_t d,
+                                       mxq_scale_rule rule, void* out_bf16, int64_t ldo,
+                                       mxq_stream_t stream);
+
+/*
  * mxq_debug_poll -- reads and clears the library's device status word, written by a
  * kernel that gave up one of its bounded waits (each wait on a barrier or a copy is
  * capped at about a second, after which the kernel records MXQ_ERR_TIMEOUT, drains

@@ -1,0 +1,475 @@
+// attention.cuh -- MXFP4 attention with the data-free UOS block-scale rule and
+// pre-normalisation quantisation (PNQ) of the softmax numerators, on tcgen05.
+// [MXAttention: Data-Free Optimal Scaling and Pre-Normalization Quantization for MXFP4
+//  Attention -- TL;DR, "Architecture", "What it actually does"]
+//
+//   O = (deq(P) deq(V)) / l,   P = MXFP4(2^(t - c)),   l = sum_j deq(P)_j,
+//   t = fl32(S * log2(e) / sqrt(d)),   S = deq(Q) deq(K)^T,
+//
+// with Q, K in 32-blocks along the head dimension, V and P in 32-blocks along the keys,
+// c an integer offset (a power-of-two factor, under which the E8M0 block scaling is
+// exactly equivariant: the codes of P do not depend on it) and 2^(t - c) the degree-7
+// Taylor polynomial of 2^g, g = t - rint(t), times 2^(rint(t) - c) (0 when rint(t) - c <
+// -126).  The row sum is taken over the quantised numerators
+// (PNQ), so the implied weights sum to one by construction; it is computed by the
+// tensor core itself: V^T carries one extra row of ones, so column d of the P V
+// accumulator is l.
+//
+// One CTA per (128 queries, head), head dimension 128, 256 keys per tile:
+//   warp 0      TMA producer: the Q tile (64-byte swizzle) once; per key tile the K
+//               tile (256 x 64 B, 64-byte swizzle), the V^T tile (128 x 128 B, 128-byte
+//               swizzle) and their scale atoms (4-D boxes, zero fill past the end).
+//   warp 1      MMA issuer: S = Q K^T (M 128, N 256, K 128) into TMEM; for the previous
+//               tile, O += P V^T (M 128, N 144: d columns + the ones row, K 256 keys);
+//               the next tile's scores are issued before the previous tile's P V, so
+//               the tensor core works while the softmax warps quantise.
+//   warps 2..9  softmax / PNQ, two threads per query row (keys [0,128) and [128,256) of
+//               the tile): scores from TMEM, the row maximum through shared memory, the
+//               offset c raised only when the maximum passes c + 8 (then O, l are
+//               rescaled in TMEM by the exact power of two), numerators, UOS/OCP block
+//               scales and E2M1 codes written to shared memory in the 128-byte-swizzled
+//               operand layout, scale bytes in the 512-byte atom layout; at the end
+//               O / l -> BF16.
+//
+// Every wait is bounded (ptx.cuh); on a timeout the kernel records MXQ_ERR_TIMEOUT,
+// drains its own copies and MMAs, and returns.
+#pragma once
+
+#include "gemm_common.cuh"
+#include "quantize.cuh"
+
+namespace mxq {
+
+constexpr int kAttnD = 128;       // head dimension
+constexpr int kAttnBM = 128;      // queries per CTA
+constexpr int kAttnBN = 256;      // keys per tile
+constexpr int kAttnStages = 3;
+constexpr int kAttnThreads = 320;  // producer, MMA, 8 softmax warps
+constexpr int kAttnNv = kAttnD + 16;  // P V's N: the d value columns and 16 rows holding the ones row
+constexpr uint32_t kAttnTmemCols = 512;
+constexpr uint32_t kColS = 0;      // scores, 256 columns
+constexpr uint32_t kColO = 256;    // output accumulator, 144 columns (column 128 = l)
+constexpr uint32_t kColSfq = 400;  // Q scales, 4 columns
+constexpr uint32_t kColSfk = 404;  // K scales: 2 parities x 8 columns (two 128-key row groups)
+constexpr uint32_t kColSfp = 420;  // P scales: 2 parities x 2 atoms x 4 columns
+constexpr uint32_t kColSfv = 436;  // V^T scales: 2 parities x 2 atoms x 8 columns (values, ones)
+
+// Shared memory (offsets from a 1024-byte aligned base).
+constexpr int kAttnQBytes = kAttnBM * 64;                   // 8 KB, 64-byte swizzle
+constexpr int kAttnKBytes = kAttnBN * 64;                   // 16 KB, 64-byte swizzle
+constexpr int kAttnVBytes = kAttnNv * 128;                  // 18 KB, 128-byte swizzle (+ ones rows)
+constexpr int kAttnStageBytes = kAttnKBytes + kAttnVBytes + 1024 /*K scales*/ + 1024 /*V scales*/;
+constexpr int kAttnOffSfq = kAttnQBytes;
+constexpr int kAttnOffStages = kAttnQBytes + 1024;
+constexpr int kAttnOffP = kAttnOffStages + kAttnStages * kAttnStageBytes;
+constexpr int kAttnOffSfp = kAttnOffP + kAttnBM * 128;      // 2 atoms
+constexpr int kAttnOffSfOnes = kAttnOffSfp + 1024;          // 2 atoms of unit scales
+constexpr int kAttnOffRmax = kAttnOffSfOnes + 1024;         // float [2 parities][2 halves][128]
+constexpr int kAttnOffBar = kAttnOffRmax + 2048;
+constexpr int kAttnSmemBytes = 1024 + kAttnOffBar + 256;
+
+// Instruction descriptors (kind::mxf4 block_scale, E2M1 x E2M1, UE8M0 scales, K-major).
+__host__ __device__ constexpr uint32_t attn_idesc(int n) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(kAttnBM >> 4) << 24);
+}
+
+struct AttnParams {
+  float exp2c[8];  // Taylor coefficients a_k = (ln 2)^k / k! of 2^g, FP32
+  float t_scale;   // fl32(log2(e) / sqrt(d))
+  int Sq;
+  int Skv;
+  int num_tiles;   // ceil(Skv / 256)
+};
+
+// Numerators of a pair of keys: 2^(t - chat) = p(g) * 2^(n - chat), n = rint(t), g = t - n,
+// p the Taylor polynomial of 2^g (Horner, FP32 fused multiply-adds), 0 when n - chat < -126.
+// Everything runs on the FMA pipe: t is first raised to chat - 127 (masked keys at -inf and
+// every t whose n - chat would be -127 or less give exactly 0 below); r = t + 1.5 * 2^23 holds
+// rint(t) in its low mantissa bits (|t| < 2^22), so n = r - 1.5 * 2^23 and g = t - n are
+// exact; and the FP32 bit pattern of 2^(n - chat) is (bits(r) + 127 - chat) * 2^23 modulo 2^32
+// (bits(1.5 * 2^23) * 2^23 vanishes modulo 2^32), one integer multiply-add, 0 for n - chat = -127.
+__device__ __forceinline__ float2 pnq_exp2_pair(float2 t, float lo, uint32_t bias_bits, const AttnParams& prm) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  t = make_float2(fmaxf(t.x, lo), fmaxf(t.y, lo));
+  const float2 r = __fadd2_rn(t, make_float2(kMagic, kMagic));
+  const float2 n = __fadd2_rn(r, make_float2(-kMagic, -kMagic));
+  const float2 g = __fadd2_rn(t, make_float2(-n.x, -n.y));
+  float2 p = make_float2(prm.exp2c[7], prm.exp2c[7]);
+#pragma unroll
+  for (int k = 6; k >= 0; --k) p = __ffma2_rn(p, g, make_float2(prm.exp2c[k], prm.exp2c[k]));
+  const float2 sc = make_float2(__uint_as_float(__float_as_uint(r.x) * 8388608u + bias_bits),
+                                __uint_as_float(__float_as_uint(r.y) * 8388608u + bias_bits));
+  return __fmul2_rn(p, sc);
+}
+
+template <bool kUOS>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    mx_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_sfq,
+                        const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_sfk,
+                        const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_sfv,
+                        __nv_bfloat16* __restrict__ out, int64_t ldo, const AttnParams prm) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sSfq = smem + kAttnOffSfq;
+  uint8_t* sStages = smem + kAttnOffStages;
+  uint8_t* sP = smem + kAttnOffP;
+  uint8_t* sSfp = smem + kAttnOffSfp;
+  uint8_t* sSfOnes = smem + kAttnOffSfOnes;
+  float* sRmax = reinterpret_cast<float*>(smem + kAttnOffRmax);
+  uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + kAttnOffBar);
+  uint64_t* kv_full = q_full + 1;
+  uint64_t* kv_empty = kv_full + kAttnStages;
+  uint64_t* s_full = kv_empty + kAttnStages;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_full = s_free + 1;
+  uint64_t* o_done = p_full + 1;
+  uint64_t* rbar = o_done + 1;  // [2]
+  uint64_t* drain = rbar + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  auto sK = [&](int s) { return sStages + s * kAttnStageBytes; };
+  auto sV = [&](int s) { return sStages + s * kAttnStageBytes + kAttnKBytes; };
+  auto sSfk = [&](int s) { return sStages + s * kAttnStageBytes + kAttnKBytes + kAttnVBytes; };
+  auto sSfv = [&](int s) { return sStages + s * kAttnStageBytes + kAttnKBytes + kAttnVBytes + 1024; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int q_tile = blockIdx.x;
+  const int head = blockIdx.y;
+  const int nt = prm.num_tiles;
+
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmap_q);
+    prefetch_tmap(&tmap_sfq);
+    prefetch_tmap(&tmap_k);
+    prefetch_tmap(&tmap_sfk);
+    prefetch_tmap(&tmap_v);
+    prefetch_tmap(&tmap_sfv);
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kAttnStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 8);   // one arrival per softmax warp
+    mbar_init(p_full, 8);
+    mbar_init(o_done, 1);
+    mbar_init(&rbar[0], 256);
+    mbar_init(&rbar[1], 256);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp >= 2) {
+    // Constant parts of the P V operand: the row of ones (row d = 128 of each V^T stage:
+    // E2M1 1.0 = code 2 in every nibble; rows 129..143 zero) and their unit scales.
+    const int t = threadIdx.x - 64;  // 0..255
+    for (int s = 0; s < kAttnStages; ++s) {
+      uint32_t* ones = reinterpret_cast<uint32_t*>(sV(s) + kAttnD * 128);  // 16 rows x 128 B = 512 words
+      ones[t] = t < 32 ? 0x22222222u : 0u;
+      ones[t + 256] = 0u;
+    }
+    reinterpret_cast<uint32_t*>(sSfOnes)[t] = 0x7F7F7F7Fu;  // 2 atoms = 256 words
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kAttnTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      bool ok = true;
+      mbar_arrive_expect_tx(q_full, kAttnQBytes + 512);
+      tma_load_2d(sQ, &tmap_q, head * 64, q_tile * kAttnBM, q_full);
+      tma_load_4d(sSfq, &tmap_sfq, 0, 0, head, q_tile, q_full);
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_phase = 0;
+      const uint32_t tx = kAttnKBytes + kAttnD * 128 + 1024 + 1024;
+      for (int j = 0; j < nt; ++j) {
+        if (!mbar_wait(&kv_empty[stage], phase ^ 1)) { ok = false; break; }
+        issued |= 1u << stage;
+        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+        mbar_arrive_expect_tx(&kv_full[stage], tx);
+        tma_load_2d(sK(stage), &tmap_k, head * 64, j * kAttnBN, &kv_full[stage]);
+        tma_load_4d(sSfk(stage), &tmap_sfk, 0, 0, head, 2 * j, &kv_full[stage]);
+        tma_load_2d(sV(stage), &tmap_v, j * (kAttnBN / 2), head * kAttnD, &kv_full[stage]);
+        tma_load_4d(sSfv(stage), &tmap_sfv, 0, 0, 2 * j, head, &kv_full[stage]);
+        if (++stage == kAttnStages) { stage = 0; phase ^= 1; }
+      }
+      mbar_wait_drain(q_full, 0);
+      if (!ok) {
+        for (int s = 0; s < kAttnStages; ++s)
+          if (issued & (1u << s)) mbar_wait_drain(&kv_full[s], (issued_phase >> s) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      bool ok = mbar_wait(q_full, 0);
+      if (ok) {
+        tc_fence_after();
+        tc_cp_sf_atom(tmem + kColSfq, smem_desc(smem_u32(sSfq), 0, 128, 0));
+      }
+      // O += P V^T for key tile i (P from shared memory, written by the softmax warps).
+      auto issue_pv = [&](int i) -> bool {
+        if (!mbar_wait(p_full, i & 1)) return false;
+        tc_fence_after();
+        const int st = i % kAttnStages;
+        const uint32_t par = static_cast<uint32_t>(i & 1);
+        const uint32_t sfp = kColSfp + par * 8, sfv = kColSfv + par * 16;
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          tc_cp_sf_atom(tmem + sfp + 4 * a, smem_desc(smem_u32(sSfp + a * 512), 0, 128, 0));
+          tc_cp_sf_atom(tmem + sfv + 8 * a, smem_desc(smem_u32(sSfv(st) + a * 512), 0, 128, 0));
+          tc_cp_sf_atom(tmem + sfv + 8 * a + 4, smem_desc(smem_u32(sSfOnes + a * 512), 0, 128, 0));
+        }
+        const uint32_t p_base = smem_u32(sP), v_base = smem_u32(sV(st));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // 4 x 64 keys
+          const int a = kk >> 1;
+          const uint32_t sf_id = static_cast<uint32_t>((kk & 1) * 2);
+          const uint32_t idesc = attn_idesc(kAttnNv) | (sf_id << 29) | (sf_id << 4);
+          tc_mma_mxf4(tmem + kColO, smem_desc(p_base + kk * 32, 16, 1024, 2), smem_desc(v_base + kk * 32, 16, 1024, 2),
+                      idesc, tmem + sfp + 4 * a, tmem + sfv + 8 * a, (i | kk) != 0);
+        }
+        tc_commit(o_done);
+        tc_commit(&kv_empty[st]);
+        return true;
+      };
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int j = 0; ok && j < nt; ++j) {
+        if (!mbar_wait(&kv_full[stage], phase)) { ok = false; break; }
+        if (j > 0 && !mbar_wait(s_free, (j - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sfk = kColSfk + static_cast<uint32_t>(j & 1) * 8;
+        tc_cp_sf_atom(tmem + sfk, smem_desc(smem_u32(sSfk(stage)), 0, 128, 0));
+        tc_cp_sf_atom(tmem + sfk + 4, smem_desc(smem_u32(sSfk(stage) + 512), 0, 128, 0));
+        const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK(stage));
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {  // 2 x 64 of the head dimension
+          const uint32_t sf_id = static_cast<uint32_t>(kk * 2);
+          const uint32_t idesc = attn_idesc(kAttnBN) | (sf_id << 29) | (sf_id << 4);
+          tc_mma_mxf4(tmem + kColS, smem_desc(q_base + kk * 32, 16, 512, 4), smem_desc(k_base + kk * 32, 16, 512, 4),
+                      idesc, tmem + kColSfq, tmem + sfk, kk != 0);
+        }
+        tc_commit(s_full);
+        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+        if (++stage == kAttnStages) { stage = 0; phase ^= 1; }
+      }
+      if (ok) ok = issue_pv(nt - 1);
+      if (!ok) {
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax / PNQ (warps 2..9)
+    const int quad = warp & 3;          // TMEM lanes [32 quad, +32)
+    const int hf = (warp - 2) >> 2;     // key half of every tile
+    const int r = quad * 32 + lane;     // query row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    int chat = 0;
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full, j & 1))) { ok = false; break; }
+      tc_fence_after();
+      float t[128];
+      {
+        uint32_t v[64];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tmem_ld64(tmem + lane_off + kColS + 128 * hf + 64 * c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 64; ++i) t[64 * c + i] = __fmul_rn(__uint_as_float(v[i]), prm.t_scale);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
+      // keys past the end do not take part (only the last tile has any)
+      const int key0 = j * kAttnBN + 128 * hf;
+      if (key0 + 128 > prm.Skv) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (key0 + i >= prm.Skv) t[i] = -INFINITY;
+      }
+      float m = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) m = fmaxf(m, t[i]);
+      float* slot = sRmax + (j & 1) * 256;
+      slot[hf * 128 + r] = m;
+      mbar_arrive(&rbar[j & 1]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&rbar[j & 1], (j >> 1) & 1))) { ok = false; break; }
+      m = fmaxf(m, slot[(1 - hf) * 128 + r]);  // finite: key j*256 is always valid
+      const int cand = static_cast<int>(ceilf(m));
+      float rescale = 1.f;
+      if (j == 0) {
+        chat = cand;
+      } else if (cand > chat + 8) {
+        rescale = __int_as_float((127 + chat - cand) << 23);  // 2^(chat - cand), exact
+        chat = cand;
+      }
+      // numerators -> MXFP4 (4 blocks of 32 keys), kept as codes and scale bytes
+      const float lo = static_cast<float>(chat - 127);
+      const uint32_t bias_bits = static_cast<uint32_t>(127 - chat) << 23;
+      uint32_t codes[16];
+      uint32_t sf_word = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        float2 p[16];
+        float amax = 0.f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          p[u] = pnq_exp2_pair(make_float2(t[32 * b + 2 * u], t[32 * b + 2 * u + 1]), lo, bias_bits, prm);
+          amax = fmaxf(amax, fmaxf(p[u].x, p[u].y));
+        }
+        const int e = block_exponent<kUOS>(__float_as_uint(amax));
+        const float s1 = exp2_neg(e);
+        const float2 sc = make_float2(s1, s1);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 v = __fmul2_rn(p[4 * w + q], sc);
+            word |= e2m1x2(v.x, v.y) << (8 * q);
+          }
+          codes[4 * b + w] = word;
+        }
+        sf_word |= static_cast<uint32_t>(e + 127) << (8 * b);
+      }
+      // the previous tile's P V must be done before P is overwritten or O rescaled
+      if (j > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1))) { ok = false; break; }
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, rescale != 1.f)) {
+        uint32_t v[64];
+        const uint32_t a0 = tmem + lane_off + kColO + 64 * hf;
+        tmem_ld64(a0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 64; ++i) v[i] = __float_as_uint(__fmul_rn(__uint_as_float(v[i]), rescale));
+        tmem_st64(a0, v);
+        if (hf == 0) {  // the l column block (column 128 and the zero columns after it)
+          const uint32_t a1 = tmem + lane_off + kColO + kAttnD;
+          tmem_ld16(a1, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__fmul_rn(__uint_as_float(v[i]), rescale));
+          tmem_st16(a1, v);
+        }
+        tmem_st_wait();
+      }
+      // codes: row r, bytes [64 hf, +64) = 16-byte chunks 4 hf + b, 128-byte swizzle
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int chunk = (4 * hf + b) ^ (r & 7);
+        *reinterpret_cast<uint4*>(sP + r * 128 + chunk * 16) =
+            make_uint4(codes[4 * b], codes[4 * b + 1], codes[4 * b + 2], codes[4 * b + 3]);
+      }
+      *reinterpret_cast<uint32_t*>(sSfp + hf * 512 + (r & 31) * 16 + (r >> 5) * 4) = sf_word;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    // ---------------------------------------------------------------- O / l -> BF16
+    if (ok && __all_sync(0xffffffffu, mbar_wait(o_done, (nt - 1) & 1))) {
+      tc_fence_after();
+      uint32_t v[64], lv[16];
+      tmem_ld64(tmem + lane_off + kColO + 64 * hf, v);
+      tmem_ld16(tmem + lane_off + kColO + kAttnD, lv);
+      tmem_ld_wait();
+      const float inv_l = __fdiv_rn(1.0f, __uint_as_float(lv[0]));
+      const int64_t row = static_cast<int64_t>(q_tile) * kAttnBM + r;
+      if (row < prm.Sq) {
+        uint4* dst = reinterpret_cast<uint4*>(out + row * ldo + head * kAttnD + 64 * hf);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            w[q] = pack_bf16x2(__fmul_rn(__uint_as_float(v[8 * c + 2 * q]), inv_l),
+                               __fmul_rn(__uint_as_float(v[8 * c + 2 * q + 1]), inv_l));
+          dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kAttnTmemCols);
+  }
+}
+
+// V [S][ldv] BF16 -> V^T in MXFP4 with 32-key blocks: codes [HD][Sp/2], scales for the
+// [HD][Sp/32] grid in the 512-byte atom layout; keys in [S, Sp) are zero.  One CTA per
+// 128 keys x 128 channels: the tile is staged in shared memory (BF16) and read back
+// column-wise (a warp: 32 consecutive channels of one key row per step).
+template <bool kUOS>
+__global__ void __launch_bounds__(256) quantize_vt_kernel(const uint16_t* __restrict__ v, int64_t S, int64_t ldv,
+                                                           int64_t Sp, uint8_t* __restrict__ codes,
+                                                           uint8_t* __restrict__ sf) {
+  constexpr int kPitch = 136;  // halfwords per staged row (272 bytes: 16-byte aligned rows)
+  __shared__ __align__(16) uint16_t tile[128 * kPitch];
+  const int tid = threadIdx.x;
+  const int64_t key0 = static_cast<int64_t>(blockIdx.y) * 128;
+  const int64_t ch0 = static_cast<int64_t>(blockIdx.x) * 128;
+  {
+    const int i = tid >> 1, c0 = 64 * (tid & 1);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t w[8];
+      if (key0 + i < S) {
+        ld_stream_v8(v + (key0 + i) * ldv + ch0 + c0 + 16 * q, w);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) w[u] = 0u;
+      }
+      uint4* dst = reinterpret_cast<uint4*>(tile + i * kPitch + c0 + 16 * q);
+      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+  }
+  __syncthreads();
+  const int c = tid & 127, th = tid >> 7;  // a warp: 32 consecutive channels, one key half
+  const int64_t row = ch0 + c;
+  auto val = [&](int k) { return __uint_as_float(static_cast<uint32_t>(tile[k * kPitch + c]) << 16); };
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    const int k0 = 64 * th + 32 * b;
+    float amax = 0.f;
+#pragma unroll
+    for (int u = 0; u < 32; ++u) amax = fmaxf(amax, fabsf(val(k0 + u)));
+    const int e = block_exponent<kUOS>(__float_as_uint(amax));
+    const float s = exp2_neg(e);
+    uint32_t word[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t x = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        x |= e2m1x2(__fmul_rn(val(k0 + 8 * w + 2 * q), s), __fmul_rn(val(k0 + 8 * w + 2 * q + 1), s)) << (8 * q);
+      word[w] = x;
+    }
+    const int64_t kb = key0 + k0;  // first key of the block
+    *reinterpret_cast<uint4*>(codes + row * (Sp / 2) + kb / 2) = make_uint4(word[0], word[1], word[2], word[3]);
+    const int64_t col = kb / 32;
+    sf[((row >> 7) * (Sp / 128) + (col >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (col & 3)] =
+        static_cast<uint8_t>(e + 127);
+  }
+}
+
+}  // namespace mxq

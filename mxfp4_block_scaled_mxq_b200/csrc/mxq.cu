@@ -13,6 +13,7 @@
 #include "gemm_pair.cuh"
 #include "gemm_swap.cuh"
 #include "policy.cuh"
+#include "attention.cuh"
 #include "quantize.cuh"
 
 namespace {
@@ -480,6 +481,95 @@ mxq_precision mxq_select_precision(double sqnr_plain_db, double sqnr_transform_d
   if (sqnr_transform_db >= high_db) return MXQ_PREC_W4A4_TRANSFORM;
   if ((sqnr_plain_db > sqnr_transform_db ? sqnr_plain_db : sqnr_transform_db) >= low_db) return MXQ_PREC_W4A8;
   return MXQ_PREC_BF16;
+}
+
+int64_t mxq_attn_padded_keys(int64_t S_kv) {
+  if (S_kv < 1 || S_kv > (int64_t(1) << 23)) return -1;
+  return (S_kv + mxq::kAttnBN - 1) / mxq::kAttnBN * mxq::kAttnBN;
+}
+
+mxq_status mxq_quantize_vt(const void* v_bf16, int64_t S, int64_t HD, int64_t ldv, mxq_scale_rule rule,
+                           void* codes_out, void* sf_out, mxq_stream_t stream) {
+  if (!v_bf16 || !codes_out || !sf_out) return MXQ_ERR_INVALID_ARG;
+  if (rule != MXQ_SCALE_OCP && rule != MXQ_SCALE_UOS) return MXQ_ERR_INVALID_ARG;
+  const int64_t Sp = mxq_attn_padded_keys(S);
+  if (Sp < 0 || HD < 128 || HD % 128 != 0 || HD > (int64_t(1) << 16)) return MXQ_ERR_SHAPE;
+  if (ldv < HD || ldv % 16 != 0) return MXQ_ERR_ALIGN;
+  if (!aligned(v_bf16, 32) || !aligned(codes_out, 16)) return MXQ_ERR_ALIGN;
+  DeviceInfo dev;
+  mxq_status st = current_device(&dev);
+  if (st != MXQ_OK) return st;
+  const dim3 grid(static_cast<unsigned>(HD / 128), static_cast<unsigned>(Sp / 128));
+  const auto* vp = static_cast<const uint16_t*>(v_bf16);
+  auto* cp = static_cast<uint8_t*>(codes_out);
+  auto* sp = static_cast<uint8_t*>(sf_out);
+  if (rule == MXQ_SCALE_UOS)
+    mxq::quantize_vt_kernel<true><<<grid, 256, 0, stream>>>(vp, S, ldv, Sp, cp, sp);
+  else
+    mxq::quantize_vt_kernel<false><<<grid, 256, 0, stream>>>(vp, S, ldv, Sp, cp, sp);
+  return launch_status();
+}
+
+mxq_status mxq_attention_mxfp4(const void* q_codes, const void* q_sf, const void* k_codes, const void* k_sf,
+                               const void* vt_codes, const void* vt_sf, int64_t S_q, int64_t S_kv, int64_t H,
+                               int64_t d, mxq_scale_rule rule, void* out_bf16, int64_t ldo, mxq_stream_t stream) {
+  if (!q_codes || !q_sf || !k_codes || !k_sf || !vt_codes || !vt_sf || !out_bf16) return MXQ_ERR_INVALID_ARG;
+  if (rule != MXQ_SCALE_OCP && rule != MXQ_SCALE_UOS) return MXQ_ERR_INVALID_ARG;
+  if (d != mxq::kAttnD) return MXQ_ERR_UNSUPPORTED;
+  const int64_t Sp = mxq_attn_padded_keys(S_kv);
+  if (Sp < 0 || S_q < 1 || S_q > (int64_t(65535) * mxq::kAttnBM) || H < 1 || H > 65535 || H * d > (int64_t(1) << 16))
+    return MXQ_ERR_SHAPE;
+  const int64_t HD = H * d;
+  if (ldo < HD || ldo % 8 != 0) return MXQ_ERR_ALIGN;
+  if (!aligned(q_codes, 16) || !aligned(k_codes, 16) || !aligned(vt_codes, 16) || !aligned(q_sf, 16) ||
+      !aligned(k_sf, 16) || !aligned(vt_sf, 16) || !aligned(out_bf16, 16))
+    return MXQ_ERR_ALIGN;
+  DeviceInfo dev;
+  mxq_status st = current_device(&dev);
+  if (st != MXQ_OK) return st;
+
+  CUtensorMap tq, tsq, tk, tsk, tv, tsv;
+  const bool ok =
+      make_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_codes, HD / 2, S_q, HD / 2, 64, mxq::kAttnBM,
+                   CU_TENSOR_MAP_SWIZZLE_64B) &&
+      make_tmap_sf(&tsq, q_sf, S_q, HD, 1, 1) &&
+      make_tmap_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_codes, HD / 2, S_kv, HD / 2, 64, mxq::kAttnBN,
+                   CU_TENSOR_MAP_SWIZZLE_64B) &&
+      make_tmap_sf(&tsk, k_sf, S_kv, HD, 1, 2) &&
+      make_tmap_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, vt_codes, Sp / 2, HD, Sp / 2, 128, mxq::kAttnD,
+                   CU_TENSOR_MAP_SWIZZLE_128B) &&
+      make_tmap_sf(&tsv, vt_sf, HD, Sp, 2, 1);
+  if (!ok) return MXQ_ERR_CUDA;
+
+  mxq::AttnParams prm;
+  {  // degree-7 Taylor coefficients of 2^g: a_0 = 1, a_k = a_(k-1) * ln 2 / k
+    double c = 1.0;
+    const double ln2 = std::log(2.0);
+    for (int k = 0; k < 8; ++k) {
+      prm.exp2c[k] = static_cast<float>(c);
+      c = c * ln2 / static_cast<double>(k + 1);
+    }
+  }
+  prm.t_scale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+  prm.Sq = static_cast<int>(S_q);
+  prm.Skv = static_cast<int>(S_kv);
+  prm.num_tiles = static_cast<int>(Sp / mxq::kAttnBN);
+
+  auto kernel = rule == MXQ_SCALE_UOS ? mxq::mx_attention_kernel<true> : mxq::mx_attention_kernel<false>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(mxq::mx_attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    mxq::kAttnSmemBytes);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(mxq::mx_attention_kernel<false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, mxq::kAttnSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return MXQ_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>((S_q + mxq::kAttnBM - 1) / mxq::kAttnBM), static_cast<unsigned>(H));
+  kernel<<<grid, mxq::kAttnThreads, mxq::kAttnSmemBytes, stream>>>(tq, tsq, tk, tsk, tv, tsv,
+                                                                   static_cast<__nv_bfloat16*>(out_bf16), ldo, prm);
+  return launch_status();
 }
 
 mxq_status mxq_debug_poll(void) {

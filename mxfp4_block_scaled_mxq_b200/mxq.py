@@ -26,7 +26,8 @@ MXQ_PREC_W4A4, MXQ_PREC_W4A4_TRANSFORM, MXQ_PREC_W4A8, MXQ_PREC_BF16 = 0, 1, 2, 
 
 EXPORTED = ("mxq_status_string", "mxq_sf_bytes", "mxq_quantize_act", "mxq_pack_weight", "mxq_gemm_w4a4",
             "mxq_gemm_w4a8", "mxq_dequant_mxfp4", "mxq_qdq_act", "mxq_channel_absmax", "mxq_smooth_factors",
-            "mxq_quantize_smooth", "mxq_sqnr_accumulate", "mxq_sqnr_db", "mxq_select_precision", "mxq_debug_poll")
+            "mxq_quantize_smooth", "mxq_sqnr_accumulate", "mxq_sqnr_db", "mxq_select_precision", "mxq_attn_padded_keys", "mxq_quantize_vt",
+            "mxq_attention_mxfp4", "mxq_debug_poll")
 
 
 class MxqError(RuntimeError):
@@ -75,6 +76,12 @@ def lib() -> ctypes.CDLL:
     L.mxq_sqnr_db.restype = ctypes.c_double
     L.mxq_select_precision.argtypes = [ctypes.c_double] * 4
     L.mxq_select_precision.restype = I32
+    L.mxq_attn_padded_keys.argtypes = [I64]
+    L.mxq_attn_padded_keys.restype = I64
+    L.mxq_quantize_vt.argtypes = [P, I64, I64, I64, I32, P, P, P]
+    L.mxq_quantize_vt.restype = I32
+    L.mxq_attention_mxfp4.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64, I32, P, I64, P]
+    L.mxq_attention_mxfp4.restype = I32
     L.mxq_debug_poll.argtypes = []
     L.mxq_debug_poll.restype = I32
     _lib = L
@@ -173,6 +180,22 @@ def mxq_sqnr_db(signal: float, noise: float) -> float:
 def mxq_select_precision(sqnr_plain_db: float, sqnr_transform_db: float, high_db: float, low_db: float) -> int:
     return int(lib().mxq_select_precision(float(sqnr_plain_db), float(sqnr_transform_db), float(high_db),
                                           float(low_db)))
+
+
+def mxq_attn_padded_keys(S_kv: int) -> int:
+    return int(lib().mxq_attn_padded_keys(int(S_kv)))
+
+
+def mxq_quantize_vt(v, S, HD, ldv, rule, codes_out, sf_out, stream=None) -> None:
+    _check(lib().mxq_quantize_vt(_ptr(v), int(S), int(HD), int(ldv), int(rule), _ptr(codes_out), _ptr(sf_out),
+                                 _stream(stream)), "mxq_quantize_vt")
+
+
+def mxq_attention_mxfp4(q_codes, q_sf, k_codes, k_sf, vt_codes, vt_sf, S_q, S_kv, H, d, rule, out, ldo,
+                        stream=None) -> None:
+    _check(lib().mxq_attention_mxfp4(_ptr(q_codes), _ptr(q_sf), _ptr(k_codes), _ptr(k_sf), _ptr(vt_codes),
+                                     _ptr(vt_sf), int(S_q), int(S_kv), int(H), int(d), int(rule), _ptr(out),
+                                     int(ldo), _stream(stream)), "mxq_attention_mxfp4")
 
 
 def mxq_debug_poll() -> int:
@@ -291,6 +314,33 @@ def quantize_smooth(x: torch.Tensor, chan_scale: torch.Tensor, rule: int = MXQ_S
     q, sf = out
     mxq_quantize_smooth(x.data_ptr(), rows, K, x.stride(0), rule, hadamard128, chan_scale, q, sf, stream)
     return q, sf
+
+
+def quantize_vt(v: torch.Tensor, rule: int = MXQ_SCALE_UOS, out=None, stream=None):
+    """V [S][H*d] -> V^T MXFP4 (codes [H*d][Sp/2], scales) with 32-key blocks."""
+    v = _bf16_2d(v, "v")
+    S, HD = v.shape
+    Sp = mxq_attn_padded_keys(S)
+    if out is None:
+        out = (torch.empty(HD, Sp // 2, dtype=torch.uint8, device=v.device),
+               torch.empty(mxq_sf_bytes(HD, Sp), dtype=torch.uint8, device=v.device))
+    mxq_quantize_vt(v.data_ptr(), S, HD, v.stride(0), rule, out[0], out[1], stream)
+    return out
+
+
+def attention_mxfp4(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, H: int, rule: int = MXQ_SCALE_UOS,
+                    out=None, stream=None) -> torch.Tensor:
+    """MXFP4 attention with UOS / PNQ: q [Sq][H*d], k, v [Skv][H*d] BF16 -> O [Sq][H*d] BF16.
+    Quantises Q, K (blocks along d) and V (blocks along the keys), then one attention launch."""
+    Sq, HD = q.shape
+    Skv = k.shape[0]
+    d = HD // H
+    qc, qs = quantize_act(q, rule, False, stream=stream)
+    kc, ks = quantize_act(k, rule, False, stream=stream)
+    vc, vs = quantize_vt(v, rule, stream=stream)
+    o = _out_bf16(Sq, HD, q.device) if out is None else out
+    mxq_attention_mxfp4(qc, qs, kc, ks, vc, vs, Sq, Skv, H, d, rule, o.data_ptr(), o.stride(0), stream)
+    return o
 
 
 def linear_w4a4(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE_OCP, hadamard128: bool = False,

@@ -68,11 +68,11 @@
 //    t = fl32(fl32(S) * fl32(log2(e) / sqrt(d))), relative to an integer offset
 //    c = ceil(max_j t_j) -- a power-of-two offset, under which E8M0 block scaling is
 //    exactly equivariant, so the codes do not depend on it; the exponential is
-//    2^(t - c) = p(g) * 2^(n - c) with n = floor(t), g = t - n - 1/2 and p the degree-7
-//    Taylor polynomial of 2^(g + 1/2) (coefficients a_0 = sqrt(2), a_k = a_(k-1) * ln 2 / k
-//    in FP64, rounded to FP32; Horner with FP32 fused multiply-adds), and numerators
-//    below 2^-126 are 0.  These FP32 steps decide the quantised codes, so they are
-//    taken in the kernel's precision; the rest is FP64.
+//    2^(t - c) = p(g) * 2^(n - c) with n = rint(t) (nearest, ties to even), g = t - n in
+//    [-1/2, 1/2] and p the degree-7 Taylor polynomial of 2^g (coefficients a_0 = 1,
+//    a_k = a_(k-1) * ln 2 / k in FP64, rounded to FP32; Horner with FP32 fused
+//    multiply-adds), and numerators with n - c < -126 are 0.  These FP32 steps decide the
+//    quantised codes, so they are taken in the kernel's precision; the rest is FP64.
 //  * Scale-factor memory layout (not given by the pages; a reading): rows padded
 //    to a multiple of 128, scale columns to a multiple of 4, 512-byte atoms of
 //    128 rows x 4 scale columns, byte
@@ -463,9 +463,9 @@ void oracle_gemm(int a_kind, const uint8_t* a_codes, const uint8_t* a_sf, int64_
 
 // ---------------------------------------------------------------- MXFP4 attention
 
-// Coefficients of the degree-7 Taylor polynomial of 2^(g + 1/2) around g = 0.
+// Coefficients of the degree-7 Taylor polynomial of 2^g around g = 0.
 static void pnq_exp2_coefficients(float* a) {
-  double c = std::sqrt(2.0);
+  double c = 1.0;
   const double ln2 = std::log(2.0);
   for (int k = 0; k < 8; ++k) {
     a[k] = static_cast<float>(c);
@@ -477,8 +477,8 @@ static void pnq_exp2_coefficients(float* a) {
 float oracle_pnq_exp2(float t, int chat) {
   float a[8];
   pnq_exp2_coefficients(a);
-  const float n = std::floor(t);
-  const float g = (t - n) - 0.5f;  // both steps exact
+  const float n = std::nearbyint(t);  // the default rounding mode: to nearest, ties to even
+  const float g = t - n;              // exact
   float p = a[7];
   for (int k = 6; k >= 0; --k) p = std::fmaf(p, g, a[k]);
   const long e = static_cast<long>(n) - chat;

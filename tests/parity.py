@@ -18,11 +18,11 @@ def sample_rows(M: int, n: int = 256) -> np.ndarray:
     spread with a stride across the whole range."""
     if M <= n:
         return np.arange(M, dtype=np.int64)
-    rows = set(range(min(32, M)))
+    rows = set(range(min(32, n // 4)))
     rows.add(M - 1)
     tail0 = (M - 1) // 128 * 128
-    rows.update(range(tail0, min(M, tail0 + 16)))
-    rows.update(np.linspace(0, M - 1, n - len(rows), dtype=np.int64).tolist())
+    rows.update(range(tail0, min(M, tail0 + min(16, n // 8))))
+    rows.update(np.linspace(0, M - 1, max(n - len(rows), 2), dtype=np.int64).tolist())
     return np.array(sorted(rows)[:n], dtype=np.int64)
 
 

@@ -174,6 +174,31 @@ def test_sqnr_validation_happens_before_any_launch(L):
     assert sq(FAKE + 8, 8, FAKE, 8, 4, 8, 0, FAKE, None) == ALIGN
 
 
+def test_attention_validation_happens_before_any_launch(L):
+    INV, SHAPE, ALIGN, UNSUP = 1, 2, 3, 4
+    assert L.mxq_attn_padded_keys(1) == 256 and L.mxq_attn_padded_keys(512) == 512
+    assert L.mxq_attn_padded_keys(0) == -1
+    vt = lambda *a: L.mxq_quantize_vt(*a)
+    assert vt(None, 10, 128, 128, 1, FAKE, FAKE, None) == INV
+    assert vt(FAKE, 10, 128, 128, 5, FAKE, FAKE, None) == INV
+    assert vt(FAKE, 0, 128, 128, 1, FAKE, FAKE, None) == SHAPE
+    assert vt(FAKE, 10, 96, 96, 1, FAKE, FAKE, None) == SHAPE                # HD % 128
+    assert vt(FAKE, 10, 128, 120, 1, FAKE, FAKE, None) == ALIGN              # ldv < HD
+    assert vt(FAKE + 16, 10, 128, 128, 1, FAKE, FAKE, None) == ALIGN         # v 32-byte aligned
+    at = lambda *a: L.mxq_attention_mxfp4(*a)
+    ok = [FAKE] * 6 + [100, 100, 2, 128, 1, FAKE, 256, None]
+    a = list(ok); a[0] = None
+    assert at(*a) == INV
+    a = list(ok); a[9] = 64
+    assert at(*a) == UNSUP                                                  # d != 128
+    a = list(ok); a[6] = 0
+    assert at(*a) == SHAPE
+    a = list(ok); a[12] = 200
+    assert at(*a) == ALIGN                                                  # ldo < H d
+    a = list(ok); a[11] = FAKE + 8
+    assert at(*a) == ALIGN
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):

@@ -1,0 +1,106 @@
+"""GPU parity of MXFP4 attention with UOS + PNQ (NEXT-1): the V^T quantiser bit for bit,
+and the attention output against the oracle's FP64 attention on the same quantised
+operands: max|O - O_ref| / max|O_ref| <= 5e-3 (BF16 output rounding and FP32
+accumulation; the numerators' codes are decided in the same FP32 arithmetic on both
+sides).
+
+[MXAttention: Data-Free Optimal Scaling and Pre-Normalization Quantization for MXFP4
+ Attention -- TL;DR, "What it actually does"]
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mxfp4_block_scaled_mxq_b200 import build, inputs, mxq
+from parity import assert_status_clean, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+ATTN_TOL = 5e-3
+D = 128
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    mxq.lib()
+    yield
+    assert_status_clean()
+
+
+@pytest.mark.parametrize("rule", [mxq.MXQ_SCALE_UOS, mxq.MXQ_SCALE_OCP])
+@pytest.mark.parametrize("S,HD", [(1, 128), (300, 256), (512, 128)])
+def test_quantize_vt_bit_exact(rule, S, HD):
+    v = inputs.heavy_tailed_bf16(S, HD, seed=S + HD)
+    codes, sf = mxq.quantize_vt(v.cuda(), rule)
+    torch.cuda.synchronize()
+    Sp = mxq.mxq_attn_padded_keys(S)
+    vt = torch.zeros(HD, Sp, dtype=torch.bfloat16)
+    vt[:, :S] = v.t()
+    want_c, want_sl = oracle.quantize_mxfp4(vt, rule=rule)
+    np.testing.assert_array_equal(codes.cpu().numpy(), want_c)
+    np.testing.assert_array_equal(sf.cpu().numpy(), oracle.sf_swizzle(want_sl, HD, Sp))
+
+
+def _check(q, k, v, H, rule=mxq.MXQ_SCALE_UOS, rows=None):
+    o = mxq.attention_mxfp4(q.cuda(), k.cuda(), v.cuda(), H, rule)
+    torch.cuda.synchronize()
+    Sq = q.shape[0]
+    rows = np.arange(Sq) if rows is None else rows
+    want, ws = oracle.attention_mxfp4(q, k, v, H, D, rows, rule=rule)
+    got = o.float().cpu().numpy()[rows].reshape(len(rows), H, D)
+    err = np.abs(got - want).max() / np.abs(want).max()
+    assert err <= ATTN_TOL, err
+    np.testing.assert_allclose(ws, 1.0, rtol=1e-12)
+    return err
+
+
+@pytest.mark.parametrize("Sq,Skv,H", [(1, 1, 1), (200, 300, 2), (128, 40, 1), (130, 512, 1), (257, 700, 2)])
+def test_attention_shapes(Sq, Skv, H):
+    """Ragged query tiles, a single partial key tile, exact and ragged key tiles."""
+    q = inputs.normal_bf16(Sq, H * D, 1.0, seed=Sq)
+    k = inputs.normal_bf16(Skv, H * D, 1.0, seed=Skv + 1)
+    v = inputs.normal_bf16(Skv, H * D, 1.0, seed=Skv + 2)
+    _check(q, k, v, H)
+
+
+@pytest.mark.parametrize("rule", [mxq.MXQ_SCALE_UOS, mxq.MXQ_SCALE_OCP])
+@pytest.mark.parametrize("scale", [0.25, 2.0])
+def test_attention_diffuse_and_peaked(rule, scale):
+    """Diffuse (small scores) and peaked (Q, K ~ N(0, 4)) attention, both rules."""
+    q = inputs.normal_bf16(160, 2 * D, scale, seed=11)
+    k = inputs.normal_bf16(600, 2 * D, scale, seed=12)
+    v = inputs.heavy_tailed_bf16(600, 2 * D, seed=13)
+    _check(q, k, v, 2, rule)
+
+
+def test_attention_rescales_when_the_maximum_jumps():
+    """Keys after the first tile score ~8x higher: the running offset moves by far more
+    than 8 in base 2, so O and l are rescaled in TMEM by exact powers of two."""
+    q = inputs.normal_bf16(128, D, 1.0, seed=21)
+    k = inputs.normal_bf16(768, D, 1.0, seed=22)
+    k[256:] = (k[256:].float() * 8.0).to(torch.bfloat16)
+    v = inputs.normal_bf16(768, D, 1.0, seed=23)
+    _check(q, k, v, 1)
+
+
+@pytest.mark.slow
+def test_full_size_wan_self_attention_sampled():
+    """Wan2.2-shaped self-attention (32760 tokens, 40 heads of 128): all heads on the
+    GPU; two heads' sampled query rows against the oracle."""
+    S, H = 32760, 40
+    q = inputs.normal_bf16(S, H * D, 1.0, seed=31, device="cuda")
+    k = inputs.normal_bf16(S, H * D, 1.0, seed=32, device="cuda")
+    v = inputs.heavy_tailed_bf16(S, H * D, seed=33, device="cuda")
+    o = mxq.attention_mxfp4(q, k, v, H)
+    torch.cuda.synchronize()
+    rows = sample_rows(S, 24)
+    for h in (0, 39):
+        cols = slice(h * D, (h + 1) * D)
+        want, _ = oracle.attention_mxfp4(q[:, cols].cpu().contiguous(), k[:, cols].cpu().contiguous(),
+                                         v[:, cols].cpu().contiguous(), 1, D, rows)
+        got = o[:, cols].float().cpu().numpy()[rows]
+        err = np.abs(got - want[:, 0, :]).max() / np.abs(want).max()
+        assert err <= ATTN_TOL, (h, err)

@@ -39,8 +39,17 @@ def test_pnq_exp2_offset_is_an_exact_power_of_two(t):
 
 
 def test_pnq_exp2_flushes_below_2_to_minus_126():
-    assert oracle.pnq_exp2(-127.5, 0) == 0.0
+    """Zero once the rounded integer part is below -126 (rint(-126.5) = -126: ties to even)."""
+    assert oracle.pnq_exp2(-127.0, 0) == 0.0
+    assert oracle.pnq_exp2(-126.6, 0) == 0.0
+    assert oracle.pnq_exp2(-126.5, 0) > 0.0
     assert oracle.pnq_exp2(-126.0, 0) > 0.0
+
+
+def test_pnq_exp2_is_exact_at_integers():
+    """g = 0 at integer t, and p(0) = a_0 = 1: an exact power of two."""
+    for t in (-100.0, -3.0, 0.0, 5.0):
+        assert oracle.pnq_exp2(t, 2) == 2.0 ** (t - 2)
 
 
 def test_equal_scores_average_the_values():
