@@ -8,9 +8,9 @@
 //
 // with Q, K in 32-blocks along the head dimension, V and P in 32-blocks along the keys,
 // c an integer offset (a power-of-two factor, under which the E8M0 block scaling is
-// exactly equivariant: the codes of P do not depend on it) and 2^(t - c) the degree-7
+// exactly equivariant: the codes of P do not depend on it) and 2^(t - c) the degree-4
 // Taylor polynomial of 2^g, g = t - rint(t), times 2^(rint(t) - c) (0 when rint(t) - c <
-// -126).  The row sum is taken over the quantised numerators
+// -126); a block's E8M0 exponent comes from the numerator of its largest score.  The row sum is taken over the quantised numerators
 // (PNQ), so the implied weights sum to one by construction; it is computed by the
 // tensor core itself: V^T carries one extra row of ones, so column d of the P V
 // accumulator is l.
@@ -23,8 +23,8 @@
 //               tile, O += P V^T (M 128, N 144: d columns + the ones row, K 256 keys);
 //               the next tile's scores are issued before the previous tile's P V, so
 //               the tensor core works while the softmax warps quantise.
-//   warps 2..9  softmax / PNQ, two threads per query row (keys [0,128) and [128,256) of
-//               the tile): scores from TMEM, the row maximum through shared memory, the
+//   warps 2..17 softmax / PNQ, four threads per query row (64 keys of the tile each):
+//               scores from TMEM, the row maximum through shared memory, the
 //               offset c raised only when the maximum passes c + 8 (then O, l are
 //               rescaled in TMEM by the exact power of two), numerators, UOS/OCP block
 //               scales and E2M1 codes written to shared memory in the 128-byte-swizzled
@@ -44,7 +44,8 @@ constexpr int kAttnD = 128;       // head dimension
 constexpr int kAttnBM = 128;      // queries per CTA
 constexpr int kAttnBN = 256;      // keys per tile
 constexpr int kAttnStages = 3;
-constexpr int kAttnThreads = 320;  // producer, MMA, 8 softmax warps
+constexpr int kAttnThreads = 576;  // producer, MMA, 16 softmax warps
+constexpr int kAttnSoftWarps = 16;  // four per TMEM lane quadrant: keys [64 q, +64) of a tile each
 constexpr int kAttnNv = kAttnD + 16;  // P V's N: the d value columns and 16 rows holding the ones row
 constexpr uint32_t kAttnTmemCols = 512;
 constexpr uint32_t kColS = 0;      // scores, 256 columns
@@ -64,8 +65,8 @@ constexpr int kAttnOffStages = kAttnQBytes + 1024;
 constexpr int kAttnOffP = kAttnOffStages + kAttnStages * kAttnStageBytes;
 constexpr int kAttnOffSfp = kAttnOffP + kAttnBM * 128;      // 2 atoms
 constexpr int kAttnOffSfOnes = kAttnOffSfp + 1024;          // 2 atoms of unit scales
-constexpr int kAttnOffRmax = kAttnOffSfOnes + 1024;         // float [2 parities][2 halves][128]
-constexpr int kAttnOffBar = kAttnOffRmax + 2048;
+constexpr int kAttnOffRmax = kAttnOffSfOnes + 1024;         // float [2 parities][4 quarters][128]
+constexpr int kAttnOffBar = kAttnOffRmax + 4096;
 constexpr int kAttnSmemBytes = 1024 + kAttnOffBar + 256;
 
 // Instruction descriptors (kind::mxf4 block_scale, E2M1 x E2M1, UE8M0 scales, K-major).
@@ -74,8 +75,10 @@ __host__ __device__ constexpr uint32_t attn_idesc(int n) {
          (static_cast<uint32_t>(kAttnBM >> 4) << 24);
 }
 
+constexpr int kExp2Terms = 5;  // degree-4 Taylor polynomial of 2^g (relative error < 6e-5)
+
 struct AttnParams {
-  float exp2c[8];  // Taylor coefficients a_k = (ln 2)^k / k! of 2^g, FP32
+  float exp2c[kExp2Terms];  // Taylor coefficients a_k = (ln 2)^k / k! of 2^g, FP32
   float t_scale;   // fl32(log2(e) / sqrt(d))
   int Sq;
   int Skv;
@@ -95,9 +98,9 @@ __device__ __forceinline__ float2 pnq_exp2_pair(float2 t, float lo, uint32_t bia
   const float2 r = __fadd2_rn(t, make_float2(kMagic, kMagic));
   const float2 n = __fadd2_rn(r, make_float2(-kMagic, -kMagic));
   const float2 g = __fadd2_rn(t, make_float2(-n.x, -n.y));
-  float2 p = make_float2(prm.exp2c[7], prm.exp2c[7]);
+  float2 p = make_float2(prm.exp2c[kExp2Terms - 1], prm.exp2c[kExp2Terms - 1]);
 #pragma unroll
-  for (int k = 6; k >= 0; --k) p = __ffma2_rn(p, g, make_float2(prm.exp2c[k], prm.exp2c[k]));
+  for (int k = kExp2Terms - 2; k >= 0; --k) p = __ffma2_rn(p, g, make_float2(prm.exp2c[k], prm.exp2c[k]));
   const float2 sc = make_float2(__uint_as_float(__float_as_uint(r.x) * 8388608u + bias_bits),
                                 __uint_as_float(__float_as_uint(r.y) * 8388608u + bias_bits));
   return __fmul2_rn(p, sc);
@@ -152,24 +155,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&kv_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 8);   // one arrival per softmax warp
-    mbar_init(p_full, 8);
+    mbar_init(s_free, kAttnSoftWarps);  // one arrival per softmax warp
+    mbar_init(p_full, kAttnSoftWarps);
     mbar_init(o_done, 1);
-    mbar_init(&rbar[0], 256);
-    mbar_init(&rbar[1], 256);
+    mbar_init(&rbar[0], 32 * kAttnSoftWarps);
+    mbar_init(&rbar[1], 32 * kAttnSoftWarps);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
   if (warp >= 2) {
     // Constant parts of the P V operand: the row of ones (row d = 128 of each V^T stage:
     // E2M1 1.0 = code 2 in every nibble; rows 129..143 zero) and their unit scales.
-    const int t = threadIdx.x - 64;  // 0..255
+    const int t = threadIdx.x - 64;  // 0..511
     for (int s = 0; s < kAttnStages; ++s) {
       uint32_t* ones = reinterpret_cast<uint32_t*>(sV(s) + kAttnD * 128);  // 16 rows x 128 B = 512 words
       ones[t] = t < 32 ? 0x22222222u : 0u;
-      ones[t + 256] = 0u;
     }
-    reinterpret_cast<uint32_t*>(sSfOnes)[t] = 0x7F7F7F7Fu;  // 2 atoms = 256 words
+    if (t < 256) reinterpret_cast<uint32_t*>(sSfOnes)[t] = 0x7F7F7F7Fu;  // 2 atoms = 256 words
     fence_proxy_async_smem();
   }
   if (warp == 1) {
@@ -270,9 +272,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------------ softmax / PNQ (warps 2..9)
+    // ------------------------------------------------------------------ softmax / PNQ (warps 2..17)
     const int quad = warp & 3;          // TMEM lanes [32 quad, +32)
-    const int hf = (warp - 2) >> 2;     // key half of every tile
+    const int qt = (warp - 2) >> 2;     // keys [64 qt, +64) of every tile
     const int r = quad * 32 + lane;     // query row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     int chat = 0;
@@ -280,35 +282,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int j = 0; j < nt; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(s_full, j & 1))) { ok = false; break; }
       tc_fence_after();
-      float t[128];
+      float t[64];
       {
         uint32_t v[64];
+        tmem_ld64(tmem + lane_off + kColS + 64 * qt, v);
+        tmem_ld_wait();
+        const float2 ts = make_float2(prm.t_scale, prm.t_scale);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tmem_ld64(tmem + lane_off + kColS + 128 * hf + 64 * c, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 64; ++i) t[64 * c + i] = __fmul_rn(__uint_as_float(v[i]), prm.t_scale);
+        for (int i = 0; i < 32; ++i) {
+          const float2 x = __fmul2_rn(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), ts);
+          t[2 * i] = x.x;
+          t[2 * i + 1] = x.y;
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);
       // keys past the end do not take part (only the last tile has any)
-      const int key0 = j * kAttnBN + 128 * hf;
-      if (key0 + 128 > prm.Skv) {
+      const int key0 = j * kAttnBN + 64 * qt;
+      if (key0 + 64 > prm.Skv) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
+        for (int i = 0; i < 64; ++i)
           if (key0 + i >= prm.Skv) t[i] = -INFINITY;
       }
-      float m = -INFINITY;
+      float bmax[2] = {-INFINITY, -INFINITY};  // per 32-key block
 #pragma unroll
-      for (int i = 0; i < 128; ++i) m = fmaxf(m, t[i]);
-      float* slot = sRmax + (j & 1) * 256;
-      slot[hf * 128 + r] = m;
+      for (int i = 0; i < 64; ++i) bmax[i >> 5] = fmaxf(bmax[i >> 5], t[i]);
+      float m = fmaxf(bmax[0], bmax[1]);
+      float* slot = sRmax + (j & 1) * 512;
+      slot[qt * 128 + r] = m;
       mbar_arrive(&rbar[j & 1]);
       if (!__all_sync(0xffffffffu, mbar_wait(&rbar[j & 1], (j >> 1) & 1))) { ok = false; break; }
-      m = fmaxf(m, slot[(1 - hf) * 128 + r]);  // finite: key j*256 is always valid
+      m = fmaxf(fmaxf(slot[r], slot[128 + r]), fmaxf(slot[256 + r], slot[384 + r]));  // finite: key j*256
       const int cand = static_cast<int>(ceilf(m));
       float rescale = 1.f;
       if (j == 0) {
@@ -317,19 +322,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         rescale = __int_as_float((127 + chat - cand) << 23);  // 2^(chat - cand), exact
         chat = cand;
       }
-      // numerators -> MXFP4 (4 blocks of 32 keys), kept as codes and scale bytes
+      // numerators -> MXFP4 (2 blocks of 32 keys), kept as codes and scale bytes
       const float lo = static_cast<float>(chat - 127);
       const uint32_t bias_bits = static_cast<uint32_t>(127 - chat) << 23;
-      uint32_t codes[16];
-      uint32_t sf_word = 0;
+      uint32_t codes[8];
+      uint32_t sf_half = 0;
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        float2 p[16];
-        float amax = 0.f;
+      for (int b = 0; b < 2; ++b) {
+        // the block exponent from the numerator of the block's largest score (0 if none)
+        const float amax = pnq_exp2_pair(make_float2(bmax[b], bmax[b]), lo, bias_bits, prm).x;
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          p[u] = pnq_exp2_pair(make_float2(t[32 * b + 2 * u], t[32 * b + 2 * u + 1]), lo, bias_bits, prm);
-          amax = fmaxf(amax, fmaxf(p[u].x, p[u].y));
+        for (int u = 0; u < 16; ++u) {  // in place: t becomes the numerators
+          const float2 p =
+              pnq_exp2_pair(make_float2(t[32 * b + 2 * u], t[32 * b + 2 * u + 1]), lo, bias_bits, prm);
+          t[32 * b + 2 * u] = p.x;
+          t[32 * b + 2 * u + 1] = p.y;
         }
         const int e = block_exponent<kUOS>(__float_as_uint(amax));
         const float s1 = exp2_neg(e);
@@ -339,12 +346,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           uint32_t word = 0;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const float2 v = __fmul2_rn(p[4 * w + q], sc);
+            const float2 v = __fmul2_rn(make_float2(t[32 * b + 8 * w + 2 * q], t[32 * b + 8 * w + 2 * q + 1]), sc);
             word |= e2m1x2(v.x, v.y) << (8 * q);
           }
           codes[4 * b + w] = word;
         }
-        sf_word |= static_cast<uint32_t>(e + 127) << (8 * b);
+        sf_half |= static_cast<uint32_t>(e + 127) << (8 * b);
       }
       // the previous tile's P V must be done before P is overwritten or O rescaled
       if (j > 0) {
@@ -352,14 +359,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
       }
       if (__any_sync(0xffffffffu, rescale != 1.f)) {
-        uint32_t v[64];
-        const uint32_t a0 = tmem + lane_off + kColO + 64 * hf;
-        tmem_ld64(a0, v);
+        uint32_t v[32];
+        const uint32_t a0 = tmem + lane_off + kColO + 32 * qt;
+        tmem_ld32(a0, *reinterpret_cast<uint32_t(*)[32]>(v));
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 64; ++i) v[i] = __float_as_uint(__fmul_rn(__uint_as_float(v[i]), rescale));
-        tmem_st64(a0, v);
-        if (hf == 0) {  // the l column block (column 128 and the zero columns after it)
+        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__fmul_rn(__uint_as_float(v[i]), rescale));
+        tmem_st32(a0, v);
+        if (qt == 0) {  // the l column block (column 128 and the zero columns after it)
           const uint32_t a1 = tmem + lane_off + kColO + kAttnD;
           tmem_ld16(a1, v);
           tmem_ld_wait();
@@ -369,14 +376,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         tmem_st_wait();
       }
-      // codes: row r, bytes [64 hf, +64) = 16-byte chunks 4 hf + b, 128-byte swizzle
+      // codes: row r, bytes [32 qt, +32) = 16-byte chunks 2 qt + b, 128-byte swizzle
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int chunk = (4 * hf + b) ^ (r & 7);
+      for (int b = 0; b < 2; ++b) {
+        const int chunk = (2 * qt + b) ^ (r & 7);
         *reinterpret_cast<uint4*>(sP + r * 128 + chunk * 16) =
             make_uint4(codes[4 * b], codes[4 * b + 1], codes[4 * b + 2], codes[4 * b + 3]);
       }
-      *reinterpret_cast<uint32_t*>(sSfp + hf * 512 + (r & 31) * 16 + (r >> 5) * 4) = sf_word;
+      *reinterpret_cast<uint16_t*>(sSfp + (qt >> 1) * 512 + (r & 31) * 16 + (r >> 5) * 4 + 2 * (qt & 1)) =
+          static_cast<uint16_t>(sf_half);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -385,16 +393,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ---------------------------------------------------------------- O / l -> BF16
     if (ok && __all_sync(0xffffffffu, mbar_wait(o_done, (nt - 1) & 1))) {
       tc_fence_after();
-      uint32_t v[64], lv[16];
-      tmem_ld64(tmem + lane_off + kColO + 64 * hf, v);
+      uint32_t v[32], lv[16];
+      tmem_ld32(tmem + lane_off + kColO + 32 * qt, *reinterpret_cast<uint32_t(*)[32]>(v));
       tmem_ld16(tmem + lane_off + kColO + kAttnD, lv);
       tmem_ld_wait();
       const float inv_l = __fdiv_rn(1.0f, __uint_as_float(lv[0]));
       const int64_t row = static_cast<int64_t>(q_tile) * kAttnBM + r;
       if (row < prm.Sq) {
-        uint4* dst = reinterpret_cast<uint4*>(out + row * ldo + head * kAttnD + 64 * hf);
+        uint4* dst = reinterpret_cast<uint4*>(out + row * ldo + head * kAttnD + 32 * qt);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q)

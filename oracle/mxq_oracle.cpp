@@ -69,10 +69,13 @@
 //    c = ceil(max_j t_j) -- a power-of-two offset, under which E8M0 block scaling is
 //    exactly equivariant, so the codes do not depend on it; the exponential is
 //    2^(t - c) = p(g) * 2^(n - c) with n = rint(t) (nearest, ties to even), g = t - n in
-//    [-1/2, 1/2] and p the degree-7 Taylor polynomial of 2^g (coefficients a_0 = 1,
+//    [-1/2, 1/2] and p the degree-4 Taylor polynomial of 2^g (coefficients a_0 = 1,
 //    a_k = a_(k-1) * ln 2 / k in FP64, rounded to FP32; Horner with FP32 fused
-//    multiply-adds), and numerators with n - c < -126 are 0.  These FP32 steps decide the
-//    quantised codes, so they are taken in the kernel's precision; the rest is FP64.
+//    multiply-adds; relative error below 6e-5, three orders of magnitude under the E2M1
+//    step), and numerators with n - c < -126 are 0.  A block's E8M0 exponent is taken from
+//    the numerator of its largest score (the exponential is monotone).  These FP32 steps
+//    decide the quantised codes, so they are taken in the kernel's precision; the rest is
+//    FP64.
 //  * Scale-factor memory layout (not given by the pages; a reading): rows padded
 //    to a multiple of 128, scale columns to a multiple of 4, 512-byte atoms of
 //    128 rows x 4 scale columns, byte
@@ -463,11 +466,13 @@ void oracle_gemm(int a_kind, const uint8_t* a_codes, const uint8_t* a_sf, int64_
 
 // ---------------------------------------------------------------- MXFP4 attention
 
-// Coefficients of the degree-7 Taylor polynomial of 2^g around g = 0.
+constexpr int kExp2Terms = 5;  // degree 4
+
+// Coefficients of the degree-4 Taylor polynomial of 2^g around g = 0.
 static void pnq_exp2_coefficients(float* a) {
   double c = 1.0;
   const double ln2 = std::log(2.0);
-  for (int k = 0; k < 8; ++k) {
+  for (int k = 0; k < kExp2Terms; ++k) {
     a[k] = static_cast<float>(c);
     c = c * ln2 / static_cast<double>(k + 1);
   }
@@ -475,12 +480,12 @@ static void pnq_exp2_coefficients(float* a) {
 
 // 2^(t - chat) by the definition above (t finite, chat an integer).
 float oracle_pnq_exp2(float t, int chat) {
-  float a[8];
+  float a[kExp2Terms];
   pnq_exp2_coefficients(a);
   const float n = std::nearbyint(t);  // the default rounding mode: to nearest, ties to even
   const float g = t - n;              // exact
-  float p = a[7];
-  for (int k = 6; k >= 0; --k) p = std::fmaf(p, g, a[k]);
+  float p = a[kExp2Terms - 1];
+  for (int k = kExp2Terms - 2; k >= 0; --k) p = std::fmaf(p, g, a[k]);
   const long e = static_cast<long>(n) - chat;
   if (e < -126) return 0.0f;
   return p * std::ldexp(1.0f, static_cast<int>(e));
@@ -548,8 +553,15 @@ void oracle_attention_mxfp4(const uint16_t* q, const uint16_t* k, const uint16_t
             for (int64_t j = 0; j < Sp; ++j) pt[j] = static_cast<float>(pt[j] / l);
           }
           for (int64_t b = 0; b < Sp / kBlock; ++b) {  // MXFP4 of the numerators, 32-key blocks
-            double amax = 0.0;
-            for (int u = 0; u < kBlock; ++u) amax = std::max(amax, static_cast<double>(pt[b * kBlock + u]));
+            // the block exponent from the numerator of the block's largest score
+            float bmax = -INFINITY;
+            for (int u = 0; u < kBlock; ++u)
+              if (b * kBlock + u < Skv) bmax = std::max(bmax, t[b * kBlock + u]);
+            double amax = bmax == -INFINITY ? 0.0 : static_cast<double>(oracle_pnq_exp2(bmax, chat));
+            if (mode == 1) {  // conventional order: the largest normalised probability
+              amax = 0.0;
+              for (int u = 0; u < kBlock; ++u) amax = std::max(amax, static_cast<double>(pt[b * kBlock + u]));
+            }
             const int e = oracle_block_exponent(amax, rule);
             for (int u = 0; u < kBlock; ++u) {
               const double x = std::ldexp(static_cast<double>(pt[b * kBlock + u]), -e);
