@@ -33,8 +33,82 @@
 #pragma once
 
 #include "gemm_common.cuh"
+#include "quantize.cuh"
 
 namespace mxq {
+
+// The activation quantiser fused into the GEMM (W4A4, no rotation).  The launch quantises
+// X into the A operand's own buffers while it multiplies: a task is 32 rows x 128 columns of
+// X (row-tile-major order, handed out by a global ticket) and four extra warps per CTA do
+// nothing but tasks until none are left; after a task's codes and scale bytes are stored,
+// `ready[row tile]` is raised with device-scope release semantics.  Before the first A load
+// of a tile, the producer waits (bounded) until its 128-row tile has all its 4 * K / 128
+// tasks, then fences the generic proxy against the async (TMA) proxy.  The quantiser warps
+// wait on nothing, so every task completes.
+struct FusedQuantArgs {
+  const uint16_t* x = nullptr;     // BF16 [M][ldx]
+  int64_t ldx = 0;
+  uint8_t* codes = nullptr;        // [M][K/2], the A codes the tensor map reads
+  uint8_t* sf = nullptr;           // A scales (atom layout), mxq_sf_bytes(M, K)
+  unsigned int* ready = nullptr;   // [row_tiles], zero at launch
+  unsigned int* ticket = nullptr;  // zero at launch
+  int row_tiles = 0;               // ceil(M / 128)
+  int tasks = 0;                   // row_tiles * 4 * K / 128
+  int uos = 0;
+};
+
+// One task on one warp: rows [128 rt + 32 qr, +32) x columns [128 kc, +128).  Lane l owns
+// in iteration i row 4 i + l / 8 of the 32 and elements [16 (l % 8), +16) (a 32-block is
+// split over lanes l, l ^ 1).  Rows at or beyond M read as zero (scale byte 0x00).
+template <bool kUOS>
+__device__ __forceinline__ void fused_quant_task(const FusedQuantArgs& fq, int task, int M, int K, int lane) {
+  const int kchunks = K / 128;
+  const int rt = task / (4 * kchunks);
+  const int rem = task - rt * 4 * kchunks;
+  const int kc = rem >> 2, qr = rem & 3;
+  const int l8 = lane & 7;
+  const int64_t k = static_cast<int64_t>(kc) * 128 + 16 * l8;
+  uint8_t* atom = fq.sf + (static_cast<int64_t>(rt) * kchunks + kc) * 512;
+  uint32_t w[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t row = static_cast<int64_t>(rt) * 128 + 32 * qr + 4 * i + (lane >> 3);
+    if (row < M) {
+      ld_stream_v8(fq.x + row * fq.ldx + k, w[i]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) w[i][j] = 0u;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int rr = 32 * qr + 4 * i + (lane >> 3);  // row within the 128-row tile
+    const int64_t row = static_cast<int64_t>(rt) * 128 + rr;
+    float f[16];
+    bf16x16_to_float(w[i], f);
+    uint32_t amax = bf16x16_absmax(w[i]);
+    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    const int e = block_exponent<kUOS>(amax);
+    const float s = exp2_neg(e);
+    uint32_t out[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint32_t packed = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        packed |= e2m1x2(__fmul_rn(f[8 * q + 2 * j], s), __fmul_rn(f[8 * q + 2 * j + 1], s)) << (8 * j);
+      out[q] = packed;
+    }
+    if (row < M) *reinterpret_cast<uint2*>(fq.codes + row * (K / 2) + k / 2) = make_uint2(out[0], out[1]);
+    if ((l8 & 1) == 0) atom[(rr & 31) * 16 + (rr >> 5) * 4 + (l8 >> 1)] = static_cast<uint8_t>(e + 127);
+  }
+  fence_proxy_async_global();
+  __syncwarp();
+  if (lane == 0) {
+    __threadfence();
+    counter_release_add(fq.ready + rt, 1u);
+  }
+}
 
 constexpr int kPairStages = 6;
 // two 256-column accumulators sharing [192, 256)
@@ -62,12 +136,18 @@ struct PairShape {
                                      (static_cast<uint32_t>(256 >> 4) << 24);
 };
 
-template <bool kW4A8>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+constexpr int kQuantWarps = 4;  // the fused launch's quantiser warps (warps 10..13)
+constexpr int kFusedThreads = kGemmThreads + 32 * kQuantWarps;
+
+// kFused: A is quantised inside the launch (W4A4 only; kUOS its scale rule), see above.
+template <bool kW4A8, bool kFused = false, bool kUOS = false>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFused ? kFusedThreads : kGemmThreads, 1)
     mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                         const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                         __nv_bfloat16* __restrict__ d, int64_t ldd, int d_vec32,
-                        const __nv_bfloat16* __restrict__ bias, int M, int N, int K, float alpha) {
+                        const __nv_bfloat16* __restrict__ bias, int M, int N, int K, float alpha,
+                        const FusedQuantArgs fq = FusedQuantArgs()) {
+  static_assert(!(kFused && kW4A8), "the fused quantiser produces MXFP4 activations");
   using S = PairShape<kW4A8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -131,9 +211,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       const uint64_t keep = l2_policy_evict_last();  // weights: reused by every row tile
+      int checked_rt = -1;
       for (int tile = cluster; tile < num_tiles; tile += nclusters) {
         const int mt = tile / n_tiles, nt = tile % n_tiles;
         bool ok = true;
+        if (kFused) {  // this CTA's 128 A rows must be quantised before they are loaded
+          const int rt = 2 * mt + static_cast<int>(rank);
+          if (rt < fq.row_tiles && rt != checked_rt) {
+            if (!counter_wait_geq(fq.ready + rt, static_cast<unsigned int>(4 * (K / 128)))) break;
+            fence_proxy_async_global();
+            checked_rt = rt;
+          }
+        }
         for (int ks = 0; ks < k_stages; ++ks) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(&full[stage], 2u * S::kTxPerCta);
@@ -209,10 +298,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         mbar_wait_drain(drain, 0);
       }
     }
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     // ------------------------------------------------------------------ epilogue (both CTAs)
     // Thread `lane` of warp (quad, chalf) owns output row 32*quad + lane of its CTA's
-    // 128 rows and columns [128*chalf, +128) of the tile.
+    // 128 rows and columns [128*chalf, +128) of the tile, drained 64 columns at a time.
     const int ew = warp - 2;
     const int quad = warp & 3;
     const int chalf = ew >> 2;
@@ -227,67 +316,71 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       // warp-uniform wait: tcgen05.ld below is .sync.aligned
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[a_idx], (it >> 1) & 1u))) break;
       tc_fence_after();
-      // v[j] = accumulator column 128 * chalf + j of this warp's 32 lanes.  The shared
-      // columns [192, 256) are this warp's upper half (accumulator 0, chalf 1) or its
-      // lower half (accumulator 1, chalf 0): those four warps load them first.
-      uint32_t v[128];
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + pair_acc_col(a_idx) + chalf * 128;
-      if (a_idx == 0 && chalf == 1) {
-        tmem_ld64(taddr + 64, v + 64);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(ovl_free_leader);
-        tmem_ld64(taddr, v);
-      } else if (a_idx == 1 && chalf == 0) {
-        tmem_ld64(taddr, v);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(ovl_free_leader);
-        tmem_ld64(taddr + 64, v + 64);
-      } else {
-        tmem_ld64(taddr, v);
-        tmem_ld64(taddr + 64, v + 64);
-      }
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(a_idx ? acc_free_leader1 : acc_free_leader0);
-
+      // The shared columns [192, 256) are this warp's upper half (accumulator 0, chalf 1) or
+      // its lower half (accumulator 1, chalf 0): those four warps drain them first, so the
+      // next tile's MMAs can start.
+      const bool shared_first = a_idx == 0 && chalf == 1;
+      const bool shared_holder = shared_first || (a_idx == 1 && chalf == 0);
       const int row = mt * 256 + static_cast<int>(rank) * 128 + quad * 32 + lane;
       __nv_bfloat16* drow = d + static_cast<int64_t>(row < M ? row : 0) * ldd;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int n0 = nt * 256 + chalf * 128 + 32 * c;
-        if (row >= M || n0 >= N) continue;
-        uint32_t packed[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          float b0 = 0.f, b1 = 0.f;
-          if (bias != nullptr) {
-            const int n = n0 + 2 * j;
-            if (n < N) b0 = __bfloat162float(bias[n]);
-            if (n + 1 < N) b1 = __bfloat162float(bias[n + 1]);
-          }
-          const float v0 = __fmaf_rn(alpha, __uint_as_float(v[32 * c + 2 * j]), b0);
-          const float v1 = __fmaf_rn(alpha, __uint_as_float(v[32 * c + 2 * j + 1]), b1);
-          packed[j] = pack_bf16x2(v0, v1);
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        const int half = shared_first ? 1 - h : h;  // 64-column half of this warp's 128
+        uint32_t v[64];
+        tmem_ld64(taddr + 64 * half, v);
+        tmem_ld_wait();
+        if (h == 0 && shared_holder) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(ovl_free_leader);
         }
-        if (d_vec32 && n0 + 32 <= N) {
-          st_global_v8_hint(drow + n0, packed, stream_out);
-          st_global_v8_hint(drow + n0 + 16, packed + 8, stream_out);
-        } else {
+        if (h == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(a_idx ? acc_free_leader1 : acc_free_leader0);
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int n0 = nt * 256 + chalf * 128 + 64 * half + 32 * c;
+          if (row >= M || n0 >= N) continue;
+          uint32_t packed[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int n = n0 + 2 * j;
-            if (n + 1 < N)
-              *reinterpret_cast<uint32_t*>(drow + n) = packed[j];
-            else if (n < N)
-              *reinterpret_cast<uint16_t*>(drow + n) = static_cast<uint16_t>(packed[j] & 0xFFFFu);
+            float b0 = 0.f, b1 = 0.f;
+            if (bias != nullptr) {
+              const int n = n0 + 2 * j;
+              if (n < N) b0 = __bfloat162float(bias[n]);
+              if (n + 1 < N) b1 = __bfloat162float(bias[n + 1]);
+            }
+            const float v0 = __fmaf_rn(alpha, __uint_as_float(v[32 * c + 2 * j]), b0);
+            const float v1 = __fmaf_rn(alpha, __uint_as_float(v[32 * c + 2 * j + 1]), b1);
+            packed[j] = pack_bf16x2(v0, v1);
+          }
+          if (d_vec32 && n0 + 32 <= N) {
+            st_global_v8_hint(drow + n0, packed, stream_out);
+            st_global_v8_hint(drow + n0 + 16, packed + 8, stream_out);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int n = n0 + 2 * j;
+              if (n + 1 < N)
+                *reinterpret_cast<uint32_t*>(drow + n) = packed[j];
+              else if (n < N)
+                *reinterpret_cast<uint16_t*>(drow + n) = static_cast<uint16_t>(packed[j] & 0xFFFFu);
+            }
           }
         }
       }
+    }
+  } else if (kFused) {
+    // ------------------------------------------------------------------ quantiser warps (fused)
+    while (true) {
+      int task = 0;
+      if (lane == 0) task = static_cast<int>(atomicAdd(fq.ticket, 1u));
+      task = __shfl_sync(0xffffffffu, task, 0);
+      if (task >= fq.tasks || status_set()) break;
+      fused_quant_task<kUOS>(fq, task, M, K, lane);
     }
   }
 

@@ -27,7 +27,7 @@ MXQ_PREC_W4A4, MXQ_PREC_W4A4_TRANSFORM, MXQ_PREC_W4A8, MXQ_PREC_BF16 = 0, 1, 2, 
 EXPORTED = ("mxq_status_string", "mxq_sf_bytes", "mxq_quantize_act", "mxq_pack_weight", "mxq_gemm_w4a4",
             "mxq_gemm_w4a8", "mxq_dequant_mxfp4", "mxq_qdq_act", "mxq_channel_absmax", "mxq_smooth_factors",
             "mxq_quantize_smooth", "mxq_sqnr_accumulate", "mxq_sqnr_db", "mxq_select_precision", "mxq_attn_padded_keys", "mxq_quantize_vt",
-            "mxq_attention_mxfp4", "mxq_debug_poll")
+            "mxq_attention_mxfp4", "mxq_linear_workspace_bytes", "mxq_linear_w4a4", "mxq_debug_poll")
 
 
 class MxqError(RuntimeError):
@@ -82,6 +82,10 @@ def lib() -> ctypes.CDLL:
     L.mxq_quantize_vt.restype = I32
     L.mxq_attention_mxfp4.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64, I32, P, I64, P]
     L.mxq_attention_mxfp4.restype = I32
+    L.mxq_linear_workspace_bytes.argtypes = [I64, I64]
+    L.mxq_linear_workspace_bytes.restype = I64
+    L.mxq_linear_w4a4.argtypes = [P, I64, I64, I64, I32, P, P, I64, F32, P, P, I64, P, I64, P]
+    L.mxq_linear_w4a4.restype = I32
     L.mxq_debug_poll.argtypes = []
     L.mxq_debug_poll.restype = I32
     _lib = L
@@ -196,6 +200,17 @@ def mxq_attention_mxfp4(q_codes, q_sf, k_codes, k_sf, vt_codes, vt_sf, S_q, S_kv
     _check(lib().mxq_attention_mxfp4(_ptr(q_codes), _ptr(q_sf), _ptr(k_codes), _ptr(k_sf), _ptr(vt_codes),
                                      _ptr(vt_sf), int(S_q), int(S_kv), int(H), int(d), int(rule), _ptr(out),
                                      int(ldo), _stream(stream)), "mxq_attention_mxfp4")
+
+
+def mxq_linear_workspace_bytes(M: int, K: int) -> int:
+    return int(lib().mxq_linear_workspace_bytes(int(M), int(K)))
+
+
+def mxq_linear_w4a4(x, M, K, ldx, rule, w_codes, w_sf, N, alpha, bias, workspace, workspace_bytes, d, ldd,
+                    stream=None) -> None:
+    _check(lib().mxq_linear_w4a4(_ptr(x), int(M), int(K), int(ldx), int(rule), _ptr(w_codes), _ptr(w_sf), int(N),
+                                 float(alpha), _ptr(bias), _ptr(workspace), int(workspace_bytes), _ptr(d), int(ldd),
+                                 _stream(stream)), "mxq_linear_w4a4")
 
 
 def mxq_debug_poll() -> int:
@@ -349,6 +364,23 @@ def linear_w4a4(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE_OC
     M, K = x.shape
     q, sf = quantize_act(x, rule, hadamard128, stream=stream)
     return gemm_w4a4(q, sf, w_codes, w_sf, M, N, K, 1.0, bias, stream=stream)
+
+
+def linear_workspace(M: int, K: int, device) -> torch.Tensor:
+    """A workspace for linear_w4a4_fused."""
+    return torch.empty(mxq_linear_workspace_bytes(M, K), dtype=torch.uint8, device=device)
+
+
+def linear_w4a4_fused(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE_OCP, alpha: float = 1.0,
+                      bias=None, workspace=None, out=None, stream=None) -> torch.Tensor:
+    """The quantized linear layer in one call (the activation quantiser fused into the GEMM)."""
+    x = _bf16_2d(x, "x")
+    M, K = x.shape
+    ws = linear_workspace(M, K, x.device) if workspace is None else workspace
+    d = _out_bf16(M, N, x.device) if out is None else out
+    mxq_linear_w4a4(x.data_ptr(), M, K, x.stride(0), rule, w_codes, w_sf, N, alpha, bias, ws, ws.numel(),
+                    d.data_ptr(), d.stride(0), stream)
+    return d
 
 
 def linear_w4a8(x: torch.Tensor, act_scale: float, w_codes, w_sf, N: int, bias=None, stream=None) -> torch.Tensor:
