@@ -42,8 +42,7 @@ FP4_PER_BF16 = 4.0                   # nominal FP4 : BF16 dense ratio (9 / 2.25 
 FP8_PER_BF16 = 2.0                   # nominal FP8 : BF16 dense ratio (4.5 / 2.25 PFLOP/s)
 # DRAM traffic per launch of the dominant kernel, from an ncu capture (see profiles/); None if
 # the kernel changed since the counters were taken.
-# Wan FFN: mean of the up (241.4 + 867.0 MB) and down (345.3 + 314.8 MB) GEMM launches.
-TRAFFIC = {"wan_ffn": (241.4e6 + 867.0e6 + 345.3e6 + 314.8e6) / 2}
+TRAFFIC = {}
 # Packed weight bytes per workload (MXFP4 codes + scales), for the L2-residency decision.
 W_BYTES = {"wan_ffn": 2 * 5120 * 13824 * 17 // 32, "wan_attn_hadamard": 4 * 5120 * 5120 * 17 // 32,
            "flux_w4a8": (9216 + 12288) * 3072 * 17 // 32, "m_sweep": 13824 * 5120 * 17 // 32, "qdq_wan_ffn": 0,
@@ -67,8 +66,6 @@ def parse():
                    default="wan_ffn")
     p.add_argument("--rule", choices=["ocp", "uos"], default=None,
                    help="activation scale rule (default: ocp; uos for the attention workload)")
-    p.add_argument("--unfused", action="store_true",
-                   help="Wan FFN: quantiser and GEMM as separate launches (default: the fused layer)")
     p.add_argument("--smooth", action="store_true",
                    help="SmoothQuant after the rotation (W4A4 workloads; factors calibrated before timing)")
     return p.parse_args()
@@ -227,7 +224,7 @@ def quant_bytes(M, K, fp8=False):
     return M * K * 2 + (M * K if fp8 else M * K // 2 + M * K // 32)
 
 
-def build_workload(name, dev, M, seed, rule_name, smooth=False, fused=True):
+def build_workload(name, dev, M, seed, rule_name, smooth=False):
     """Returns (description, parts, inputs [(device tensor)], outputs [(device tensor)], flops per step)."""
     import torch
     from mxfp4_block_scaled_mxq_b200 import inputs, mxq
@@ -268,29 +265,12 @@ def build_workload(name, dev, M, seed, rule_name, smooth=False, fused=True):
     if name == "wan_ffn":
         x_up, w_up = inputs.wan_ffn(seed=seed, which="up", device=dev, M=M)
         x_dn, w_dn = inputs.wan_ffn(seed=seed, which="down", device=dev, M=M)
-        if fused:  # one launch per layer: the activation quantiser runs inside the GEMM
-            p1, p2, outs = [], [], []
-            for label, x, w, parts_l in (("up", x_up, w_up, p1), ("down", x_dn, w_dn, p2)):
-                rows, K = x.shape
-                N = w.shape[0]
-                wc, wsf = mxq.pack_weight(w, mxq.MXQ_SCALE_OCP, False)
-                ws = mxq.linear_workspace(rows, K, dev)
-                d = out(rows, N)
-                outs.append(d)
-                parts_l.append(Part(f"linear_{label}", "gemm",
-                                    (lambda x=x, wc=wc, wsf=wsf, N=N, ws=ws, d=d:
-                                     mxq.linear_w4a4_fused(x, wc, wsf, N, rule, workspace=ws, out=d)),
-                                    flops=2.0 * rows * N * K))
-            d1, d2 = outs
-        else:
-            p1, _, d1 = w4a4_layer("up", x_up, w_up, False)
-            p2, _, d2 = w4a4_layer("down", x_dn, w_dn, False)
+        p1, _, d1 = w4a4_layer("up", x_up, w_up, False)
+        p2, _, d2 = w4a4_layer("down", x_dn, w_dn, False)
         rows = x_up.shape[0]
         desc = WORKLOAD if rows == M_TOK else WORKLOAD.replace("32760", str(rows))
         if rule_name == "uos":
             desc = desc.replace("OCP rule", "UOS rule")
-        desc += ("; the activation quantiser runs inside each GEMM launch" if fused
-                 else "; quantiser and GEMM as separate launches")
         return desc, p1 + p2, [x_up, x_dn], [d1, d2], sum(p.flops for p in p1 + p2)
 
     if name == "wan_attn_hadamard":
@@ -456,7 +436,7 @@ def main():
     M = args.m if args.m else default_m
     rule = args.rule or ("uos" if args.workload == "attn_wan" else "ocp")
     desc, parts, x_in, d_out, flops_step = build_workload(args.workload, dev, M, rank_seed(rank), rule,
-                                                          args.smooth, not args.unfused)
+                                                          args.smooth)
     stream = torch.cuda.current_stream(dev)
 
     def step():
@@ -569,7 +549,7 @@ def main():
                     "unit": "TFLOP/s", "frac": achieved_g / peak_of[gemm_kind],
                     "peak_source": f"{peak_kind} bf16_tflops (burst) x "
                                    f"{FP4_PER_BF16 if gemm_kind == 'fp4' else FP8_PER_BF16} (nominal ratio)",
-                    "traffic": TRAFFIC.get(args.workload) if M == M_TOK and args.unfused else None,
+                    "traffic": None,
                     "traffic_note": "DRAM bytes per GEMM launch, mean over the step's launches (ncu)"}
     else:
         roofline = {"bound": "hbm", "kernel": "quantize_act", "achieved": achieved_q, "peak": peaks["hbm_gbs"],

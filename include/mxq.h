@@ -167,22 +167,19 @@ MXQ_API mxq_status mxq_gemm_w4a8(const void* a_e4m3, float act_scale, const void
 /*
  * mxq_linear_w4a4 -- the quantized linear layer in one call:
  *   D[M][N] = bf16_rne(alpha * sum_k deq(Q(X))[m][k] * deqW[n][k] + bias[n]),
- * Q = the dynamic MXFP4 activation quantiser of mxq_quantize_act (rule `rule`, no rotation).
- * For M > 128 the quantiser runs inside the GEMM launch: the epilogue warps quantise 32-row
- * x 128-column pieces of X into the workspace while the tensor cores work, and each A tile is
- * loaded once its 128 rows are complete, so the activation pass overlaps the GEMM instead of
- * preceding it.  For M <= 128 it is the quantiser followed by the few-token GEMM.
- * [the layer: AMD Quark adds native W4A8 ... Wan2.2 -- "MXFP4 formats and precision levels";
- *  FLUX.1-dev MXFP4 page -- the GEMM takes the MX operands directly]
+ * Q = the dynamic MXFP4 activation quantiser of mxq_quantize_act (rule `rule`, no rotation),
+ * run into the caller's workspace, then the block-scaled GEMM of mxq_gemm_w4a4 (two launches
+ * on `stream`).  [the layer: AMD Quark adds native W4A8 ... Wan2.2 -- "MXFP4 formats and
+ * precision levels"; FLUX.1-dev MXFP4 page -- the GEMM takes the MX operands directly]
  *
  * x_bf16: [M][ldx] BF16, 32-byte aligned, ldx >= K, ldx % 16 == 0.  w_codes / w_sf: from
  * mxq_pack_weight (N rows).  bias_bf16, d_bf16, ldd and the shape limits as for mxq_gemm_w4a4
  * (K % 128 == 0), and M <= 8388480.
- * workspace: device, 16-byte aligned, at least mxq_linear_workspace_bytes(M, K) bytes,
- * owned by the caller.  After the call it holds the quantised activations: codes at offset 0
+ * workspace: device, 16-byte aligned, at least mxq_linear_workspace_bytes(M, K) bytes, owned
+ * by the caller.  After the call it holds the quantised activations: codes at offset 0
  * ([M][K/2], as mxq_quantize_act writes them), scales at offset ceil(M*K/2 / 1024) * 1024
- * (mxq_sf_bytes(M, K) bytes), then the launch's counters (cleared by each call on `stream`).
- * Calls that share a workspace must not overlap (issue them on one stream).
+ * (mxq_sf_bytes(M, K) bytes).  Calls that share a workspace must not overlap (issue them on
+ * one stream).
  */
 MXQ_API int64_t mxq_linear_workspace_bytes(int64_t M, int64_t K);
 

@@ -33,82 +33,8 @@
 #pragma once
 
 #include "gemm_common.cuh"
-#include "quantize.cuh"
 
 namespace mxq {
-
-// The activation quantiser fused into the GEMM (W4A4, no rotation).  The launch quantises
-// X into the A operand's own buffers while it multiplies: a task is 32 rows x 128 columns of
-// X (row-tile-major order, handed out by a global ticket) and four extra warps per CTA do
-// nothing but tasks until none are left; after a task's codes and scale bytes are stored,
-// `ready[row tile]` is raised with device-scope release semantics.  Before the first A load
-// of a tile, the producer waits (bounded) until its 128-row tile has all its 4 * K / 128
-// tasks, then fences the generic proxy against the async (TMA) proxy.  The quantiser warps
-// wait on nothing, so every task completes.
-struct FusedQuantArgs {
-  const uint16_t* x = nullptr;     // BF16 [M][ldx]
-  int64_t ldx = 0;
-  uint8_t* codes = nullptr;        // [M][K/2], the A codes the tensor map reads
-  uint8_t* sf = nullptr;           // A scales (atom layout), mxq_sf_bytes(M, K)
-  unsigned int* ready = nullptr;   // [row_tiles], zero at launch
-  unsigned int* ticket = nullptr;  // zero at launch
-  int row_tiles = 0;               // ceil(M / 128)
-  int tasks = 0;                   // row_tiles * 4 * K / 128
-  int uos = 0;
-};
-
-// One task on one warp: rows [128 rt + 32 qr, +32) x columns [128 kc, +128).  Lane l owns
-// in iteration i row 4 i + l / 8 of the 32 and elements [16 (l % 8), +16) (a 32-block is
-// split over lanes l, l ^ 1).  Rows at or beyond M read as zero (scale byte 0x00).
-template <bool kUOS>
-__device__ __forceinline__ void fused_quant_task(const FusedQuantArgs& fq, int task, int M, int K, int lane) {
-  const int kchunks = K / 128;
-  const int rt = task / (4 * kchunks);
-  const int rem = task - rt * 4 * kchunks;
-  const int kc = rem >> 2, qr = rem & 3;
-  const int l8 = lane & 7;
-  const int64_t k = static_cast<int64_t>(kc) * 128 + 16 * l8;
-  uint8_t* atom = fq.sf + (static_cast<int64_t>(rt) * kchunks + kc) * 512;
-  uint32_t w[8][8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int64_t row = static_cast<int64_t>(rt) * 128 + 32 * qr + 4 * i + (lane >> 3);
-    if (row < M) {
-      ld_stream_v8(fq.x + row * fq.ldx + k, w[i]);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) w[i][j] = 0u;
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int rr = 32 * qr + 4 * i + (lane >> 3);  // row within the 128-row tile
-    const int64_t row = static_cast<int64_t>(rt) * 128 + rr;
-    float f[16];
-    bf16x16_to_float(w[i], f);
-    uint32_t amax = bf16x16_absmax(w[i]);
-    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    const int e = block_exponent<kUOS>(amax);
-    const float s = exp2_neg(e);
-    uint32_t out[2];
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      uint32_t packed = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        packed |= e2m1x2(__fmul_rn(f[8 * q + 2 * j], s), __fmul_rn(f[8 * q + 2 * j + 1], s)) << (8 * j);
-      out[q] = packed;
-    }
-    if (row < M) *reinterpret_cast<uint2*>(fq.codes + row * (K / 2) + k / 2) = make_uint2(out[0], out[1]);
-    if ((l8 & 1) == 0) atom[(rr & 31) * 16 + (rr >> 5) * 4 + (l8 >> 1)] = static_cast<uint8_t>(e + 127);
-  }
-  fence_proxy_async_global();
-  __syncwarp();
-  if (lane == 0) {
-    __threadfence();
-    counter_release_add(fq.ready + rt, 1u);
-  }
-}
 
 constexpr int kPairStages = 6;
 // two 256-column accumulators sharing [192, 256)
@@ -136,18 +62,12 @@ struct PairShape {
                                      (static_cast<uint32_t>(256 >> 4) << 24);
 };
 
-constexpr int kQuantWarps = 4;  // the fused launch's quantiser warps (warps 10..13)
-constexpr int kFusedThreads = kGemmThreads + 32 * kQuantWarps;
-
-// kFused: A is quantised inside the launch (W4A4 only; kUOS its scale rule), see above.
-template <bool kW4A8, bool kFused = false, bool kUOS = false>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFused ? kFusedThreads : kGemmThreads, 1)
+template <bool kW4A8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                         const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                         __nv_bfloat16* __restrict__ d, int64_t ldd, int d_vec32,
-                        const __nv_bfloat16* __restrict__ bias, int M, int N, int K, float alpha,
-                        const FusedQuantArgs fq = FusedQuantArgs()) {
-  static_assert(!(kFused && kW4A8), "the fused quantiser produces MXFP4 activations");
+                        const __nv_bfloat16* __restrict__ bias, int M, int N, int K, float alpha) {
   using S = PairShape<kW4A8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -211,18 +131,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFused ? kFusedThrea
       int stage = 0;
       uint32_t phase = 0;
       const uint64_t keep = l2_policy_evict_last();  // weights: reused by every row tile
-      int checked_rt = -1;
       for (int tile = cluster; tile < num_tiles; tile += nclusters) {
         const int mt = tile / n_tiles, nt = tile % n_tiles;
         bool ok = true;
-        if (kFused) {  // this CTA's 128 A rows must be quantised before they are loaded
-          const int rt = 2 * mt + static_cast<int>(rank);
-          if (rt < fq.row_tiles && rt != checked_rt) {
-            if (!counter_wait_geq(fq.ready + rt, static_cast<unsigned int>(4 * (K / 128)))) break;
-            fence_proxy_async_global();
-            checked_rt = rt;
-          }
-        }
         for (int ks = 0; ks < k_stages; ++ks) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(&full[stage], 2u * S::kTxPerCta);
@@ -298,7 +209,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFused ? kFusedThrea
         mbar_wait_drain(drain, 0);
       }
     }
-  } else if (warp < 2 + kEpiWarps) {
+  } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
     // Thread `lane` of warp (quad, chalf) owns output row 32*quad + lane of its CTA's
     // 128 rows and columns [128*chalf, +128) of the tile, drained 64 columns at a time.
@@ -372,15 +283,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFused ? kFusedThrea
           }
         }
       }
-    }
-  } else if (kFused) {
-    // ------------------------------------------------------------------ quantiser warps (fused)
-    while (true) {
-      int task = 0;
-      if (lane == 0) task = static_cast<int>(atomicAdd(fq.ticket, 1u));
-      task = __shfl_sync(0xffffffffu, task, 0);
-      if (task >= fq.tasks || status_set()) break;
-      fused_quant_task<kUOS>(fq, task, M, K, lane);
     }
   }
 

@@ -99,12 +99,11 @@ bool make_tmap_sf(CUtensorMap* m, const void* base, int64_t rows, int64_t K, uin
 
 // Two-CTA path (one 256 x 256 tile per CTA pair), persistent over as many pairs as
 // can be resident at once.
-template <bool kW4A8, bool kFused = false, bool kUOS = false>
+template <bool kW4A8>
 mxq_status launch_gemm_pair(const void* a, const void* a_sf, const void* b, const void* b_sf, int64_t M, int64_t N,
-                            int64_t K, float alpha, const void* bias, void* d, int64_t ldd, cudaStream_t stream,
-                            const mxq::FusedQuantArgs& fq = mxq::FusedQuantArgs()) {
+                            int64_t K, float alpha, const void* bias, void* d, int64_t ldd, cudaStream_t stream) {
   using S = mxq::PairShape<kW4A8>;
-  auto kernel = mxq::mx_gemm_pair_kernel<kW4A8, kFused, kUOS>;
+  auto kernel = mxq::mx_gemm_pair_kernel<kW4A8>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   static int max_clusters = 0;
@@ -113,7 +112,7 @@ mxq_status launch_gemm_pair(const void* a, const void* a_sf, const void* b, cons
     if (attr_err != cudaSuccess) return;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
-    cfg.blockDim = dim3(kFused ? mxq::kFusedThreads : mxq::kGemmThreads, 1, 1);
+    cfg.blockDim = dim3(mxq::kGemmThreads, 1, 1);
     cfg.dynamicSmemBytes = S::kSmemBytes;
     attr_err = cudaOccupancyMaxActiveClusters(&max_clusters, kernel, &cfg);
   });
@@ -137,16 +136,15 @@ mxq_status launch_gemm_pair(const void* a, const void* a_sf, const void* b, cons
   const int clusters = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
   // 32-byte output stores need 32-byte aligned rows
   const int d_vec32 = (ldd % 16 == 0 && aligned(d, 32)) ? 1 : 0;
-  kernel<<<2 * clusters, kFused ? mxq::kFusedThreads : mxq::kGemmThreads, S::kSmemBytes, stream>>>(
+  kernel<<<2 * clusters, mxq::kGemmThreads, S::kSmemBytes, stream>>>(
       ta, tb, tsa, tsb, static_cast<__nv_bfloat16*>(d), ldd, d_vec32, static_cast<const __nv_bfloat16*>(bias),
-      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), alpha, fq);
+      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), alpha);
   return launch_status();
 }
 
-// Workspace of the fused linear layer: A codes, A scales, then the row-tile counters and
-// the task ticket (the only part that must start at zero).
+// Workspace of the quantized linear layer: the quantised activations (codes, then scales).
 struct LinearWorkspace {
-  int64_t codes = 0, sf = 0, counters = 0, bytes = 0;
+  int64_t codes = 0, sf = 0, bytes = 0;
 };
 
 LinearWorkspace linear_workspace(int64_t M, int64_t K) {
@@ -154,8 +152,7 @@ LinearWorkspace linear_workspace(int64_t M, int64_t K) {
   LinearWorkspace w;
   w.codes = 0;
   w.sf = up(M * (K / 2));
-  w.counters = w.sf + up((M + 127) / 128 * 128 * ((K / 32 + 3) / 4 * 4));
-  w.bytes = w.counters + up(((M + 127) / 128 + 1) * 4);
+  w.bytes = w.sf + up((M + 127) / 128 * 128 * ((K / 32 + 3) / 4 * 4));
   return w;
 }
 
@@ -613,31 +610,9 @@ mxq_status mxq_linear_w4a4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx
   DeviceInfo dev;
   st = current_device(&dev);
   if (st != MXQ_OK) return st;
-  if (M <= mxq::kBM) {  // few tokens: the weight-streaming kernel; quantising M rows is negligible
-    st = launch_mxfp4(false, x_bf16, M, K, ldx, rule, 0, a_codes, a_sf, stream);
-    if (st != MXQ_OK) return st;
-    return launch_gemm_swap<false>(dev, a_codes, a_sf, w_codes, w_sf, M, N, K, alpha, bias_bf16, d_bf16, ldd,
-                                   stream);
-  }
-  auto* counters = reinterpret_cast<unsigned int*>(base + ws.counters);
-  const int row_tiles = static_cast<int>((M + 127) / 128);
-  if (cudaMemsetAsync(counters, 0, static_cast<size_t>(row_tiles + 1) * 4, stream) != cudaSuccess)
-    return MXQ_ERR_CUDA;
-  mxq::FusedQuantArgs fq;
-  fq.x = static_cast<const uint16_t*>(x_bf16);
-  fq.ldx = ldx;
-  fq.codes = static_cast<uint8_t*>(a_codes);
-  fq.sf = static_cast<uint8_t*>(a_sf);
-  fq.ready = counters;
-  fq.ticket = counters + row_tiles;
-  fq.row_tiles = row_tiles;
-  fq.tasks = row_tiles * 4 * static_cast<int>(K / 128);
-  fq.uos = rule == MXQ_SCALE_UOS;
-  if (rule == MXQ_SCALE_UOS)
-    return launch_gemm_pair<false, true, true>(a_codes, a_sf, w_codes, w_sf, M, N, K, alpha, bias_bf16, d_bf16,
-                                               ldd, stream, fq);
-  return launch_gemm_pair<false, true, false>(a_codes, a_sf, w_codes, w_sf, M, N, K, alpha, bias_bf16, d_bf16, ldd,
-                                              stream, fq);
+  st = launch_mxfp4(false, x_bf16, M, K, ldx, rule, 0, a_codes, a_sf, stream);
+  if (st != MXQ_OK) return st;
+  return launch_gemm<false>(a_codes, a_sf, w_codes, w_sf, M, N, K, alpha, bias_bf16, d_bf16, ldd, stream);
 }
 
 mxq_status mxq_debug_poll(void) {

@@ -63,19 +63,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test (try_wait may suspend the thread for a while before it fails).
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Waits for the phase with the given parity to complete.  Returns false (after
 // recording a timeout) if it does not within kWaitLimitCycles, or as soon as
 // another thread of the grid has recorded one.
@@ -108,42 +95,6 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
 // ----------------------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// Orders this thread's generic-proxy global accesses before later async-proxy (TMA)
-// accesses, and the reverse.
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Device-scope release increment / acquire load of a counter in global memory.
-__device__ __forceinline__ void counter_release_add(unsigned int* p, unsigned int v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ unsigned int counter_acquire_load(const unsigned int* p) {
-  unsigned int v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Waits until *p >= target (written by other CTAs of this launch, all of them resident),
-// with the same bound as mbar_wait.
-__device__ __forceinline__ bool counter_wait_geq(const unsigned int* p, unsigned int target) {
-  if (counter_acquire_load(p) >= target) return true;
-  const long long t0 = clock64();
-  uint32_t spins = 0;
-  while (counter_acquire_load(p) < target) {
-    __nanosleep(64);
-    if ((++spins & 63u) == 0) {
-      if (status_set()) return false;
-      if (clock64() - t0 > kWaitLimitCycles) {
-        report_timeout();
-        return false;
-      }
-    }
-  }
-  return true;
 }
 
 // ----------------------------------------------------------------------------- TMA

@@ -367,13 +367,13 @@ def linear_w4a4(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE_OC
 
 
 def linear_workspace(M: int, K: int, device) -> torch.Tensor:
-    """A workspace for linear_w4a4_fused."""
+    """A workspace for linear_w4a4_ws (the quantised activations)."""
     return torch.empty(mxq_linear_workspace_bytes(M, K), dtype=torch.uint8, device=device)
 
 
-def linear_w4a4_fused(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE_OCP, alpha: float = 1.0,
-                      bias=None, workspace=None, out=None, stream=None) -> torch.Tensor:
-    """The quantized linear layer in one call (the activation quantiser fused into the GEMM)."""
+def linear_w4a4_ws(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE_OCP, alpha: float = 1.0,
+                   bias=None, workspace=None, out=None, stream=None) -> torch.Tensor:
+    """The quantized linear layer in one call of the C ABI (quantised activations in `workspace`)."""
     x = _bf16_2d(x, "x")
     M, K = x.shape
     ws = linear_workspace(M, K, x.device) if workspace is None else workspace

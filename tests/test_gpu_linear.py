@@ -1,6 +1,6 @@
-"""GPU parity of the fused quantized linear layer (activation quantiser inside the GEMM
-launch): D against the oracle's layer (GEMM tolerance), and the quantised activations
-the launch leaves in its workspace against the oracle's quantiser, bit for bit."""
+"""GPU parity of the one-call quantized linear layer (mxq_linear_w4a4): D against the
+oracle's layer (GEMM tolerance), and the quantised activations the call leaves in its
+workspace against the oracle's quantiser, bit for bit."""
 
 import numpy as np
 import pytest
@@ -26,7 +26,7 @@ def _run(x, w, rule=mxq.MXQ_SCALE_OCP, alpha=1.0, bias=None, workspace=None):
     wc, wsf = mxq.pack_weight(wd)
     M, K = x.shape
     ws = mxq.linear_workspace(M, K, "cuda") if workspace is None else workspace
-    d = mxq.linear_w4a4_fused(xd, wc, wsf, w.shape[0], rule, alpha, None if bias is None else bias.cuda(), ws)
+    d = mxq.linear_w4a4_ws(xd, wc, wsf, w.shape[0], rule, alpha, None if bias is None else bias.cuda(), ws)
     torch.cuda.synchronize()
     return d, ws
 
@@ -43,7 +43,7 @@ def _check_workspace(x, ws, rule):
 @pytest.mark.parametrize("rule", [mxq.MXQ_SCALE_OCP, mxq.MXQ_SCALE_UOS])
 @pytest.mark.parametrize("M,N,K", [(129, 256, 256), (300, 520, 1280), (1000, 264, 384), (257, 136, 640),
                                    (64, 392, 512)])
-def test_fused_layer(rule, M, N, K):
+def test_linear_layer(rule, M, N, K):
     x = inputs.heavy_tailed_bf16(M, K, seed=M + K)
     w = inputs.normal_bf16(N, K, 0.02, seed=N)
     d, ws = _run(x, w, rule)
@@ -52,8 +52,8 @@ def test_fused_layer(rule, M, N, K):
     _check_workspace(x, ws, rule)
 
 
-def test_fused_layer_bias_alpha_and_workspace_reuse():
-    """Two calls in a row on one workspace (the counters are cleared by each call)."""
+def test_linear_layer_bias_alpha_and_workspace_reuse():
+    """Two calls in a row on one workspace."""
     x1 = inputs.outlier_channels_bf16(700, 512, 0.02, 30.0, seed=41)
     x2 = inputs.heavy_tailed_bf16(700, 512, seed=42)
     w = inputs.normal_bf16(300, 512, 0.02, seed=43)
@@ -68,10 +68,10 @@ def test_fused_layer_bias_alpha_and_workspace_reuse():
 
 @pytest.mark.slow
 @pytest.mark.parametrize("which", ["up", "down"])
-def test_full_size_fused_wan_ffn(which):
+def test_full_size_linear_wan_ffn(which):
     x, w = inputs.wan_ffn(which=which, device="cuda")
     wc, wsf = mxq.pack_weight(w)
-    d = mxq.linear_w4a4_fused(x, wc, wsf, w.shape[0])
+    d = mxq.linear_w4a4_ws(x, wc, wsf, w.shape[0])
     torch.cuda.synchronize()
     rows = sample_rows(x.shape[0], 96)
     assert gemm_rel_err(d, rows, oracle_w4a4(x, w, rows)) <= GEMM_TOL
