@@ -190,6 +190,24 @@ MXQ_API mxq_status mxq_linear_w4a4(const void* x_bf16, int64_t M, int64_t K, int
                                    mxq_stream_t stream);
 
 /*
+ * mxq_linear_w4a4_static -- mxq_linear_w4a4 without a caller workspace, allocating nothing:
+ * the quantised activations go to a fixed buffer inside the library (one per device, a
+ * file-scope device array of MXQ_STATIC_SCRATCH_BYTES = 16 MiB, whose address is looked up
+ * once per device).  The pages have no counterpart of this call; it serves callers that
+ * cannot hand out device memory.  Returns MXQ_ERR_SHAPE when mxq_linear_workspace_bytes(M, K)
+ * exceeds the buffer (for K = 5120 about 6100 rows).  Nothing in the buffer needs to start at
+ * zero.  The buffer is shared by every call on the device: calls that overlap in time
+ * (different streams or host threads) race on it and must be serialised by the caller.
+ * Other arguments, limits and errors as for mxq_linear_w4a4.
+ */
+#define MXQ_STATIC_SCRATCH_BYTES (16ll << 20)
+
+MXQ_API mxq_status mxq_linear_w4a4_static(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                                          mxq_scale_rule rule, const void* w_codes, const void* w_sf,
+                                          int64_t N, float alpha, const void* bias_bf16, void* d_bf16,
+                                          int64_t ldd, mxq_stream_t stream);
+
+/*
  * mxq_dequant_mxfp4 -- out[r][k] = bf16(E2M1 value of code (r, k) * 2^(scale byte - 127)):
  * the MXFP4 -> BF16 expansion of a tensor in the layout above (weights from
  * mxq_pack_weight or activations from mxq_quantize_act).  Every product is a power of

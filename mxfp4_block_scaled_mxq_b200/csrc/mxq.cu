@@ -16,6 +16,10 @@
 #include "attention.cuh"
 #include "quantize.cuh"
 
+// Scratch of mxq_linear_w4a4_static: the quantised activations of one call, per device.
+constexpr int64_t kStaticScratchBytes = int64_t(16) << 20;
+static __device__ __align__(256) uint8_t g_linear_scratch[kStaticScratchBytes];
+
 namespace {
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -140,6 +144,18 @@ mxq_status launch_gemm_pair(const void* a, const void* a_sf, const void* b, cons
       ta, tb, tsa, tsb, static_cast<__nv_bfloat16*>(d), ldd, d_vec32, static_cast<const __nv_bfloat16*>(bias),
       static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), alpha);
   return launch_status();
+}
+
+// Device address of g_linear_scratch on device `dev`, looked up once per device.
+void* static_scratch(int dev) {
+  static void* addr[64];
+  static std::once_flag once[64];
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::call_once(once[dev], [dev] {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_linear_scratch) == cudaSuccess) addr[dev] = p;
+  });
+  return addr[dev];
 }
 
 // Workspace of the quantized linear layer: the quantised activations (codes, then scales).
@@ -613,6 +629,21 @@ mxq_status mxq_linear_w4a4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx
   st = launch_mxfp4(false, x_bf16, M, K, ldx, rule, 0, a_codes, a_sf, stream);
   if (st != MXQ_OK) return st;
   return launch_gemm<false>(a_codes, a_sf, w_codes, w_sf, M, N, K, alpha, bias_bf16, d_bf16, ldd, stream);
+}
+
+mxq_status mxq_linear_w4a4_static(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, mxq_scale_rule rule,
+                                  const void* w_codes, const void* w_sf, int64_t N, float alpha,
+                                  const void* bias_bf16, void* d_bf16, int64_t ldd, mxq_stream_t stream) {
+  const int64_t need = mxq_linear_workspace_bytes(M, K);
+  if (need < 0 || need > kStaticScratchBytes) return MXQ_ERR_SHAPE;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MXQ_ERR_CUDA;
+  void* scratch = static_scratch(dev);
+  if (!scratch) return MXQ_ERR_CUDA;
+  // Nothing in the scratch has to start at zero: the quantiser writes every byte the GEMM
+  // reads (codes of all M rows, whole scale atoms including their padding).
+  return mxq_linear_w4a4(x_bf16, M, K, ldx, rule, w_codes, w_sf, N, alpha, bias_bf16, scratch, kStaticScratchBytes,
+                         d_bf16, ldd, stream);
 }
 
 mxq_status mxq_debug_poll(void) {

@@ -27,7 +27,8 @@ MXQ_PREC_W4A4, MXQ_PREC_W4A4_TRANSFORM, MXQ_PREC_W4A8, MXQ_PREC_BF16 = 0, 1, 2, 
 EXPORTED = ("mxq_status_string", "mxq_sf_bytes", "mxq_quantize_act", "mxq_pack_weight", "mxq_gemm_w4a4",
             "mxq_gemm_w4a8", "mxq_dequant_mxfp4", "mxq_qdq_act", "mxq_channel_absmax", "mxq_smooth_factors",
             "mxq_quantize_smooth", "mxq_sqnr_accumulate", "mxq_sqnr_db", "mxq_select_precision", "mxq_attn_padded_keys", "mxq_quantize_vt",
-            "mxq_attention_mxfp4", "mxq_linear_workspace_bytes", "mxq_linear_w4a4", "mxq_debug_poll")
+            "mxq_attention_mxfp4", "mxq_linear_workspace_bytes", "mxq_linear_w4a4", "mxq_linear_w4a4_static",
+            "mxq_debug_poll")
 
 
 class MxqError(RuntimeError):
@@ -86,6 +87,8 @@ def lib() -> ctypes.CDLL:
     L.mxq_linear_workspace_bytes.restype = I64
     L.mxq_linear_w4a4.argtypes = [P, I64, I64, I64, I32, P, P, I64, F32, P, P, I64, P, I64, P]
     L.mxq_linear_w4a4.restype = I32
+    L.mxq_linear_w4a4_static.argtypes = [P, I64, I64, I64, I32, P, P, I64, F32, P, P, I64, P]
+    L.mxq_linear_w4a4_static.restype = I32
     L.mxq_debug_poll.argtypes = []
     L.mxq_debug_poll.restype = I32
     _lib = L
@@ -211,6 +214,12 @@ def mxq_linear_w4a4(x, M, K, ldx, rule, w_codes, w_sf, N, alpha, bias, workspace
     _check(lib().mxq_linear_w4a4(_ptr(x), int(M), int(K), int(ldx), int(rule), _ptr(w_codes), _ptr(w_sf), int(N),
                                  float(alpha), _ptr(bias), _ptr(workspace), int(workspace_bytes), _ptr(d), int(ldd),
                                  _stream(stream)), "mxq_linear_w4a4")
+
+
+def mxq_linear_w4a4_static(x, M, K, ldx, rule, w_codes, w_sf, N, alpha, bias, d, ldd, stream=None) -> None:
+    _check(lib().mxq_linear_w4a4_static(_ptr(x), int(M), int(K), int(ldx), int(rule), _ptr(w_codes), _ptr(w_sf),
+                                        int(N), float(alpha), _ptr(bias), _ptr(d), int(ldd), _stream(stream)),
+           "mxq_linear_w4a4_static")
 
 
 def mxq_debug_poll() -> int:
@@ -380,6 +389,17 @@ def linear_w4a4_ws(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE
     d = _out_bf16(M, N, x.device) if out is None else out
     mxq_linear_w4a4(x.data_ptr(), M, K, x.stride(0), rule, w_codes, w_sf, N, alpha, bias, ws, ws.numel(),
                     d.data_ptr(), d.stride(0), stream)
+    return d
+
+
+def linear_w4a4_static(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE_OCP, alpha: float = 1.0,
+                       bias=None, out=None, stream=None) -> torch.Tensor:
+    """The quantized linear layer with the library's own fixed scratch (no allocation by the call)."""
+    x = _bf16_2d(x, "x")
+    M, K = x.shape
+    d = _out_bf16(M, N, x.device) if out is None else out
+    mxq_linear_w4a4_static(x.data_ptr(), M, K, x.stride(0), rule, w_codes, w_sf, N, alpha, bias, d.data_ptr(),
+                           d.stride(0), stream)
     return d
 
 

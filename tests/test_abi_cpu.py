@@ -199,6 +199,12 @@ def test_attention_validation_happens_before_any_launch(L):
     assert at(*a) == ALIGN
 
 
+def test_static_scratch_rejects_oversize_before_any_launch(L):
+    SHAPE = 2
+    assert L.mxq_linear_w4a4_static(FAKE, 8192, 5120, 5120, 0, FAKE, FAKE, 256, 1.0, None, FAKE, 256, None) == SHAPE
+    assert L.mxq_linear_w4a4_static(FAKE, 10, 100, 128, 0, FAKE, FAKE, 256, 1.0, None, FAKE, 256, None) == SHAPE
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
