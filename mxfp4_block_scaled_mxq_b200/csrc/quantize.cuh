@@ -274,25 +274,24 @@ __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__
   }
 }
 
-// The rotated variant of the tile: two lanes per 128-element chunk, each holding 64
-// consecutive elements as 32 packed pairs P[i] = (t[i], t[i + 32]) -- so the pair's
-// halves are exactly the thread's two 32-element blocks.  Butterfly strides 1..16
-// run on packed pairs (FP32x2 add / fma with -1, both exact per half), stride 32 is
-// the within-pair butterfly, stride 64 is the one cross-lane exchange (xor 1); the
-// stage order and every rounding are those of the definition, so the rotated values
-// are bit-identical to the element-by-element butterfly.
+// The rotated variant of the tile: four lanes per 128-element chunk, lane j holding the
+// chunk's 32-block j as 16 packed pairs P[i] = (t[i], t[i + 16]).  Butterfly strides 1..8
+// run on packed pairs (FP32x2 add / fma with -1, both exact per half), stride 16 is the
+// within-pair butterfly, strides 32 and 64 are cross-lane exchanges (lanes xor 1 and xor 2);
+// the stage order and every rounding are those of the definition, so the rotated values are
+// bit-identical to the element-by-element butterfly.  A lane ends with exactly one 32-block:
+// its maximum, scale and 16 code bytes need no further exchange.  256 threads cover 64 rows
+// per pass, two passes per 128-row tile.
 template <bool kUOS, int kOut = kOutCodes, bool kSmooth = false>
 __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __restrict__ x, int64_t rows,
                                                              int64_t K, int64_t ld, const TileArgs& o) {
   constexpr bool kQdq = kOut == kOutQdq;
-  __shared__ __align__(16) uint8_t atom[512];
+  __shared__ __align__(16) uint8_t atom[512];  // scale atom, or the 128 column maxima (kOutAbsmax)
   __shared__ __align__(16) float s_chan[kSmooth ? 128 : 1];  // the tile's 128 channel factors
   const int tid = threadIdx.x;
-  const int r = tid >> 1;   // row within the tile
-  const int half = tid & 1; // elements [64 * half, +64) of the tile's 128 columns
-  const int64_t row = static_cast<int64_t>(blockIdx.y) * 128 + r;
-  const int64_t k = static_cast<int64_t>(blockIdx.x) * 128 + 64 * half;  // K % 128 == 0
-  const bool ok = row < rows;
+  const int lane = tid & 31;
+  const int j = tid & 3;  // 32-block of the chunk
+  const int64_t k = static_cast<int64_t>(blockIdx.x) * 128 + 32 * j;  // K % 128 == 0
 
   reinterpret_cast<uint32_t*>(atom)[tid & 127] = 0u;
   if constexpr (kSmooth) {
@@ -300,132 +299,130 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
       reinterpret_cast<float4*>(s_chan)[tid] =
           reinterpret_cast<const float4*>(o.chan + static_cast<int64_t>(blockIdx.x) * 128)[tid];
   }
-
-  float2 P[32];
-  {
-    uint32_t w[4][8];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if (ok) {
-        ld_stream_v8(x + row * ld + k + 16 * q, w[q]);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) w[q][j] = 0u;
-      }
-    }
-    // element j = 16 q + 2 jj (+1) sits in w[q][jj] (low / high half)
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int jl = i, jh = i + 32;
-      const uint32_t wl = w[jl >> 4][(jl & 15) >> 1], wh = w[jh >> 4][(jh & 15) >> 1];
-      P[i].x = __uint_as_float((jl & 1) ? (wl & 0xFFFF0000u) : (wl << 16));
-      P[i].y = __uint_as_float((jh & 1) ? (wh & 0xFFFF0000u) : (wh << 16));
-    }
-  }
   __syncthreads();  // atom zeroed, channel factors staged
 
-  const float2 minus1 = make_float2(-1.f, -1.f);
-#pragma unroll
-  for (int h = 1; h < 32; h *= 2) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      if (i & h) continue;
-      const float2 a = P[i], b = P[i + h];
-      P[i] = __fadd2_rn(a, b);
-      P[i + h] = __ffma2_rn(b, minus1, a);  // a - b, exactly rounded
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {  // stride 32: the two halves of each pair
-    const float a = P[i].x, b = P[i].y;
-    P[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
-  }
-  {  // stride 64 across the lane pair: lower lane t + partner, upper lane partner - t
-    const float sgn = half ? -1.f : 1.f;
-    const float2 sg = make_float2(sgn, sgn);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float2 p = make_float2(__shfl_xor_sync(0xffffffffu, P[i].x, 1), __shfl_xor_sync(0xffffffffu, P[i].y, 1));
-      P[i] = __ffma2_rn(P[i], sg, p);
-    }
-  }
   const float c = __uint_as_float(kInvSqrt128Bits);
   const float2 cc = make_float2(c, c);
-  if constexpr (kOut == kOutAbsmax) {
-    // column maxima over the 16 rows of this warp with the same `half` (lanes of one
-    // parity), then over the warps in shared memory, then into the global maxima
-    uint32_t* cmax = reinterpret_cast<uint32_t*>(atom);  // 128 columns, FP32 bits
+  const float2 minus1 = make_float2(-1.f, -1.f);
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const int r = 64 * pass + (tid >> 2);  // row within the tile
+    const int64_t row = static_cast<int64_t>(blockIdx.y) * 128 + r;
+    const bool ok = row < rows;
+    float2 P[16];
+    {
+      uint32_t w[2][8];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      float a = fabsf(__fmul_rn(P[i].x, c)), b = fabsf(__fmul_rn(P[i].y, c));
+      for (int q = 0; q < 2; ++q) {
+        if (ok) {
+          ld_stream_v8(x + row * ld + k + 16 * q, w[q]);
+        } else {
 #pragma unroll
-      for (int sh = 2; sh < 32; sh *= 2) {
-        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, sh));
-        b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, sh));
+          for (int u = 0; u < 8; ++u) w[q][u] = 0u;
+        }
       }
-      if ((tid & 31) < 2) {
-        atomicMax(cmax + 64 * half + i, __float_as_uint(a));
-        atomicMax(cmax + 64 * half + 32 + i, __float_as_uint(b));
+      // element i of the block sits in w[i / 16][(i % 16) / 2] (low / high half)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint32_t wl = w[0][i >> 1], wh = w[1][i >> 1];
+        P[i].x = __uint_as_float((i & 1) ? (wl & 0xFFFF0000u) : (wl << 16));
+        P[i].y = __uint_as_float((i & 1) ? (wh & 0xFFFF0000u) : (wh << 16));
       }
     }
-    __syncthreads();
-    if (tid < 128)
-      atomicMax(reinterpret_cast<unsigned int*>(o.chan_amax) + static_cast<int64_t>(blockIdx.x) * 128 + tid,
-                cmax[tid]);
-    return;
-  }
-  float m0 = 0.f, m1 = 0.f;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    P[i] = __fmul2_rn(P[i], cc);
-    if constexpr (kSmooth) P[i] = __fmul2_rn(P[i], make_float2(s_chan[64 * half + i], s_chan[64 * half + 32 + i]));
-    m0 = fmaxf(m0, fabsf(P[i].x));
-    m1 = fmaxf(m1, fabsf(P[i].y));
-  }
-  const int e0 = block_exponent<kUOS>(__float_as_uint(m0));
-  const int e1 = block_exponent<kUOS>(__float_as_uint(m1));
-  const float2 sc = make_float2(exp2_neg(e0), exp2_neg(e1));
-  uint32_t out[8];
+    for (int h = 1; h < 16; h *= 2) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint32_t lo = 0, hi = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 a = __fmul2_rn(P[8 * q + 2 * j], sc);
-      const float2 b = __fmul2_rn(P[8 * q + 2 * j + 1], sc);
-      lo |= e2m1x2(a.x, b.x) << (8 * j);  // block 0: elements 8q + 2j, 8q + 2j + 1
-      hi |= e2m1x2(a.y, b.y) << (8 * j);  // block 1: elements 32 + 8q + 2j, ...
+      for (int i = 0; i < 16; ++i) {
+        if (i & h) continue;
+        const float2 a = P[i], b = P[i + h];
+        P[i] = __fadd2_rn(a, b);
+        P[i + h] = __ffma2_rn(b, minus1, a);  // a - b, exactly rounded
+      }
     }
-    out[q] = lo;
-    out[4 + q] = hi;
-  }
-  if (kQdq) {
-    if (ok) {  // block 0 = elements [k, k+32) (out[0..3]), block 1 = [k+32, k+64) (out[4..7])
-      const float up0 = exp2_pos(e0), up1 = exp2_pos(e1);
 #pragma unroll
-      for (int blk = 0; blk < 2; ++blk) {
+    for (int i = 0; i < 16; ++i) {  // stride 16: the two halves of each pair
+      const float a = P[i].x, b = P[i].y;
+      P[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+#pragma unroll
+    for (int sh = 1; sh <= 2; sh <<= 1) {  // strides 32 (lanes xor 1) and 64 (lanes xor 2):
+      // the lower block gets own + partner, the upper partner - own
+      const float sgn = (j & sh) ? -1.f : 1.f;
+      const float2 sg = make_float2(sgn, sgn);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 p =
+            make_float2(__shfl_xor_sync(0xffffffffu, P[i].x, sh), __shfl_xor_sync(0xffffffffu, P[i].y, sh));
+        P[i] = __ffma2_rn(P[i], sg, p);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      P[i] = __fmul2_rn(P[i], cc);
+      if constexpr (kSmooth) P[i] = __fmul2_rn(P[i], make_float2(s_chan[32 * j + i], s_chan[32 * j + 16 + i]));
+    }
+    if constexpr (kOut == kOutAbsmax) {
+      // column maxima over the 8 rows of this warp with the same j (lanes xor 4, 8, 16),
+      // then over the warps and passes in shared memory
+      uint32_t* cmax = reinterpret_cast<uint32_t*>(atom);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float a = fabsf(P[i].x), b = fabsf(P[i].y);
+#pragma unroll
+        for (int sh = 4; sh < 32; sh *= 2) {
+          a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, sh));
+          b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, sh));
+        }
+        if (lane < 4) {
+          atomicMax(cmax + 32 * j + i, __float_as_uint(a));
+          atomicMax(cmax + 32 * j + 16 + i, __float_as_uint(b));
+        }
+      }
+      continue;
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fmaxf(fabsf(P[i].x), fabsf(P[i].y)));
+    const int e = block_exponent<kUOS>(__float_as_uint(m));
+    const float s1 = exp2_neg(e);
+    const float2 sc = make_float2(s1, s1);
+    uint32_t out[4];  // element 2q, 2q + 1 of word w: 8 w + 2 q (< 16: P[.].x, else P[. - 16].y)
+#pragma unroll
+    for (int wd = 0; wd < 4; ++wd) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int e0 = 8 * wd + 2 * q;
+        const float2 v = (e0 < 16) ? __fmul2_rn(make_float2(P[e0].x, P[e0 + 1].x), sc)
+                                   : __fmul2_rn(make_float2(P[e0 - 16].y, P[e0 - 15].y), sc);
+        word |= e2m1x2(v.x, v.y) << (8 * q);
+      }
+      out[wd] = word;
+    }
+    if (kQdq) {
+      if (ok) {
+        const float up = exp2_pos(e);
         uint32_t b[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          b[j] = e2m1x2_to_bf16x2((out[4 * blk + (j >> 2)] >> (8 * (j & 3))) & 0xFFu, blk ? up1 : up0);
-        uint4* dst = reinterpret_cast<uint4*>(o.qdq + row * o.ldq + k + 32 * blk);
+        for (int u = 0; u < 16; ++u) b[u] = e2m1x2_to_bf16x2((out[u >> 2] >> (8 * (u & 3))) & 0xFFu, up);
+        uint4* dst = reinterpret_cast<uint4*>(o.qdq + row * o.ldq + k);
 #pragma unroll
         for (int q = 0; q < 4; ++q) dst[q] = make_uint4(b[4 * q], b[4 * q + 1], b[4 * q + 2], b[4 * q + 3]);
       }
+    } else {
+      if (ok)
+        *reinterpret_cast<uint4*>(o.codes + row * (K / 2) + k / 2) = make_uint4(out[0], out[1], out[2], out[3]);
+      atom[(r & 31) * 16 + (r >> 5) * 4 + j] = static_cast<uint8_t>(e + 127);
     }
-    return;  // uniform: no scale atom to write
   }
-  if (ok) {
-    uint4* dst = reinterpret_cast<uint4*>(o.codes + row * (K / 2) + k / 2);  // 16-byte aligned
-    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-    *reinterpret_cast<uint16_t*>(atom + (r & 31) * 16 + (r >> 5) * 4 + 2 * half) =
-        static_cast<uint16_t>((e0 + 127) | ((e1 + 127) << 8));
-  }
+  if (kQdq) return;  // uniform: no scale atom to write
   __syncthreads();
-  if (tid < 32) {
-    const int64_t atoms_per_row_tile = K / 128;
-    const int64_t idx = static_cast<int64_t>(blockIdx.y) * atoms_per_row_tile + blockIdx.x;
+  if constexpr (kOut == kOutAbsmax) {
+    if (tid < 128)
+      atomicMax(reinterpret_cast<unsigned int*>(o.chan_amax) + static_cast<int64_t>(blockIdx.x) * 128 + tid,
+                reinterpret_cast<const uint32_t*>(atom)[tid]);
+  } else if (tid < 32) {
+    const int64_t idx = static_cast<int64_t>(blockIdx.y) * (K / 128) + blockIdx.x;
     reinterpret_cast<uint4*>(o.sf + idx * 512)[tid] = reinterpret_cast<const uint4*>(atom)[tid];
   }
 }
