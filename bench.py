@@ -42,7 +42,8 @@ FP4_PER_BF16 = 4.0                   # nominal FP4 : BF16 dense ratio (9 / 2.25 
 FP8_PER_BF16 = 2.0                   # nominal FP8 : BF16 dense ratio (4.5 / 2.25 PFLOP/s)
 # DRAM traffic per launch of the dominant kernel, from an ncu capture (see profiles/); None if
 # the kernel changed since the counters were taken.
-TRAFFIC = {}
+# Wan FFN: mean of the up (239.0 + 867.2 MB) and down (363.0 + 315.0 MB) GEMM launches.
+TRAFFIC = {"wan_ffn": (239.0e6 + 867.2e6 + 363.0e6 + 315.0e6) / 2}
 # Packed weight bytes per workload (MXFP4 codes + scales), for the L2-residency decision.
 W_BYTES = {"wan_ffn": 2 * 5120 * 13824 * 17 // 32, "wan_attn_hadamard": 4 * 5120 * 5120 * 17 // 32,
            "flux_w4a8": (9216 + 12288) * 3072 * 17 // 32, "m_sweep": 13824 * 5120 * 17 // 32, "qdq_wan_ffn": 0,
@@ -549,7 +550,7 @@ def main():
                     "unit": "TFLOP/s", "frac": achieved_g / peak_of[gemm_kind],
                     "peak_source": f"{peak_kind} bf16_tflops (burst) x "
                                    f"{FP4_PER_BF16 if gemm_kind == 'fp4' else FP8_PER_BF16} (nominal ratio)",
-                    "traffic": None,
+                    "traffic": TRAFFIC.get(args.workload) if M == M_TOK else None,
                     "traffic_note": "DRAM bytes per GEMM launch, mean over the step's launches (ncu)"}
     else:
         roofline = {"bound": "hbm", "kernel": "quantize_act", "achieved": achieved_q, "peak": peaks["hbm_gbs"],
