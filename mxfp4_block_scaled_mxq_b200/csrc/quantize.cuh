@@ -204,73 +204,72 @@ __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__
     __syncthreads();
     const int64_t col = static_cast<int64_t>(blockIdx.x) * 128 + tid;
     if (tid < 128 && col < K) atomicMax(reinterpret_cast<unsigned int*>(o.chan_amax) + col, cmax[tid]);
-    return;
-  }
-
-  float cm[16];  // kSmooth: this thread's 16 channel factors (the same for all its rows)
-  if constexpr (kSmooth) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 v = k_ok ? *reinterpret_cast<const float4*>(o.chan + k + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
-      cm[4 * q] = v.x;
-      cm[4 * q + 1] = v.y;
-      cm[4 * q + 2] = v.z;
-      cm[4 * q + 3] = v.w;
-    }
-  }
-
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = 16 * warp + 4 * i + (lane >> 3);  // row within the tile
-    const int64_t row = row0 + r;
-    float f[16];
-    bf16x16_to_float(w[i], f);
-    uint32_t amax;
+  } else {
+    float cm[16];  // kSmooth: this thread's 16 channel factors (the same for all its rows)
     if constexpr (kSmooth) {
-      float m = 0.f;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        f[j] = __fmul_rn(f[j], cm[j]);
-        m = fmaxf(m, fabsf(f[j]));
+      for (int q = 0; q < 4; ++q) {
+        const float4 v = k_ok ? *reinterpret_cast<const float4*>(o.chan + k + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
+        cm[4 * q] = v.x;
+        cm[4 * q + 1] = v.y;
+        cm[4 * q + 2] = v.z;
+        cm[4 * q + 3] = v.w;
       }
-      amax = __float_as_uint(m);
-    } else {
-      amax = bf16x16_absmax(w[i]);
     }
-    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));  // the other half of the block
-    const int e = block_exponent<kUOS>(amax);
-    const float s = exp2_neg(e);  // exact power of two
 
-    uint32_t out[2];
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      uint32_t packed = 0;
+    for (int i = 0; i < 4; ++i) {
+      const int r = 16 * warp + 4 * i + (lane >> 3);  // row within the tile
+      const int64_t row = row0 + r;
+      float f[16];
+      bf16x16_to_float(w[i], f);
+      uint32_t amax;
+      if constexpr (kSmooth) {
+        float m = 0.f;
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        packed |= e2m1x2(__fmul_rn(f[8 * q + 2 * j], s), __fmul_rn(f[8 * q + 2 * j + 1], s)) << (8 * j);
-      out[q] = packed;
-    }
-    if (kQdq) {
-      if (row < rows && k_ok) {
-        const float up = exp2_pos(e);
-        uint32_t b[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) b[j] = e2m1x2_to_bf16x2((out[j >> 2] >> (8 * (j & 3))) & 0xFFu, up);
-        uint4* dst = reinterpret_cast<uint4*>(o.qdq + row * o.ldq + k);
-        dst[0] = make_uint4(b[0], b[1], b[2], b[3]);
-        dst[1] = make_uint4(b[4], b[5], b[6], b[7]);
+        for (int j = 0; j < 16; ++j) {
+          f[j] = __fmul_rn(f[j], cm[j]);
+          m = fmaxf(m, fabsf(f[j]));
+        }
+        amax = __float_as_uint(m);
+      } else {
+        amax = bf16x16_absmax(w[i]);
       }
-    } else if (row < rows && k_ok) {
-      *reinterpret_cast<uint2*>(o.codes + row * (K / 2) + k / 2) = make_uint2(out[0], out[1]);
-      if ((l8 & 1) == 0) atom[(r & 31) * 16 + (r >> 5) * 4 + (l8 >> 1)] = static_cast<uint8_t>(e + 127);
+      amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));  // the other half of the block
+      const int e = block_exponent<kUOS>(amax);
+      const float s = exp2_neg(e);  // exact power of two
+
+      uint32_t out[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t packed = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          packed |= e2m1x2(__fmul_rn(f[8 * q + 2 * j], s), __fmul_rn(f[8 * q + 2 * j + 1], s)) << (8 * j);
+        out[q] = packed;
+      }
+      if (kQdq) {
+        if (row < rows && k_ok) {
+          const float up = exp2_pos(e);
+          uint32_t b[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) b[j] = e2m1x2_to_bf16x2((out[j >> 2] >> (8 * (j & 3))) & 0xFFu, up);
+          uint4* dst = reinterpret_cast<uint4*>(o.qdq + row * o.ldq + k);
+          dst[0] = make_uint4(b[0], b[1], b[2], b[3]);
+          dst[1] = make_uint4(b[4], b[5], b[6], b[7]);
+        }
+      } else if (row < rows && k_ok) {
+        *reinterpret_cast<uint2*>(o.codes + row * (K / 2) + k / 2) = make_uint2(out[0], out[1]);
+        if ((l8 & 1) == 0) atom[(r & 31) * 16 + (r >> 5) * 4 + (l8 >> 1)] = static_cast<uint8_t>(e + 127);
+      }
     }
-  }
-  if (kQdq) return;  // uniform: no scale atom to write
-  __syncthreads();
-  if (tid < 32) {
-    const int64_t atoms_per_row_tile = (K + 127) / 128;
-    const int64_t idx = static_cast<int64_t>(blockIdx.y) * atoms_per_row_tile + blockIdx.x;
-    reinterpret_cast<uint4*>(o.sf + idx * 512)[tid] = reinterpret_cast<const uint4*>(atom)[tid];
+    if (kQdq) return;  // uniform: no scale atom to write
+    __syncthreads();
+    if (tid < 32) {
+      const int64_t atoms_per_row_tile = (K + 127) / 128;
+      const int64_t idx = static_cast<int64_t>(blockIdx.y) * atoms_per_row_tile + blockIdx.x;
+      reinterpret_cast<uint4*>(o.sf + idx * 512)[tid] = reinterpret_cast<const uint4*>(atom)[tid];
+    }
   }
 }
 
