@@ -12,7 +12,7 @@
 //   [AMD Quark adds native W4A8 ... Wan2.2 -- "MXFP4 formats and precision levels",
 //    "Native execution paths"]
 //
-//   gemm_pair.cuh  M > 128: a two-CTA cluster per 256 x 256 output tile.
+//   gemm_pair.cuh  M > 128: a two-CTA cluster per 256 x 192 output tile.
 //   gemm_swap.cuh  M <= 128: one CTA per 128 weight rows, the tokens as the MMA's N.
 //
 // Every wait is bounded (ptx.cuh): on a timeout a kernel records MXQ_ERR_TIMEOUT,
@@ -28,7 +28,7 @@
 namespace mxq {
 
 constexpr int kBM = 128;           // rows of one CTA's share of a tile (TMEM lanes)
-constexpr int kBN = 256;           // output columns of a CTA-pair tile
+constexpr int kBN = 192;           // output columns of a CTA-pair tile
 constexpr int kGemmThreads = 320;  // CTA-pair kernel: producer, MMA and 8 epilogue warps
 constexpr int kEpiWarps = 8;
 constexpr uint32_t kTmemCols = 512;

@@ -1,12 +1,15 @@
 // gemm_pair.cuh -- the block-scaled GEMM (gemm_common.cuh) for M > 128 with a pair of
-// CTAs (a two-CTA thread-block cluster on two SMs) per 256 x 256 output tile.
+// CTAs (a two-CTA thread-block cluster on two SMs) per 256 x 192 output tile.
 //
-// One tcgen05.mma.cta_group::2 of M = 256 spans both SMs: CTA r holds rows
-// [128r, 128r + 128) of the A tile and of the B tile (the N half), its own A-row
-// scales and all 256 B-row scales, and accumulates D[its 128 rows][256] in its own
-// TMEM.  Compared with one CTA per 128 x 256 tile, each SM moves 64 instead of 96
-// bytes of operands per MMA clock out of L2 and through shared memory, and a stage
-// is 35 KB instead of 51 KB, so the ring is deeper.
+// One tcgen05.mma.cta_group::2 of M = 256, N = 192 spans both SMs: CTA r holds rows
+// [128r, 128r + 128) of the A tile and rows [96r, 96r + 96) of the B tile (its N
+// half), its own A-row scales and the scales of all 192 B rows, and accumulates
+// D[its 128 rows][192] in its own TMEM.  Compared with one CTA per 128-row tile, each
+// SM moves half the B operand per MMA clock out of L2 and through shared memory.
+//
+// B scales of an odd weight tile: rows [192 nt, 192 nt + 192) start 64 rows into a
+// 128-row scale atom.  The two covering atoms land in TMEM as 8 columns, one column per
+// 32 rows, so the MMA reads that tile's scales from 2 columns further on.
 //
 // Protocol (one elected thread per role):
 //   producer (warp 0, both CTAs)   waits its own `empty[s]`, loads its halves with
@@ -21,13 +24,11 @@
 //                                  LEADER's barriers, then scale / bias / round and
 //                                  store their 128 rows.
 //
-// Overlapping accumulators: a 256-column FP32 accumulator per tile leaves no room for
-// two disjoint buffers next to the scale columns, so tiles alternate between two
-// accumulators at TMEM columns 0 and 192 that share columns [192, 256).  The next
-// tile's MMAs need only (a) the previous tile's shared 64 columns drained -- the four
-// warps holding them load those first and arrive on `ovl_free` -- and (b) their own
-// accumulator fully drained two tiles ago (`acc_free[a]`).  The accumulator hand-off
-// then costs one 64-column TMEM load instead of the whole 256-column drain.
+// Two disjoint 192-column accumulators (TMEM columns [0, 192) and [192, 384)) beside the
+// scale columns: tiles alternate between them, so the next tile's MMAs wait only for the
+// drain of the tile two back (`acc_free[a]`), which the epilogue finished long before,
+// and the tensor pipe never idles at a tile boundary.  (256-column tiles would need two
+// accumulators sharing columns and a hand-off wait that cost 10 % of the mainloop.)
 // Every wait is bounded (ptx.cuh); the CTAs leave only after a final cluster
 // barrier, so neither frees TMEM or shared memory the pair's MMAs may still use.
 #pragma once
@@ -36,11 +37,11 @@
 
 namespace mxq {
 
-constexpr int kPairStages = 6;
-// two 256-column accumulators sharing [192, 256)
-__device__ __forceinline__ constexpr uint32_t pair_acc_col(uint32_t a) { return a ? 192u : 0u; }
-constexpr uint32_t kPairSfa = 448;           // A scales: 2 parities x 2 atoms x 4 columns
-constexpr uint32_t kPairSfb = 464;           // B scales: 2 parities x 2 atoms x 8 columns (to 496)
+constexpr int kPairStages = 7;
+__device__ __forceinline__ constexpr uint32_t pair_acc_col(uint32_t a) { return a * kBN; }
+constexpr uint32_t kPairSfa = 2 * kBN;       // A scales: 2 parities x 2 atoms x 4 columns
+constexpr uint32_t kPairSfb = kPairSfa + 16; // B scales: 2 parities x 2 atoms x 8 columns (to 432)
+static_assert(kPairSfb + 32 <= kTmemCols, "accumulators and scales exceed TMEM");
 
 template <bool kW4A8>
 struct PairShape {
@@ -50,15 +51,16 @@ struct PairShape {
   static constexpr int kMmas = kBK / kMmaK;            // MMAs per stage (4)
   static constexpr int kMmaPerAtom = 128 / kMmaK;
   static constexpr int kAStage = 128 * 128;            // this CTA's 128 A rows
-  static constexpr int kBStage = 128 * 128;            // this CTA's 128 B rows (8-bit containers for W4A8)
+  static constexpr int kBRows = kBN / 2;               // this CTA's B rows
+  static constexpr int kBStage = kBRows * 128;         // (8-bit containers for W4A8)
   static constexpr int kSfaStage = kW4A8 ? 0 : kAtoms * 512;
   static constexpr int kSfbStage = 2 * kAtoms * 512;   // [B row tile j][atom a], both halves of N
   static constexpr int kSfaConst = kW4A8 ? 512 : 0;
   static constexpr uint32_t kTxPerCta =
-      128 * 128 + (kW4A8 ? 128 * 64 : 128 * 128) + kSfaStage + kSfbStage;  // unpacked FP4 counts packed bytes
+      128 * 128 + (kW4A8 ? kBRows * 64 : kBRows * 128) + kSfaStage + kSfbStage;  // unpacked FP4 counts packed bytes
   static constexpr int kSmemBytes = 1024 + kPairStages * (kAStage + kBStage + kSfaStage + kSfbStage) + kSfaConst + 256;
   static constexpr uint32_t kIdesc = (kW4A8 ? (0u << 7) | (5u << 10) : (1u << 7) | (1u << 10)) |
-                                     (static_cast<uint32_t>(256 >> 3) << 17) | (1u << 23) |
+                                     (static_cast<uint32_t>(kBN >> 3) << 17) | (1u << 23) |
                                      (static_cast<uint32_t>(256 >> 4) << 24);
 };
 
@@ -79,8 +81,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t* empty = full + kPairStages;
   uint64_t* acc_full = empty + kPairStages;  // [2]
   uint64_t* acc_free = acc_full + 2;         // [2], leader's used
-  uint64_t* ovl_free = acc_free + 2;         // leader's used
-  uint64_t* drain = ovl_free + 1;
+  uint64_t* drain = acc_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -88,7 +89,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int m_tiles = (M + 255) / 256;
-  const int n_tiles = (N + 255) / 256;
+  const int n_tiles = (N + kBN - 1) / kBN;
   const int num_tiles = m_tiles * n_tiles;
   const int k_stages = (K + S::kBK - 1) / S::kBK;
   const int cluster = static_cast<int>(cluster_id_x());
@@ -107,7 +108,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_free[a], 2 * kEpiWarps);  // every epilogue warp of both CTAs
     }
-    mbar_init(ovl_free, kEpiWarps);  // the 4 warps per CTA that hold the shared columns
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -139,10 +139,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (leader) mbar_arrive_expect_tx(&full[stage], 2u * S::kTxPerCta);
           const uint32_t bar = map_to_rank(&full[stage], 0);
           tma_load_2d_pair(sA + stage * S::kAStage, &tmap_a, ks * 128, mt * 256 + rank * 128, bar);
-          tma_load_2d_pair_hint(sB + stage * S::kBStage, &tmap_b, ks * 128, nt * 256 + rank * 128, bar, keep);
+          tma_load_2d_pair_hint(sB + stage * S::kBStage, &tmap_b, ks * 128, nt * kBN + rank * S::kBRows, bar, keep);
           if (!kW4A8)
             tma_load_4d_pair(sSfa + stage * S::kSfaStage, &tmap_sfa, 0, 0, ks * S::kAtoms, 2 * mt + rank, bar);
-          tma_load_4d_pair(sSfb + stage * S::kSfbStage, &tmap_sfb, 0, 0, ks * S::kAtoms, 2 * nt, bar);
+          // the two 128-row scale atoms that cover the tile's B rows
+          tma_load_4d_pair(sSfb + stage * S::kSfbStage, &tmap_sfb, 0, 0, ks * S::kAtoms, nt * kBN / 128, bar);
           if (++stage == kPairStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
@@ -159,9 +160,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       for (int tile = cluster; ok && tile < num_tiles; tile += nclusters, ++it) {
         const uint32_t a_idx = it & 1u;
         if (!mbar_wait(&acc_free[a_idx], ((it >> 1) & 1u) ^ 1u)) { ok = false; break; }  // drained 2 tiles ago
-        if (!mbar_wait(ovl_free, (it & 1u) ^ 1u)) { ok = false; break; }               // previous tile's shared cols
         tc_fence_after();
         const uint32_t acc_col = pair_acc_col(a_idx);
+        // first B row of the tile within its first scale atom, in 32-row TMEM columns (0 or 2)
+        const uint32_t sfb_shift = static_cast<uint32_t>((tile % n_tiles) * kBN % 128) / 32u;
         for (int ks = 0; ks < k_stages; ++ks) {
           if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
           tc_fence_after();
@@ -192,7 +194,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const uint64_t adesc = smem_desc(a_base + kk * 32, 16, 1024, 2);
             const uint64_t bdesc = smem_desc(b_base + kk * 32, 16, 1024, 2);
             const uint32_t tsfa = kW4A8 ? tmem + kPairSfa : tmem + sfa_base + 4 * a;
-            const uint32_t tsfb = tmem + sfb_base + 8 * a;
+            const uint32_t tsfb = tmem + sfb_base + 8 * a + sfb_shift;
             if (kW4A8)
               tc_mma_mxf8f6f4_pair(tmem + acc_col, adesc, bdesc, idesc, tsfa, tsfb, (ks | kk) != 0);
             else
@@ -212,13 +214,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
     // Thread `lane` of warp (quad, chalf) owns output row 32*quad + lane of its CTA's
-    // 128 rows and columns [128*chalf, +128) of the tile, drained 64 columns at a time.
+    // 128 rows and columns [96*chalf, +96) of the tile: it loads all 96 accumulator
+    // columns, releases the accumulator, then scales, rounds and stores them.
+    constexpr int kCols = kBN / 2;
     const int ew = warp - 2;
     const int quad = warp & 3;
     const int chalf = ew >> 2;
     const uint32_t acc_free_leader0 = map_to_rank(&acc_free[0], 0);
     const uint32_t acc_free_leader1 = map_to_rank(&acc_free[1], 0);
-    const uint32_t ovl_free_leader = map_to_rank(ovl_free, 0);
     const uint64_t stream_out = l2_policy_evict_first();
     uint32_t it = 0;
     for (int tile = cluster; tile < num_tiles; tile += nclusters, ++it) {
@@ -227,59 +230,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       // warp-uniform wait: tcgen05.ld below is .sync.aligned
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[a_idx], (it >> 1) & 1u))) break;
       tc_fence_after();
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + pair_acc_col(a_idx) + chalf * 128;
-      // The shared columns [192, 256) are this warp's upper half (accumulator 0, chalf 1) or
-      // its lower half (accumulator 1, chalf 0): those four warps drain them first, so the
-      // next tile's MMAs can start.
-      const bool shared_first = a_idx == 0 && chalf == 1;
-      const bool shared_holder = shared_first || (a_idx == 1 && chalf == 0);
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + pair_acc_col(a_idx) + chalf * kCols;
+      uint32_t v[kCols];
+      tmem_ld64(taddr, *reinterpret_cast<uint32_t(*)[64]>(v));
+      tmem_ld32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(a_idx ? acc_free_leader1 : acc_free_leader0);
       const int row = mt * 256 + static_cast<int>(rank) * 128 + quad * 32 + lane;
-      __nv_bfloat16* drow = d + static_cast<int64_t>(row < M ? row : 0) * ldd;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        const int half = shared_first ? 1 - h : h;  // 64-column half of this warp's 128
-        uint32_t v[64];
-        tmem_ld64(taddr + 64 * half, v);
-        tmem_ld_wait();
-        if (h == 0 && shared_holder) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(ovl_free_leader);
-        }
-        if (h == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(a_idx ? acc_free_leader1 : acc_free_leader0);
-        }
+      if (row >= M) continue;
+      __nv_bfloat16* drow = d + static_cast<int64_t>(row) * ldd;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int n0 = nt * 256 + chalf * 128 + 64 * half + 32 * c;
-          if (row >= M || n0 >= N) continue;
-          uint32_t packed[16];
+      for (int c = 0; c < kCols / 32; ++c) {
+        const int n0 = nt * kBN + chalf * kCols + 32 * c;
+        if (n0 >= N) continue;
+        uint32_t packed[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float b0 = 0.f, b1 = 0.f;
+          if (bias != nullptr) {
+            const int n = n0 + 2 * j;
+            if (n < N) b0 = __bfloat162float(bias[n]);
+            if (n + 1 < N) b1 = __bfloat162float(bias[n + 1]);
+          }
+          const float v0 = __fmaf_rn(alpha, __uint_as_float(v[32 * c + 2 * j]), b0);
+          const float v1 = __fmaf_rn(alpha, __uint_as_float(v[32 * c + 2 * j + 1]), b1);
+          packed[j] = pack_bf16x2(v0, v1);
+        }
+        if (d_vec32 && n0 + 32 <= N) {
+          st_global_v8_hint(drow + n0, packed, stream_out);
+          st_global_v8_hint(drow + n0 + 16, packed + 8, stream_out);
+        } else {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            float b0 = 0.f, b1 = 0.f;
-            if (bias != nullptr) {
-              const int n = n0 + 2 * j;
-              if (n < N) b0 = __bfloat162float(bias[n]);
-              if (n + 1 < N) b1 = __bfloat162float(bias[n + 1]);
-            }
-            const float v0 = __fmaf_rn(alpha, __uint_as_float(v[32 * c + 2 * j]), b0);
-            const float v1 = __fmaf_rn(alpha, __uint_as_float(v[32 * c + 2 * j + 1]), b1);
-            packed[j] = pack_bf16x2(v0, v1);
-          }
-          if (d_vec32 && n0 + 32 <= N) {
-            st_global_v8_hint(drow + n0, packed, stream_out);
-            st_global_v8_hint(drow + n0 + 16, packed + 8, stream_out);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int n = n0 + 2 * j;
-              if (n + 1 < N)
-                *reinterpret_cast<uint32_t*>(drow + n) = packed[j];
-              else if (n < N)
-                *reinterpret_cast<uint16_t*>(drow + n) = static_cast<uint16_t>(packed[j] & 0xFFFFu);
-            }
+            const int n = n0 + 2 * j;
+            if (n + 1 < N)
+              *reinterpret_cast<uint32_t*>(drow + n) = packed[j];
+            else if (n < N)
+              *reinterpret_cast<uint16_t*>(drow + n) = static_cast<uint16_t>(packed[j] & 0xFFFFu);
           }
         }
       }

@@ -101,7 +101,7 @@ bool make_tmap_sf(CUtensorMap* m, const void* base, int64_t rows, int64_t K, uin
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Two-CTA path (one 256 x 256 tile per CTA pair), persistent over as many pairs as
+// Two-CTA path (one 256 x 192 tile per CTA pair), persistent over as many pairs as
 // can be resident at once.
 template <bool kW4A8>
 mxq_status launch_gemm_pair(const void* a, const void* a_sf, const void* b, const void* b_sf, int64_t M, int64_t N,
@@ -126,17 +126,18 @@ mxq_status launch_gemm_pair(const void* a, const void* a_sf, const void* b, cons
   bool ok;
   if (kW4A8) {
     ok = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K, M, K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, b, K, N, K / 2, 128, 128,
+         make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, b, K, N, K / 2, 128, S::kBRows,
                       CU_TENSOR_MAP_SWIZZLE_128B);
     tsa = tb;  // unused: E4M3 activations carry unit scales
   } else {
     ok = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K / 2, M, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K / 2, N, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K / 2, N, K / 2, 128, S::kBRows,
+                      CU_TENSOR_MAP_SWIZZLE_128B) &&
          make_tmap_sf(&tsa, a_sf, M, K, S::kAtoms, 1);
   }
   ok = ok && make_tmap_sf(&tsb, b_sf, N, K, S::kAtoms, 2);
   if (!ok) return MXQ_ERR_CUDA;
-  const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  const int64_t tiles = ((M + 255) / 256) * ((N + mxq::kBN - 1) / mxq::kBN);
   const int clusters = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
   // 32-byte output stores need 32-byte aligned rows
   const int d_vec32 = (ldd % 16 == 0 && aligned(d, 32)) ? 1 : 0;

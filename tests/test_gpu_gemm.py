@@ -55,17 +55,20 @@ def test_tiny_config():
 @pytest.mark.parametrize("M,N,K", [(1, 256, 256), (130, 200, 384), (257, 520, 128), (64, 1000, 640),
                                    (300, 256, 1280)])
 def test_ragged_tiles(M, N, K):
-    """M and N not multiples of the 128 x 256 tile, K % 256 == 128 (half last stage)."""
+    """M and N not multiples of the tiles (128 or 256 rows, 192 weight rows), K % 256 ==
+    128 (half last stage)."""
     x = inputs.heavy_tailed_bf16(M, K, seed=M)
     w = inputs.normal_bf16(N, K, 0.02, seed=N)
     check_w4a4(x, w)
 
 
 @pytest.mark.parametrize("M,N,K", [(129, 384, 384), (256, 128, 256), (257, 136, 640), (511, 264, 128),
-                                   (384, 512, 1152)])
+                                   (384, 512, 1152), (300, 1000, 256), (640, 1160, 384)])
 def test_cta_pair_edges(M, N, K):
     """Shapes for the two-CTA path (M > 128): a nearly empty second CTA, B tiles whose
-    second half is missing or ragged, a half last K stage, exact multiples."""
+    second half is missing or ragged, a half last K stage, exact multiples, and runs of
+    192-row weight tiles whose odd members start 64 rows into a scale atom (ending on an
+    odd or an even tile)."""
     x = inputs.heavy_tailed_bf16(M, K, seed=M + 7)
     w = inputs.normal_bf16(N, K, 0.02, seed=N + 7)
     check_w4a4(x, w)
