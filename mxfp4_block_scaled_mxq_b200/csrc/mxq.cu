@@ -173,13 +173,14 @@ LinearWorkspace linear_workspace(int64_t M, int64_t K) {
   return w;
 }
 
-// Few tokens (M <= 128): D^T = W X^T with the weights on the MMA's 128-row side.
-template <bool kW4A8>
-mxq_status launch_gemm_swap(const DeviceInfo& dev, const void* a, const void* a_sf, const void* b, const void* b_sf,
-                            int64_t M, int64_t N, int64_t K, float alpha, const void* bias, void* d, int64_t ldd,
-                            cudaStream_t stream) {
+// Few tokens (M <= 128): D^T = W X^T with the weights on the MMA's 128-row side; one
+// kernel instance per token tile width Mt (the tokens rounded up to 16).
+template <bool kW4A8, int Mt>
+mxq_status launch_gemm_swap_mt(const DeviceInfo& dev, const CUtensorMap& tw, const CUtensorMap& tt,
+                               const CUtensorMap& tsw, const CUtensorMap& tst, int64_t M, int64_t N, int64_t K,
+                               float alpha, const void* bias, void* d, int64_t ldd, cudaStream_t stream) {
   using S = mxq::SwapShape<kW4A8>;
-  auto kernel = mxq::mx_gemm_swap_kernel<kW4A8>;
+  auto kernel = mxq::mx_gemm_swap_kernel<kW4A8, Mt>;
   constexpr int kMaxSmem = 232448;  // opt-in shared memory per CTA on sm_100
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -187,11 +188,39 @@ mxq_status launch_gemm_swap(const DeviceInfo& dev, const void* a, const void* a_
     attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
   });
   if (attr_err != cudaSuccess) return MXQ_ERR_CUDA;
-  const int Mt = static_cast<int>((M + 15) / 16 * 16);
-  int stages = (kMaxSmem - S::kFixedBytes) / S::stage_bytes(Mt);
+  int stages = (kMaxSmem - S::kFixedBytes - S::out_bytes(Mt)) / S::stage_bytes(Mt);
   stages = stages > mxq::kSwapMaxStages ? mxq::kSwapMaxStages : stages;
-  const int smem = S::kFixedBytes + stages * S::stage_bytes(Mt);
+  const int smem = S::kFixedBytes + S::out_bytes(Mt) + stages * S::stage_bytes(Mt);
+  // D [M][N] BF16 written as [Mt][128] boxes (row stride ldd * 2 bytes: ldd % 8 == 0)
+  CUtensorMap td;
+  if (!make_tmap_2d(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, N, M, ldd * 2, 128, Mt, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return MXQ_ERR_CUDA;
+  const int64_t tiles = (N + 127) / 128;
+  const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+  // Programmatic stream serialisation: the kernel may start while the kernel before it
+  // (normally the activation quantiser) finishes; it waits for it before reading inputs.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(mxq::kSwapThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, tw, tt, tsw, tst, td,
+                                             static_cast<const __nv_bfloat16*>(bias), static_cast<int>(M),
+                                             static_cast<int>(N), static_cast<int>(K), alpha, stages);
+  return err == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
 
+template <bool kW4A8>
+mxq_status launch_gemm_swap(const DeviceInfo& dev, const void* a, const void* a_sf, const void* b, const void* b_sf,
+                            int64_t M, int64_t N, int64_t K, float alpha, const void* bias, void* d, int64_t ldd,
+                            cudaStream_t stream) {
+  using S = mxq::SwapShape<kW4A8>;
+  const int Mt = static_cast<int>((M + 15) / 16 * 16);
   CUtensorMap tw, tt, tsw, tst;
   bool ok;
   if (kW4A8) {
@@ -205,12 +234,14 @@ mxq_status launch_gemm_swap(const DeviceInfo& dev, const void* a, const void* a_
   }
   ok = ok && make_tmap_sf(&tsw, b_sf, N, K, S::kAtoms, 1);
   if (!ok) return MXQ_ERR_CUDA;
-  const int64_t tiles = (N + 127) / 128;
-  const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-  kernel<<<grid, mxq::kSwapThreads, smem, stream>>>(tw, tt, tsw, tst, static_cast<__nv_bfloat16*>(d), ldd,
-                                                    static_cast<const __nv_bfloat16*>(bias), static_cast<int>(M),
-                                                    static_cast<int>(N), static_cast<int>(K), alpha, stages);
-  return launch_status();
+  switch (Mt) {
+#define MXQ_SWAP_CASE(T) \
+  case T: return launch_gemm_swap_mt<kW4A8, T>(dev, tw, tt, tsw, tst, M, N, K, alpha, bias, d, ldd, stream);
+    MXQ_SWAP_CASE(16) MXQ_SWAP_CASE(32) MXQ_SWAP_CASE(48) MXQ_SWAP_CASE(64)
+    MXQ_SWAP_CASE(80) MXQ_SWAP_CASE(96) MXQ_SWAP_CASE(112) MXQ_SWAP_CASE(128)
+#undef MXQ_SWAP_CASE
+    default: return MXQ_ERR_SHAPE;
+  }
 }
 
 template <bool kW4A8>

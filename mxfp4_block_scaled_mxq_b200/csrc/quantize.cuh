@@ -439,6 +439,7 @@ template <bool kHadamard, bool kUOS>
 __global__ void __launch_bounds__(kQuantThreads) quantize_act_mxfp4_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ldx, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ sf) {
+  griddep_launch_dependents();  // a GEMM launched after this may run its prologue now
   TileArgs o;
   o.codes = codes;
   o.sf = sf;
@@ -571,6 +572,7 @@ __global__ void __launch_bounds__(kQuantThreads) dequant_mxfp4_kernel(const uint
 __global__ void __launch_bounds__(kQuantThreads) quantize_act_fp8_kernel(const uint16_t* __restrict__ x, int64_t M,
                                                                           int64_t K, int64_t ldx, float inv_scale,
                                                                           uint8_t* __restrict__ q) {
+  griddep_launch_dependents();  // a GEMM launched after this may run its prologue now
   const int64_t chunks_per_row = K / 16;
   const int64_t total = M * chunks_per_row;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;

@@ -100,9 +100,12 @@ def test_w4a8_few_tokens(M):
     assert gemm_rel_err(d, rows, oracle_w4a8(x, w, s, rows, bias=bias)) <= GEMM_TOL
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 13824, 512), (7, 136, 384), (33, 1000, 1280), (100, 392, 640)])
+@pytest.mark.parametrize("M,N,K", [(1, 13824, 512), (7, 136, 384), (33, 1000, 1280), (100, 392, 640),
+                                   (48, 20000, 256), (128, 19000, 384)])
 def test_few_token_shapes(M, N, K):
-    """Ragged M (rounded up to 16 for the MMA), N not a multiple of 128, K % 256 == 128."""
+    """Ragged M (rounded up to 16 for the MMA; 4, 2 or 1 accumulators), N not a multiple
+    of 128, K % 256 == 128, and more 128-row weight tiles than SMs, so that CTAs reuse
+    their shared-memory output tile for a second tile."""
     x = inputs.heavy_tailed_bf16(M, K, seed=3 * M + 1)
     w = inputs.normal_bf16(N, K, 0.02, seed=N + 3)
     bias = (torch.randn(N, generator=torch.Generator().manual_seed(N)) * 0.1).to(torch.bfloat16)
