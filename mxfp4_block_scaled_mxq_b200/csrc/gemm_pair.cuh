@@ -31,6 +31,7 @@
 // accumulators sharing columns and a hand-off wait that cost 10 % of the mainloop.)
 // Every wait is bounded (ptx.cuh); the CTAs leave only after a final cluster
 // barrier, so neither frees TMEM or shared memory the pair's MMAs may still use.
+// The kernel is launched with programmatic stream serialisation (griddep_wait below).
 #pragma once
 
 #include "gemm_common.cuh"
@@ -124,6 +125,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   cluster_sync();  // both CTAs hold their TMEM before the leader's first MMA
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Launched with programmatic stream serialisation: everything above, and an L2
+  // prefetch of the first weight stages, may overlap the kernel before this one (the
+  // activation quantiser); nothing that kernel may write is read before griddep_wait.
+  if (warp == 0 && lane == 0 && cluster < num_tiles) {
+    const int nt = cluster % n_tiles;
+    const int pre = kPairStages < k_stages ? kPairStages : k_stages;
+    for (int s = 0; s < pre; ++s) {
+      tma_prefetch_2d(&tmap_b, s * 128, nt * kBN + static_cast<int>(rank) * S::kBRows);
+      tma_prefetch_4d(&tmap_sfb, 0, 0, s * S::kAtoms, nt * kBN / 128);
+    }
+  }
+  griddep_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer (both CTAs)

@@ -72,6 +72,25 @@ mxq_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start while the kernel
+// before it in the stream (normally the activation quantiser, which lets dependents start)
+// finishes; the kernel executes griddepcontrol.wait before it reads any input.
+template <typename... KArgs, typename... Args>
+mxq_status launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t stream,
+                            Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
 // 2-D tensor map over a row-major [rows][cols] matrix.
 bool make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t cols, uint64_t rows,
                   uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
@@ -141,10 +160,10 @@ mxq_status launch_gemm_pair(const void* a, const void* a_sf, const void* b, cons
   const int clusters = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
   // 32-byte output stores need 32-byte aligned rows
   const int d_vec32 = (ldd % 16 == 0 && aligned(d, 32)) ? 1 : 0;
-  kernel<<<2 * clusters, mxq::kGemmThreads, S::kSmemBytes, stream>>>(
-      ta, tb, tsa, tsb, static_cast<__nv_bfloat16*>(d), ldd, d_vec32, static_cast<const __nv_bfloat16*>(bias),
-      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), alpha);
-  return launch_status();
+  return launch_dependent(kernel, dim3(static_cast<unsigned>(2 * clusters), 1, 1), dim3(mxq::kGemmThreads, 1, 1),
+                          S::kSmemBytes, stream, ta, tb, tsa, tsb, static_cast<__nv_bfloat16*>(d), ldd, d_vec32,
+                          static_cast<const __nv_bfloat16*>(bias), static_cast<int>(M), static_cast<int>(N),
+                          static_cast<int>(K), alpha);
 }
 
 // Device address of g_linear_scratch on device `dev`, looked up once per device.
@@ -197,22 +216,9 @@ mxq_status launch_gemm_swap_mt(const DeviceInfo& dev, const CUtensorMap& tw, con
     return MXQ_ERR_CUDA;
   const int64_t tiles = (N + 127) / 128;
   const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-  // Programmatic stream serialisation: the kernel may start while the kernel before it
-  // (normally the activation quantiser) finishes; it waits for it before reading inputs.
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-  cfg.blockDim = dim3(mxq::kSwapThreads, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, tw, tt, tsw, tst, td,
-                                             static_cast<const __nv_bfloat16*>(bias), static_cast<int>(M),
-                                             static_cast<int>(N), static_cast<int>(K), alpha, stages);
-  return err == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+  return launch_dependent(kernel, dim3(static_cast<unsigned>(grid), 1, 1), dim3(mxq::kSwapThreads, 1, 1), smem,
+                          stream, tw, tt, tsw, tst, td, static_cast<const __nv_bfloat16*>(bias), static_cast<int>(M),
+                          static_cast<int>(N), static_cast<int>(K), alpha, stages);
 }
 
 template <bool kW4A8>
