@@ -303,30 +303,34 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
   const float c = __uint_as_float(kInvSqrt128Bits);
   const float2 cc = make_float2(c, c);
   const float2 minus1 = make_float2(-1.f, -1.f);
-#pragma unroll 1
+  // both passes' rows are loaded before either is computed: the second pass's loads are
+  // in flight during the first pass's arithmetic
+  uint32_t w[2][2][8];
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int64_t row = static_cast<int64_t>(blockIdx.y) * 128 + 64 * pass + (tid >> 2);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      if (row < rows) {
+        ld_stream_v8(x + row * ld + k + 16 * q, w[pass][q]);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) w[pass][q][u] = 0u;
+      }
+    }
+  }
+#pragma unroll
   for (int pass = 0; pass < 2; ++pass) {
     const int r = 64 * pass + (tid >> 2);  // row within the tile
     const int64_t row = static_cast<int64_t>(blockIdx.y) * 128 + r;
     const bool ok = row < rows;
     float2 P[16];
-    {
-      uint32_t w[2][8];
+    // element i of the block sits in w[pass][i / 16][(i % 16) / 2] (low / high half)
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        if (ok) {
-          ld_stream_v8(x + row * ld + k + 16 * q, w[q]);
-        } else {
-#pragma unroll
-          for (int u = 0; u < 8; ++u) w[q][u] = 0u;
-        }
-      }
-      // element i of the block sits in w[i / 16][(i % 16) / 2] (low / high half)
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint32_t wl = w[0][i >> 1], wh = w[1][i >> 1];
-        P[i].x = __uint_as_float((i & 1) ? (wl & 0xFFFF0000u) : (wl << 16));
-        P[i].y = __uint_as_float((i & 1) ? (wh & 0xFFFF0000u) : (wh << 16));
-      }
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t wl = w[pass][0][i >> 1], wh = w[pass][1][i >> 1];
+      P[i].x = __uint_as_float((i & 1) ? (wl & 0xFFFF0000u) : (wl << 16));
+      P[i].y = __uint_as_float((i & 1) ? (wh & 0xFFFF0000u) : (wh << 16));
     }
 #pragma unroll
     for (int h = 1; h < 16; h *= 2) {
