@@ -343,13 +343,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float2 sc = make_float2(s1, s1);
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-          uint32_t word = 0;
+          float2 v[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 v = __fmul2_rn(make_float2(t[32 * b + 8 * w + 2 * q], t[32 * b + 8 * w + 2 * q + 1]), sc);
-            word |= e2m1x2(v.x, v.y) << (8 * q);
-          }
-          codes[4 * b + w] = word;
+          for (int q = 0; q < 4; ++q)
+            v[q] = __fmul2_rn(make_float2(t[32 * b + 8 * w + 2 * q], t[32 * b + 8 * w + 2 * q + 1]), sc);
+          codes[4 * b + w] = e2m1x8(v[0].x, v[0].y, v[1].x, v[1].y, v[2].x, v[2].y, v[3].x, v[3].y);
         }
         sf_half |= static_cast<uint32_t>(e + 127) << (8 * b);
       }
@@ -466,11 +464,10 @@ __global__ void __launch_bounds__(256) quantize_vt_kernel(const uint16_t* __rest
     uint32_t word[4];
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-      uint32_t x = 0;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        x |= e2m1x2(__fmul_rn(val(k0 + 8 * w + 2 * q), s), __fmul_rn(val(k0 + 8 * w + 2 * q + 1), s)) << (8 * q);
-      word[w] = x;
+      const int b = k0 + 8 * w;
+      word[w] = e2m1x8(__fmul_rn(val(b), s), __fmul_rn(val(b + 1), s), __fmul_rn(val(b + 2), s),
+                       __fmul_rn(val(b + 3), s), __fmul_rn(val(b + 4), s), __fmul_rn(val(b + 5), s),
+                       __fmul_rn(val(b + 6), s), __fmul_rn(val(b + 7), s));
     }
     const int64_t kb = key0 + k0;  // first key of the block
     *reinterpret_cast<uint4*>(codes + row * (Sp / 2) + kb / 2) = make_uint4(word[0], word[1], word[2], word[3]);
