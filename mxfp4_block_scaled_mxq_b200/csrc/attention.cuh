@@ -85,6 +85,20 @@ struct AttnParams {
   int num_tiles;   // ceil(Skv / 256)
 };
 
+// max(a, b, c) and min(a, b, c) in one instruction each (exact, like fmaxf / fminf; the
+// inputs are never NaN).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Numerators of a pair of keys: 2^(t - chat) = p(g) * 2^(n - chat), n = rint(t), g = t - n,
 // p the Taylor polynomial of 2^g (Horner, FP32 fused multiply-adds), 0 when n - chat < -126.
 // Everything runs on the FMA pipe: t is first raised to chat - 127 (masked keys at -inf and
@@ -92,9 +106,11 @@ struct AttnParams {
 // rint(t) in its low mantissa bits (|t| < 2^22), so n = r - 1.5 * 2^23 and g = t - n are
 // exact; and the FP32 bit pattern of 2^(n - chat) is (bits(r) + 127 - chat) * 2^23 modulo 2^32
 // (bits(1.5 * 2^23) * 2^23 vanishes modulo 2^32), one integer multiply-add, 0 for n - chat = -127.
+// kClamp = false skips the raise to chat - 127 for pairs already at or above it.
+template <bool kClamp = true>
 __device__ __forceinline__ float2 pnq_exp2_pair(float2 t, float lo, uint32_t bias_bits, const AttnParams& prm) {
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  t = make_float2(fmaxf(t.x, lo), fmaxf(t.y, lo));
+  if (kClamp) t = make_float2(fmaxf(t.x, lo), fmaxf(t.y, lo));
   const float2 r = __fadd2_rn(t, make_float2(kMagic, kMagic));
   const float2 n = __fadd2_rn(r, make_float2(-kMagic, -kMagic));
   const float2 g = __fadd2_rn(t, make_float2(-n.x, -n.y));
@@ -305,9 +321,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int i = 0; i < 64; ++i)
           if (key0 + i >= prm.Skv) t[i] = -INFINITY;
       }
-      float bmax[2] = {-INFINITY, -INFINITY};  // per 32-key block
+      float bmax[2], bmin[2];  // per 32-key block, three operands per instruction
 #pragma unroll
-      for (int i = 0; i < 64; ++i) bmax[i >> 5] = fmaxf(bmax[i >> 5], t[i]);
+      for (int b = 0; b < 2; ++b) {
+        float mb = t[32 * b], nb = t[32 * b];
+#pragma unroll
+        for (int i = 1; i < 31; i += 2) {
+          mb = fmax3(mb, t[32 * b + i], t[32 * b + i + 1]);
+          nb = fmin3(nb, t[32 * b + i], t[32 * b + i + 1]);
+        }
+        bmax[b] = fmaxf(mb, t[32 * b + 31]);
+        bmin[b] = fminf(nb, t[32 * b + 31]);
+      }
       float m = fmaxf(bmax[0], bmax[1]);
       float* slot = sRmax + (j & 1) * 512;
       slot[qt * 128 + r] = m;
@@ -331,12 +356,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int b = 0; b < 2; ++b) {
         // the block exponent from the numerator of the block's largest score (0 if none)
         const float amax = pnq_exp2_pair(make_float2(bmax[b], bmax[b]), lo, bias_bits, prm).x;
+        if (bmin[b] >= lo) {  // no key of the block below chat - 127 (the usual case)
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {  // in place: t becomes the numerators
-          const float2 p =
-              pnq_exp2_pair(make_float2(t[32 * b + 2 * u], t[32 * b + 2 * u + 1]), lo, bias_bits, prm);
-          t[32 * b + 2 * u] = p.x;
-          t[32 * b + 2 * u + 1] = p.y;
+          for (int u = 0; u < 16; ++u) {  // in place: t becomes the numerators
+            const float2 p =
+                pnq_exp2_pair<false>(make_float2(t[32 * b + 2 * u], t[32 * b + 2 * u + 1]), lo, bias_bits, prm);
+            t[32 * b + 2 * u] = p.x;
+            t[32 * b + 2 * u + 1] = p.y;
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const float2 p =
+                pnq_exp2_pair<true>(make_float2(t[32 * b + 2 * u], t[32 * b + 2 * u + 1]), lo, bias_bits, prm);
+            t[32 * b + 2 * u] = p.x;
+            t[32 * b + 2 * u + 1] = p.y;
+          }
         }
         const int e = block_exponent<kUOS>(__float_as_uint(amax));
         const float s1 = exp2_neg(e);
