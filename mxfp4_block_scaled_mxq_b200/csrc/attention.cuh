@@ -174,8 +174,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(s_free, kAttnSoftWarps);  // one arrival per softmax warp
     mbar_init(p_full, kAttnSoftWarps);
     mbar_init(o_done, 1);
-    mbar_init(&rbar[0], 32 * kAttnSoftWarps);
-    mbar_init(&rbar[1], 32 * kAttnSoftWarps);
+    mbar_init(&rbar[0], kAttnSoftWarps);  // one arrival per softmax warp
+    mbar_init(&rbar[1], kAttnSoftWarps);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -336,7 +336,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float m = fmaxf(bmax[0], bmax[1]);
       float* slot = sRmax + (j & 1) * 512;
       slot[qt * 128 + r] = m;
-      mbar_arrive(&rbar[j & 1]);
+      __syncwarp();  // the warp's 32 slots are written before its one (release) arrival
+      if (lane == 0) mbar_arrive(&rbar[j & 1]);
       if (!__all_sync(0xffffffffu, mbar_wait(&rbar[j & 1], (j >> 1) & 1))) { ok = false; break; }
       m = fmaxf(fmaxf(slot[r], slot[128 + r]), fmaxf(slot[256 + r], slot[384 + r]));  // finite: key j*256
       const int cand = static_cast<int>(ceilf(m));
