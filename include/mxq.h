@@ -26,6 +26,13 @@
  *     state (it reads its own static device status word, see mxq_debug_poll).
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and never synchronises it.  Calls are thread-safe.
+ *   - Stream order holds as for any kernel, with one refinement: the GEMM kernels
+ *     (mxq_gemm_*, mxq_linear_*) are launched with programmatic stream
+ *     serialisation.  If the kernel before them in the stream lets dependents start
+ *     early (the activation quantisers of this library do), a GEMM may begin its
+ *     set-up and prefetch its weight tiles into L2 while that kernel runs; it reads
+ *     no operand and writes no output before the earlier kernel has completed and
+ *     its writes are visible.  After any other kernel, or a copy, it starts as usual.
  *   - Arguments are validated on the host before anything is launched; on any
  *     error nothing is launched and a status other than MXQ_OK is returned.  A
  *     launch failure returns MXQ_ERR_CUDA.  No C++ exception crosses this ABI.
