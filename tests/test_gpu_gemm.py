@@ -244,3 +244,36 @@ def test_full_output_against_fp32_matmul_of_expanded_operands(which):
         torch.backends.cuda.matmul.allow_tf32 = prev
     err = ((d.float() - ref).abs().max() / ref.abs().max()).item()
     assert err <= GEMM_TOL, err
+
+
+@pytest.mark.parametrize("M", [64, 300])
+def test_back_to_back_reuse_of_the_activation_buffers(M):
+    """Quantise -> GEMM six times in a row on one stream, every time into the same code,
+    scale and output buffers, with no synchronisation in between: the GEMM starts early
+    (programmatic dependent launch after the quantiser) but must read each step's codes,
+    never the previous step's.  Every step's D (copied out in stream order) against an
+    FP32 matmul of that step's operands expanded by the (oracle-exact) dequantiser."""
+    K, N = 512, 1000
+    w = inputs.normal_bf16(N, K, 0.02, seed=91).cuda()
+    wc, wsf = mxq.pack_weight(w)
+    xs = [inputs.heavy_tailed_bf16(M, K, seed=100 + i).cuda() for i in range(6)]
+    q = torch.empty(M, K // 2, dtype=torch.uint8, device="cuda")
+    sf = torch.empty(mxq.mxq_sf_bytes(M, K), dtype=torch.uint8, device="cuda")
+    d = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    outs = []
+    for x in xs:
+        mxq.quantize_act(x, out=(q, sf))
+        mxq.gemm_w4a4(q, sf, wc, wsf, M, N, K, out=d)
+        outs.append(d.clone())
+    torch.cuda.synchronize()
+    wdeq = mxq.dequant_mxfp4(wc, wsf, K).float()
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        for x, got in zip(xs, outs):
+            qx, sx = mxq.quantize_act(x)
+            ref = mxq.dequant_mxfp4(qx, sx, K).float() @ wdeq.T
+            err = ((got.float() - ref).abs().max() / ref.abs().max()).item()
+            assert err <= GEMM_TOL, err
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
