@@ -226,6 +226,15 @@ def gemm_bytes(M, N, K, a_bytes_per_elt=17 / 32):
     return M * K * a_bytes_per_elt + N * K * 17 / 32 + 2.0 * M * N
 
 
+def weight_copies(workload, working_set, w_bytes, l2):
+    """How many copies of the weights the timed loop rotates over: 1 (no rotation) unless
+    the M sweep's working set fits in 4x L2, then at least 4 and at least 2x L2 in total, so
+    that every step streams its weights from HBM."""
+    if workload != "m_sweep" or working_set >= 4 * l2 or w_bytes <= 0:
+        return 1
+    return max(4, -(-2 * l2 // w_bytes))
+
+
 def quant_bytes(M, K, fp8=False):
     """Algorithmic bytes of one activation-quantiser launch: BF16 in, codes (+ scales) out."""
     return M * K * 2 + (M * K if fp8 else M * K // 2 + M * K // 32)
@@ -454,9 +463,7 @@ def main():
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     w_bytes = W_BYTES.get(args.workload, 0)
     working_set = sum(t.numel() * t.element_size() for t in x_in + d_out) + w_bytes
-    copies = 1
-    if args.workload == "m_sweep" and working_set < 4 * l2:
-        copies = max(4, -(-2 * l2 // w_bytes))
+    copies = weight_copies(args.workload, working_set, w_bytes, l2)
     part_sets = [parts] + [build_workload(args.workload, dev, M, rank_seed(rank) + 7919 * i, rule, args.smooth)[1]
                            for i in range(1, copies)]
     flush = working_set < 4 * l2 and copies == 1

@@ -48,3 +48,20 @@ def test_whole_job_rate_counts_every_rank():
     two = bench.whole_job_rate(9.27e12, 10, 2, 20.0)
     assert two == pytest.approx(2 * one)
     assert one == pytest.approx(9.27e12 * 10 / 0.02 / 1e12)
+
+
+def test_algorithmic_bytes_of_a_gemm_and_a_quantiser():
+    """MXFP4 operands: half a byte per element plus one scale byte per 32; D in BF16."""
+    M, N, K = 32760, 13824, 5120
+    assert bench.gemm_bytes(M, N, K) == pytest.approx(M * K * 0.53125 + N * K * 0.53125 + 2 * M * N)
+    assert bench.gemm_bytes(M, N, K, 1.0) == pytest.approx(M * K + N * K * 0.53125 + 2 * M * N)  # FP8 A
+    assert bench.gemm_bytes(M, N, K) / 1e6 == pytest.approx(1032.0, abs=0.5)  # Wan FFN up: A + B + D
+
+
+def test_weight_rotation_for_small_working_sets():
+    l2 = 126 << 20
+    w = 13824 * 5120 * 17 // 32  # 37.6 MB of packed weights
+    assert bench.weight_copies("m_sweep", 50 << 20, w, l2) == 8  # >= 2 x L2 in total
+    assert bench.weight_copies("m_sweep", 50 << 20, 200 << 20, l2) == 4  # at least 4
+    assert bench.weight_copies("m_sweep", 5 * l2, w, l2) == 1  # working set beyond 4 x L2
+    assert bench.weight_copies("flux_w4a8", 50 << 20, w, l2) == 1  # other workloads flush instead
