@@ -371,6 +371,17 @@ MXQ_API mxq_status mxq_attention_mxfp4(const void* q_codes, const void* q_sf, co
  */
 MXQ_API mxq_status mxq_debug_poll(void);
 
+/*
+ * mxq_selftest_wait_timeout -- diagnostic of the failure path above: launches on `stream`
+ * a one-thread kernel that waits, with the same bounded wait as every kernel of the
+ * library, on a barrier nothing arrives on.  After about a second the wait gives up and
+ * records MXQ_ERR_TIMEOUT, and the kernel returns: the next mxq_debug_poll returns
+ * MXQ_ERR_TIMEOUT (and clears it), and the device stays usable.  While the status word
+ * is set, waits in other kernels of the library give up at once, so nothing else should
+ * run between this call and that poll.  Returns MXQ_ERR_UNSUPPORTED off B200.
+ */
+MXQ_API mxq_status mxq_selftest_wait_timeout(mxq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

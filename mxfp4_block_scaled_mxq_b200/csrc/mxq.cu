@@ -684,6 +684,14 @@ mxq_status mxq_linear_w4a4_static(const void* x_bf16, int64_t M, int64_t K, int6
                          d_bf16, ldd, stream);
 }
 
+mxq_status mxq_selftest_wait_timeout(mxq_stream_t stream) {
+  DeviceInfo dev;
+  const mxq_status st = current_device(&dev);
+  if (st != MXQ_OK) return st;
+  mxq::selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return launch_status();
+}
+
 mxq_status mxq_debug_poll(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return MXQ_ERR_CUDA;
   unsigned int v = 0;

@@ -92,6 +92,17 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   return true;
 }
 
+// Diagnostic: one thread waits, through mbar_wait, on an mbarrier that nothing arrives
+// on, so the wait gives up after kWaitLimitCycles and records the timeout -- the failure
+// path that every wait of the library's kernels takes -- and the kernel returns.
+__global__ void selftest_wait_timeout_kernel() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  mbar_wait(&bar, 0);  // phase 0 never completes
+}
+
 // ----------------------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

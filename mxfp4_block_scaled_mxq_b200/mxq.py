@@ -28,7 +28,7 @@ EXPORTED = ("mxq_status_string", "mxq_sf_bytes", "mxq_quantize_act", "mxq_pack_w
             "mxq_gemm_w4a8", "mxq_dequant_mxfp4", "mxq_qdq_act", "mxq_channel_absmax", "mxq_smooth_factors",
             "mxq_quantize_smooth", "mxq_sqnr_accumulate", "mxq_sqnr_db", "mxq_select_precision", "mxq_attn_padded_keys", "mxq_quantize_vt",
             "mxq_attention_mxfp4", "mxq_linear_workspace_bytes", "mxq_linear_w4a4", "mxq_linear_w4a4_static",
-            "mxq_debug_poll")
+            "mxq_debug_poll", "mxq_selftest_wait_timeout")
 
 
 class MxqError(RuntimeError):
@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
     L.mxq_linear_w4a4_static.restype = I32
     L.mxq_debug_poll.argtypes = []
     L.mxq_debug_poll.restype = I32
+    L.mxq_selftest_wait_timeout.argtypes = [P]
+    L.mxq_selftest_wait_timeout.restype = I32
     _lib = L
     return L
 
@@ -224,6 +226,10 @@ def mxq_linear_w4a4_static(x, M, K, ldx, rule, w_codes, w_sf, N, alpha, bias, d,
 
 def mxq_debug_poll() -> int:
     return int(lib().mxq_debug_poll())
+
+
+def mxq_selftest_wait_timeout(stream=None) -> None:
+    _check(lib().mxq_selftest_wait_timeout(_stream(stream)), "mxq_selftest_wait_timeout")
 
 
 # ------------------------------------------------------------------ allocating helpers

@@ -209,3 +209,9 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         mxq.quantize_act(torch.zeros(4, 32, dtype=torch.bfloat16))
+
+
+def test_selftest_without_a_b200_launches_nothing(L):
+    """Off a B200 (here: no GPU at all) the diagnostic launches nothing and reports why."""
+    UNSUPPORTED, CUDA = 4, 5
+    assert L.mxq_selftest_wait_timeout(None) in (UNSUPPORTED, CUDA)
