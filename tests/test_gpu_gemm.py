@@ -277,3 +277,32 @@ def test_back_to_back_reuse_of_the_activation_buffers(M):
             assert err <= GEMM_TOL, err
     finally:
         torch.backends.cuda.matmul.allow_tf32 = prev
+
+
+def _random_shapes(seed, n):
+    """Seeded shapes across both GEMM kernels: M in [1, 700] (few-token kernel up to 128,
+    CTA pairs above), N a multiple of 8 in [8, 1400] (ragged 192-row weight tiles, odd
+    tiles starting mid scale atom), K a multiple of 128 in [128, 1536] (half last stages)."""
+    g = np.random.default_rng(seed)
+    return [(int(g.integers(1, 701)), 8 * int(g.integers(1, 176)), 128 * int(g.integers(1, 13))) for _ in range(n)]
+
+
+@pytest.mark.parametrize("M,N,K", _random_shapes(2024, 10))
+def test_random_shapes_w4a4(M, N, K):
+    x = inputs.heavy_tailed_bf16(M, K, seed=M + 3 * N + 7 * K)
+    w = inputs.normal_bf16(N, K, 0.02, seed=N + 11)
+    bias = (torch.randn(N, generator=torch.Generator().manual_seed(K)) * 0.1).to(torch.bfloat16)
+    check_w4a4(x, w, bias=bias, alpha=0.75)
+
+
+@pytest.mark.parametrize("M,N,K", _random_shapes(77, 6))
+def test_random_shapes_w4a8(M, N, K):
+    x = inputs.normal_bf16(M, K, 1.0, seed=M + N)
+    x_cal = inputs.normal_bf16(M, K, 1.0, seed=M + N + 1)
+    w = inputs.normal_bf16(N, K, 0.02, seed=K + 5)
+    s = inputs.static_fp8_scale(x_cal)
+    wc, wsf = mxq.pack_weight(w.cuda())
+    d = mxq.linear_w4a8(x.cuda(), s, wc, wsf, N)
+    torch.cuda.synchronize()
+    rows = np.arange(M)
+    assert gemm_rel_err(d, rows, oracle_w4a8(x, w, s, rows)) <= GEMM_TOL
