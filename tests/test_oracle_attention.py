@@ -118,3 +118,36 @@ def test_uos_beats_ocp(scale):
     (o, _), _, (o_ref, _) = _three_modes(scale, oracle.RULE_OCP)
     err = lambda a, r: np.linalg.norm(a - r) / np.linalg.norm(r)
     assert err(u, u_ref) < err(o, o_ref), (err(u, u_ref), err(o, o_ref))
+
+
+def _deq(x, rule):
+    """MXFP4 round trip of the rows of x (blocks along the rows), FP64."""
+    codes, sl = oracle.quantize_mxfp4(x.contiguous(), rule=rule)
+    rows, K = x.shape
+    return oracle.dequant_mxfp4(codes, oracle.sf_swizzle(sl, rows, K), rows, K)
+
+
+@pytest.mark.parametrize("rule", [oracle.RULE_UOS, oracle.RULE_OCP])
+def test_unquantised_mode_is_the_textbook_softmax_of_the_quantised_operands(rule):
+    """With P left unquantised, the oracle is softmax(Q K^T / sqrt(d)) V over the
+    dequantised MXFP4 Q and K (blocks along the head dimension) and V (blocks along the
+    keys), head by head -- written here independently in FP64 NumPy.  The oracle takes
+    the exponent in base 2 from FP32 scores, so the two agree to FP32 rounding; a wrong
+    scale, a transposed product or a head mix-up would not."""
+    H, d, Sq, Skv = 2, 64, 5, 70
+    q = inputs.normal_bf16(Sq, H * d, 1.5, seed=41)
+    k = inputs.normal_bf16(Skv, H * d, 1.5, seed=42)
+    v = inputs.heavy_tailed_bf16(Skv, H * d, seed=43)
+    got, ws = oracle.attention_mxfp4(q, k, v, H, d, rule=rule, mode=oracle.ATTN_UNQUANTISED_P)
+    Q, K = _deq(q, rule), _deq(k, rule)
+    Skv_pad = (Skv + 31) // 32 * 32
+    vt = torch.zeros(H * d, Skv_pad, dtype=torch.bfloat16)
+    vt[:, :Skv] = v.t()
+    V = _deq(vt, rule)[:, :Skv].T  # [Skv][H*d]
+    for h in range(H):
+        cols = slice(h * d, (h + 1) * d)
+        s = Q[:, cols] @ K[:, cols].T / math.sqrt(d)
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        want = (p / p.sum(axis=1, keepdims=True)) @ V[:, cols]
+        np.testing.assert_allclose(got[:, h, :], want, rtol=2e-5, atol=2e-5 * np.abs(want).max())
+    np.testing.assert_allclose(ws, 1.0, rtol=1e-12)
