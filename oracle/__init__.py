@@ -21,6 +21,17 @@ Parity status per function (what pins each one is in ``tests/test_oracle_*.py``)
                               identities, error-quadrature property
   bf16_rne / qdq_* /          pinned: torch's FP32->BF16 conversion, tie cases,
   dequant_mxfp4_bf16          recomposition from the pinned codecs
+  quantize_mxfp4_smooth       pinned: unit multiplier = plain quantiser, powers of two
+                              shift only the scale, a worked rotation-then-multiplier case
+  channel_absmax /            pinned: column maxima of the (rotated) rows; closed forms of
+  smooth_factors              the migration factors at alpha = 0.5, 1 and 0
+  sqnr_sums / sqnr_db /       pinned: closed forms (uniform relative error, known pairs,
+  select_precision            limits) and every tier boundary
+  pnq_exp2                    pinned: Taylor remainder bound, exact at integers, exact
+                              power-of-two offsets, the flush below 2^-126
+  attention_mxfp4             pinned: the textbook FP64 softmax of the dequantised
+                              operands (P unquantised), equal-score and dominant-key
+                              closed forms, PNQ weights summing to one
 """
 
 from __future__ import annotations
