@@ -317,6 +317,13 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
   const float c = __uint_as_float(kInvSqrt128Bits);
   const float2 cc = make_float2(c, c);
   const float2 minus1 = make_float2(-1.f, -1.f);
+  // kOutAbsmax: this lane's 32 column maxima over its rows of both passes; column k of
+  // block j is cm[k] (k < 16: element k, else element k of the pairs' upper halves)
+  float cm[kOut == kOutAbsmax ? 32 : 1];
+  if constexpr (kOut == kOutAbsmax) {
+#pragma unroll
+    for (int q = 0; q < 32; ++q) cm[q] = 0.f;
+  }
   // both passes' rows are loaded before either is computed: the second pass's loads are
   // in flight during the first pass's arithmetic
   uint32_t w[2][2][8];
@@ -379,21 +386,10 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
       if constexpr (kSmooth) P[i] = __fmul2_rn(P[i], make_float2(s_chan[32 * j + i], s_chan[32 * j + 16 + i]));
     }
     if constexpr (kOut == kOutAbsmax) {
-      // column maxima over the 8 rows of this warp with the same j (lanes xor 4, 8, 16),
-      // then over the warps and passes in shared memory
-      uint32_t* cmax = reinterpret_cast<uint32_t*>(atom);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        float a = fabsf(P[i].x), b = fabsf(P[i].y);
-#pragma unroll
-        for (int sh = 4; sh < 32; sh *= 2) {
-          a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, sh));
-          b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, sh));
-        }
-        if (lane < 4) {
-          atomicMax(cmax + 32 * j + i, __float_as_uint(a));
-          atomicMax(cmax + 32 * j + 16 + i, __float_as_uint(b));
-        }
+        cm[i] = fmaxf(cm[i], fabsf(P[i].x));
+        cm[16 + i] = fmaxf(cm[16 + i], fabsf(P[i].y));
       }
       continue;
     }
@@ -432,6 +428,33 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
     }
   }
   if (kQdq) return;  // uniform: no scale atom to write
+  if constexpr (kOut == kOutAbsmax) {
+    // Column maxima over the 8 rows of this warp that share block j (lanes xor 4, 8, 16)
+    // by reduce-scatter: each round keeps half of the columns and takes the partner's
+    // maxima of them (28 shuffles instead of 96), leaving every lane 4 finished columns;
+    // then over the warps in shared memory.
+    const int b4 = (lane >> 4) & 1, b3 = (lane >> 3) & 1, b2 = (lane >> 2) & 1;
+    float c16[16], c8[8], c4[4];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const float send = b4 ? cm[q] : cm[16 + q];
+      c16[q] = fmaxf(b4 ? cm[16 + q] : cm[q], __shfl_xor_sync(0xffffffffu, send, 16));
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float send = b3 ? c16[q] : c16[8 + q];
+      c8[q] = fmaxf(b3 ? c16[8 + q] : c16[q], __shfl_xor_sync(0xffffffffu, send, 8));
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float send = b2 ? c8[q] : c8[4 + q];
+      c4[q] = fmaxf(b2 ? c8[4 + q] : c8[q], __shfl_xor_sync(0xffffffffu, send, 4));
+    }
+    uint32_t* cmax = reinterpret_cast<uint32_t*>(atom);
+    const int col = 32 * j + 16 * b4 + 8 * b3 + 4 * b2;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) atomicMax(cmax + col + q, __float_as_uint(c4[q]));
+  }
   __syncthreads();
   if constexpr (kOut == kOutAbsmax) {
     if (tid < 128)
