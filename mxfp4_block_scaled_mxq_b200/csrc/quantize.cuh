@@ -514,6 +514,7 @@ template <bool kHadamard, bool kUOS>
 __global__ void __launch_bounds__(kQuantThreads) quantize_smooth_mxfp4_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ld, const float* __restrict__ chan,
     uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  griddep_launch_dependents();  // a GEMM launched after this may run its prologue now
   TileArgs o;
   o.codes = codes;
   o.sf = sf;
