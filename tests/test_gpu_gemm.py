@@ -306,3 +306,24 @@ def test_random_shapes_w4a8(M, N, K):
     torch.cuda.synchronize()
     rows = np.arange(M)
     assert gemm_rel_err(d, rows, oracle_w4a8(x, w, s, rows)) <= GEMM_TOL
+
+
+@pytest.mark.parametrize("M,N,K", [(40, 1000, 256), (300, 1000, 256), (300, 200, 384)])
+def test_writes_stay_inside_d(M, N, K):
+    """D with a padded row stride (ldd = N + 72) inside a larger buffer filled with a
+    sentinel: the padding columns of every row and the rows past M keep the sentinel, and
+    the M x N block matches the oracle (few-token and CTA-pair kernels, ragged N)."""
+    x = inputs.heavy_tailed_bf16(M, K, seed=M + 5)
+    w = inputs.normal_bf16(N, K, 0.02, seed=N + 5)
+    ldd = N + 72
+    sentinel = -12288.0  # exact in BF16
+    buf = torch.full((M + 3, ldd), sentinel, dtype=torch.bfloat16, device="cuda")
+    wc, wsf = mxq.pack_weight(w.cuda())
+    q, sf = mxq.quantize_act(x.cuda())
+    mxq.gemm_w4a4(q, sf, wc, wsf, M, N, K, out=buf[:M, :N])
+    torch.cuda.synchronize()
+    host = buf.float().cpu()
+    assert (host[:M, N:] == sentinel).all()
+    assert (host[M:, :] == sentinel).all()
+    rows = np.arange(M)
+    assert gemm_rel_err(buf[:M, :N], rows, oracle_w4a4(x, w, rows)) <= GEMM_TOL
