@@ -104,3 +104,23 @@ def test_full_size_wan_self_attention_sampled():
         got = o[:, cols].float().cpu().numpy()[rows]
         err = np.abs(got - want[:, 0, :]).max() / np.abs(want).max()
         assert err <= ATTN_TOL, (h, err)
+
+
+def test_attention_writes_stay_inside_o():
+    """O with a padded row stride (ldo = H*d + 64) inside a larger buffer filled with a
+    sentinel: the padding columns and the rows past Sq keep it; O itself matches."""
+    Sq, Skv, H = 130, 300, 2
+    q = inputs.normal_bf16(Sq, H * D, 1.0, seed=51)
+    k = inputs.normal_bf16(Skv, H * D, 1.0, seed=52)
+    v = inputs.normal_bf16(Skv, H * D, 1.0, seed=53)
+    sentinel = -12288.0  # exact in BF16
+    buf = torch.full((Sq + 3, H * D + 64), sentinel, dtype=torch.bfloat16, device="cuda")
+    mxq.attention_mxfp4(q.cuda(), k.cuda(), v.cuda(), H, out=buf[:Sq, :H * D])
+    torch.cuda.synchronize()
+    host = buf.float().cpu()
+    assert (host[:Sq, H * D:] == sentinel).all()
+    assert (host[Sq:, :] == sentinel).all()
+    rows = np.arange(Sq)
+    want, _ = oracle.attention_mxfp4(q, k, v, H, D, rows)
+    got = host[:Sq, :H * D].numpy().reshape(Sq, H, D)
+    assert np.abs(got - want).max() / np.abs(want).max() <= ATTN_TOL
