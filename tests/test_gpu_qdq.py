@@ -124,3 +124,37 @@ def test_full_size_qdq_wan_ffn_activations():
     rows = sample_rows(x.shape[0], 96)
     idx = torch.as_tensor(rows, device="cuda")
     np.testing.assert_array_equal(_bits(got[idx]), oracle.qdq_mxfp4(x[idx].cpu()))
+
+
+@pytest.mark.parametrize("fmt,hadamard", [(mxq.MXQ_ACT_MXFP4, False), (mxq.MXQ_ACT_MXFP4, True),
+                                          (mxq.MXQ_ACT_FP8_E4M3, False)])
+def test_outputs_stay_inside_their_rows(fmt, hadamard):
+    """QDQ (and, for plain MXFP4, the expansion) into buffers with a padded row stride
+    (+64 columns) and 3 rows more than written, filled with a sentinel: only the
+    [rows][K] block changes, and it equals the oracle's bits (ragged rows: 130)."""
+    rows, K, s = 130, 384, 0.05
+    x = inputs.heavy_tailed_bf16(rows, K, seed=61)
+    sentinel = -12288.0  # exact in BF16
+
+    def padded():
+        return torch.full((rows + 3, K + 64), sentinel, dtype=torch.bfloat16, device="cuda")
+
+    def check(buf, want_bits):
+        host = buf.float().cpu()
+        assert (host[:rows, K:] == sentinel).all() and (host[rows:, :] == sentinel).all()
+        np.testing.assert_array_equal(_bits(buf[:rows, :K]), want_bits)
+
+    buf = padded()
+    mxq.qdq_act(x.cuda(), fmt, mxq.MXQ_SCALE_OCP, hadamard, act_scale=s, out=buf[:rows, :K])
+    torch.cuda.synchronize()
+    if fmt == mxq.MXQ_ACT_FP8_E4M3:
+        check(buf, oracle.qdq_fp8(x, s))
+        return
+    check(buf, oracle.qdq_mxfp4(x, hadamard=hadamard))
+    if not hadamard:
+        codes, sl = oracle.quantize_mxfp4(x)
+        sf = oracle.sf_swizzle(sl, rows, K)
+        buf2 = padded()
+        mxq.dequant_mxfp4(torch.from_numpy(codes).cuda(), torch.from_numpy(sf).cuda(), K, out=buf2[:rows, :K])
+        torch.cuda.synchronize()
+        check(buf2, oracle.dequant_mxfp4_bf16(codes, sf, rows, K))
