@@ -122,6 +122,59 @@ __device__ __forceinline__ float2 pnq_exp2_pair(float2 t, float lo, uint32_t bia
   return __fmul2_rn(p, sc);
 }
 
+// E2M1 codes of one 32-key block: numerators 2^(t - c) (raised to c - 127 first, so
+// keys past the end and underflowing keys give 0) times the block's 2^-e, rounded to
+// nearest even with saturation.  The general form.
+__device__ __forceinline__ void pnq_block_codes(const float* t, float lo, uint32_t bias_bits, float s1,
+                                                const AttnParams& prm, uint32_t* codes) {
+  const float2 sc = make_float2(s1, s1);
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    float2 v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      v[q] = __fmul2_rn(pnq_exp2_pair<true>(make_float2(t[8 * w + 2 * q], t[8 * w + 2 * q + 1]), lo, bias_bits, prm),
+                        sc);
+    codes[w] = e2m1x8(v[0].x, v[0].y, v[1].x, v[1].y, v[2].x, v[2].y, v[3].x, v[3].y);
+  }
+}
+
+// The same codes, two multiplies fewer per pair of keys, for a block in which every key has
+// rint(t) - c >= -126 and rint(t) - c - e >= -125, with |ce| <= 100 (ce = c + e).  The
+// factor 2^-(c + e) rides on the polynomial's coefficients: a power of two, so every Horner
+// step rounds as it would unscaled and p'(g) = p(g) 2^-(c + e) exactly.  2^n then enters
+// by an integer add to the exponent field (bits(r) * 2^23 = n * 2^23 modulo 2^32, as in
+// pnq_exp2_pair), which stays within [1, 254]: the value is p(g) 2^(n - c) 2^-e, the one the
+// general form rounds to E2M1.
+__device__ __forceinline__ void pnq_block_codes_folded(const float* t, int ce, const AttnParams& prm,
+                                                       uint32_t* codes) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const float f = __uint_as_float(static_cast<uint32_t>(127 - ce) << 23);
+  float2 a[kExp2Terms];
+#pragma unroll
+  for (int k = 0; k < kExp2Terms; ++k) {
+    const float ak = __fmul_rn(prm.exp2c[k], f);
+    a[k] = make_float2(ak, ak);
+  }
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    float v[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 x = make_float2(t[8 * w + 2 * q], t[8 * w + 2 * q + 1]);
+      const float2 r = __fadd2_rn(x, make_float2(kMagic, kMagic));
+      const float2 n = __fadd2_rn(r, make_float2(-kMagic, -kMagic));
+      const float2 g = __fadd2_rn(x, make_float2(-n.x, -n.y));
+      float2 p = a[kExp2Terms - 1];
+#pragma unroll
+      for (int k = kExp2Terms - 2; k >= 0; --k) p = __ffma2_rn(p, g, a[k]);
+      v[2 * q] = __uint_as_float(__float_as_uint(p.x) + __float_as_uint(r.x) * 8388608u);
+      v[2 * q + 1] = __uint_as_float(__float_as_uint(p.y) + __float_as_uint(r.y) * 8388608u);
+    }
+    codes[w] = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+  }
+}
+
 template <bool kUOS>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     mx_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_sfq,
@@ -333,59 +386,63 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         bmax[b] = fmaxf(mb, t[32 * b + 31]);
         bmin[b] = fminf(nb, t[32 * b + 31]);
       }
-      float m = fmaxf(bmax[0], bmax[1]);
+      // Publish this thread's maximum; the row's offset is settled after the codes.
+      const float m_own = fmaxf(bmax[0], bmax[1]);
       float* slot = sRmax + (j & 1) * 512;
-      slot[qt * 128 + r] = m;
+      slot[qt * 128 + r] = m_own;
       __syncwarp();  // the warp's 32 slots are written before its one (release) arrival
       if (lane == 0) mbar_arrive(&rbar[j & 1]);
+      // Provisional offset cp: the lazy rule applied to this thread's own keys.  The row's
+      // offset chat (settled below) is never below it, and the E8M0 block scaling is
+      // equivariant under the power of two 2^(cp - chat): the codes computed against cp
+      // are the row's codes, and only the scale bytes move by cp - chat.
+      int cp = chat;
+      if (m_own > -INFINITY) {
+        const int own = static_cast<int>(ceilf(m_own));
+        if (j == 0 || own > chat + 8) cp = own;
+      } else if (j == 0) {
+        cp = 0;  // every key of this thread is past the end: codes 0 whatever the offset
+      }
+      uint32_t codes[8];
+      int eb[2];
+      {
+        const float lo = static_cast<float>(cp - 127);
+        const uint32_t bias_bits = static_cast<uint32_t>(127 - cp) << 23;
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          // the block exponent from the numerator of the block's largest score (0 if none)
+          const float amax = pnq_exp2_pair(make_float2(bmax[b], bmax[b]), lo, bias_bits, prm).x;
+          const int e = block_exponent<kUOS>(__float_as_uint(amax));
+          eb[b] = e;
+          const int ce = cp + e;
+          if (ce >= -100 && ce <= 100 && bmin[b] >= static_cast<float>(max(cp - 126, ce - 125))) {
+            pnq_block_codes_folded(t + 32 * b, ce, prm, codes + 4 * b);  // the usual case
+          } else {
+            pnq_block_codes(t + 32 * b, lo, bias_bits, exp2_neg(e), prm, codes + 4 * b);
+          }
+        }
+      }
+      // The row's offset: the maximum over its four threads, raised lazily.
       if (!__all_sync(0xffffffffu, mbar_wait(&rbar[j & 1], (j >> 1) & 1))) { ok = false; break; }
-      m = fmaxf(fmaxf(slot[r], slot[128 + r]), fmaxf(slot[256 + r], slot[384 + r]));  // finite: key j*256
+      const float m = fmaxf(fmaxf(slot[r], slot[128 + r]), fmaxf(slot[256 + r], slot[384 + r]));  // key j*256: finite
       const int cand = static_cast<int>(ceilf(m));
       float rescale = 1.f;
       if (j == 0) {
         chat = cand;
       } else if (cand > chat + 8) {
-        rescale = __int_as_float((127 + chat - cand) << 23);  // 2^(chat - cand), exact
+        // 2^(chat - cand), exact; 0 once it is below the normal range
+        rescale = cand - chat > 126 ? 0.f : __int_as_float((127 + chat - cand) << 23);
         chat = cand;
       }
-      // numerators -> MXFP4 (2 blocks of 32 keys), kept as codes and scale bytes
-      const float lo = static_cast<float>(chat - 127);
-      const uint32_t bias_bits = static_cast<uint32_t>(127 - chat) << 23;
-      uint32_t codes[8];
       uint32_t sf_half = 0;
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
-        // the block exponent from the numerator of the block's largest score (0 if none)
-        const float amax = pnq_exp2_pair(make_float2(bmax[b], bmax[b]), lo, bias_bits, prm).x;
-        if (bmin[b] >= lo) {  // no key of the block below chat - 127 (the usual case)
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {  // in place: t becomes the numerators
-            const float2 p =
-                pnq_exp2_pair<false>(make_float2(t[32 * b + 2 * u], t[32 * b + 2 * u + 1]), lo, bias_bits, prm);
-            t[32 * b + 2 * u] = p.x;
-            t[32 * b + 2 * u + 1] = p.y;
-          }
-        } else {
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const float2 p =
-                pnq_exp2_pair<true>(make_float2(t[32 * b + 2 * u], t[32 * b + 2 * u + 1]), lo, bias_bits, prm);
-            t[32 * b + 2 * u] = p.x;
-            t[32 * b + 2 * u + 1] = p.y;
-          }
+        int e = eb[b] + cp - chat;
+        if (e < -127) {  // below the E8M0 range relative to the row: numerators < 2^-120 of it
+          codes[4 * b] = codes[4 * b + 1] = codes[4 * b + 2] = codes[4 * b + 3] = 0u;
+          e = -127;
         }
-        const int e = block_exponent<kUOS>(__float_as_uint(amax));
-        const float s1 = exp2_neg(e);
-        const float2 sc = make_float2(s1, s1);
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          float2 v[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            v[q] = __fmul2_rn(make_float2(t[32 * b + 8 * w + 2 * q], t[32 * b + 8 * w + 2 * q + 1]), sc);
-          codes[4 * b + w] = e2m1x8(v[0].x, v[0].y, v[1].x, v[1].y, v[2].x, v[2].y, v[3].x, v[3].y);
-        }
-        sf_half |= static_cast<uint32_t>(e + 127) << (8 * b);
+        sf_half |= static_cast<uint32_t>(min(e, 127) + 127) << (8 * b);
       }
       // the previous tile's P V must be done before P is overwritten or O rescaled
       if (j > 0) {
