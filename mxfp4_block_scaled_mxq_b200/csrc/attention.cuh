@@ -8,7 +8,7 @@
 //
 // with Q, K in 32-blocks along the head dimension, V and P in 32-blocks along the keys,
 // c an integer offset (a power-of-two factor, under which the E8M0 block scaling is
-// exactly equivariant: the codes of P do not depend on it) and 2^(t - c) the degree-4
+// exactly equivariant: the codes of P do not depend on it) and 2^(t - c) the degree-3
 // Taylor polynomial of 2^g, g = t - rint(t), times 2^(rint(t) - c) (0 when rint(t) - c <
 // -126); a block's E8M0 exponent comes from the numerator of its largest score.  The row sum is taken over the quantised numerators
 // (PNQ), so the implied weights sum to one by construction; it is computed by the
@@ -75,7 +75,7 @@ __host__ __device__ constexpr uint32_t attn_idesc(int n) {
          (static_cast<uint32_t>(kAttnBM >> 4) << 24);
 }
 
-constexpr int kExp2Terms = 5;  // degree-4 Taylor polynomial of 2^g (relative error < 6e-5)
+constexpr int kExp2Terms = 4;  // degree-3 Taylor polynomial of 2^g (relative error < 8.6e-4)
 
 struct AttnParams {
   float exp2c[kExp2Terms];  // Taylor coefficients a_k = (ln 2)^k / k! of 2^g, FP32
@@ -408,12 +408,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       {
         const float lo = static_cast<float>(cp - 127);
         const uint32_t bias_bits = static_cast<uint32_t>(127 - cp) << 23;
+        // the block exponents from the numerators of the blocks' largest scores (0 if none)
+        const float2 amax = pnq_exp2_pair(make_float2(bmax[0], bmax[1]), lo, bias_bits, prm);
+        eb[0] = block_exponent<kUOS>(__float_as_uint(amax.x));
+        eb[1] = block_exponent<kUOS>(__float_as_uint(amax.y));
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
-          // the block exponent from the numerator of the block's largest score (0 if none)
-          const float amax = pnq_exp2_pair(make_float2(bmax[b], bmax[b]), lo, bias_bits, prm).x;
-          const int e = block_exponent<kUOS>(__float_as_uint(amax));
-          eb[b] = e;
+          const int e = eb[b];
           const int ce = cp + e;
           if (ce >= -100 && ce <= 100 && bmin[b] >= static_cast<float>(max(cp - 126, ce - 125))) {
             pnq_block_codes_folded(t + 32 * b, ce, prm, codes + 4 * b);  // the usual case

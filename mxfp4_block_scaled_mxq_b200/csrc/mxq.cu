@@ -610,7 +610,7 @@ mxq_status mxq_attention_mxfp4(const void* q_codes, const void* q_sf, const void
   if (!ok) return MXQ_ERR_CUDA;
 
   mxq::AttnParams prm;
-  {  // degree-4 Taylor coefficients of 2^g: a_0 = 1, a_k = a_(k-1) * ln 2 / k
+  {  // degree-3 Taylor coefficients of 2^g: a_0 = 1, a_k = a_(k-1) * ln 2 / k
     double c = 1.0;
     const double ln2 = std::log(2.0);
     for (int k = 0; k < mxq::kExp2Terms; ++k) {

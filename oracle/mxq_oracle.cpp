@@ -69,10 +69,10 @@
 //    c = ceil(max_j t_j) -- a power-of-two offset, under which E8M0 block scaling is
 //    exactly equivariant, so the codes do not depend on it; the exponential is
 //    2^(t - c) = p(g) * 2^(n - c) with n = rint(t) (nearest, ties to even), g = t - n in
-//    [-1/2, 1/2] and p the degree-4 Taylor polynomial of 2^g (coefficients a_0 = 1,
+//    [-1/2, 1/2] and p the degree-3 Taylor polynomial of 2^g (coefficients a_0 = 1,
 //    a_k = a_(k-1) * ln 2 / k in FP64, rounded to FP32; Horner with FP32 fused
-//    multiply-adds; relative error below 6e-5, three orders of magnitude under the E2M1
-//    step), and numerators with n - c < -126 are 0.  A block's E8M0 exponent is taken from
+//    multiply-adds; relative error below 8.6e-4, more than two orders of magnitude under
+//    the E2M1 step), and numerators with n - c < -126 are 0.  A block's E8M0 exponent is taken from
 //    the numerator of its largest score (the exponential is monotone).  These FP32 steps
 //    decide the quantised codes, so they are taken in the kernel's precision; the rest is
 //    FP64.
@@ -466,9 +466,9 @@ void oracle_gemm(int a_kind, const uint8_t* a_codes, const uint8_t* a_sf, int64_
 
 // ---------------------------------------------------------------- MXFP4 attention
 
-constexpr int kExp2Terms = 5;  // degree 4
+constexpr int kExp2Terms = 4;  // degree 3
 
-// Coefficients of the degree-4 Taylor polynomial of 2^g around g = 0.
+// Coefficients of the degree-3 Taylor polynomial of 2^g around g = 0.
 static void pnq_exp2_coefficients(float* a) {
   double c = 1.0;
   const double ln2 = std::log(2.0);

@@ -20,14 +20,16 @@ def _f32(x):
 
 
 def test_pnq_exp2_accuracy():
-    """Within 6e-5 relative of 2^(t - c) over the range softmax numerators use (the
-    degree-4 Taylor remainder of 2^g on |g| <= 1/2: (ln 2 / 2)^5 / 5! * 2^(1/2) = 5.9e-5)."""
+    """Relative error against 2^(t - c) over the range softmax numerators use: below the
+    degree-3 Taylor remainder of 2^g on |g| <= 1/2, (ln 2 / 2)^4 / 4! * 2^(1/2) = 8.50e-4,
+    and above (ln 2 / 2)^4 / 4! = 6.01e-4, which it reaches near g = 1/2 (so a polynomial
+    of another degree fails one side)."""
     ts = np.float32(np.linspace(-40.0, 8.0, 20011))
     worst = 0.0
     for t in ts:
         want = 2.0 ** (float(t) - 3)
         worst = max(worst, abs(oracle.pnq_exp2(float(t), 3) - want) / want)
-    assert worst < 6e-5, worst
+    assert 5.5e-4 < worst < 8.6e-4, worst
 
 
 @pytest.mark.parametrize("t", [-17.37, -0.001, 0.0, 2.5, 7.99])
