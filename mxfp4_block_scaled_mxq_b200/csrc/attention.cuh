@@ -23,7 +23,8 @@
 //               tile, O += P V^T (M 128, N 144: d columns + the ones row, K 256 keys);
 //               the next tile's scores are issued before the previous tile's P V, so
 //               the tensor core works while the softmax warps quantise.
-//   warps 2..17 softmax / PNQ, four threads per query row (64 keys of the tile each):
+//   warps 2, 3  idle (their warpgroup hands its registers to the softmax warps)
+//   warps 4..19 softmax / PNQ, four threads per query row (64 keys of the tile each):
 //               scores from TMEM, the row maximum through shared memory, the
 //               offset c raised only when the maximum passes c + 8 (then O, l are
 //               rescaled in TMEM by the exact power of two), numerators, UOS/OCP block
@@ -44,7 +45,13 @@ constexpr int kAttnD = 128;       // head dimension
 constexpr int kAttnBM = 128;      // queries per CTA
 constexpr int kAttnBN = 256;      // keys per tile
 constexpr int kAttnStages = 3;
-constexpr int kAttnThreads = 576;  // producer, MMA, 16 softmax warps
+constexpr int kAttnThreads = 640;  // producer, MMA, 2 idle warps, 16 softmax warps
+// Registers: launched with 96 a thread (640 x 96 = 61440); the control warpgroup (warps
+// 0-3) then gives up all but 32 and the four softmax warpgroups take 112: 128 x 32 +
+// 512 x 112 = 61440, exactly the launch's total, so the increase always completes.
+constexpr int kAttnCtrlRegs = 32;
+constexpr int kAttnSoftRegs = 112;
+static_assert(128 * kAttnCtrlRegs + 512 * kAttnSoftRegs <= kAttnThreads * 96, "register split");
 constexpr int kAttnSoftWarps = 16;  // four per TMEM lane quadrant: keys [64 q, +64) of a tile each
 constexpr int kAttnNv = kAttnD + 16;  // P V's N: the d value columns and 16 rows holding the ones row
 constexpr uint32_t kAttnTmemCols = 512;
@@ -232,10 +239,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(drain, 1);
     fence_mbar_init();
   }
-  if (warp >= 2) {
+  if (warp >= 4) {
     // Constant parts of the P V operand: the row of ones (row d = 128 of each V^T stage:
     // E2M1 1.0 = code 2 in every nibble; rows 129..143 zero) and their unit scales.
-    const int t = threadIdx.x - 64;  // 0..511
+    const int t = threadIdx.x - 128;  // 0..511
     for (int s = 0; s < kAttnStages; ++s) {
       uint32_t* ones = reinterpret_cast<uint32_t*>(sV(s) + kAttnD * 128);  // 16 rows x 128 B = 512 words
       ones[t] = t < 32 ? 0x22222222u : 0u;
@@ -251,99 +258,108 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    if (elect_one()) {
-      bool ok = true;
-      mbar_arrive_expect_tx(q_full, kAttnQBytes + 512);
-      tma_load_2d(sQ, &tmap_q, head * 64, q_tile * kAttnBM, q_full);
-      tma_load_4d(sSfq, &tmap_sfq, 0, 0, head, q_tile, q_full);
-      int stage = 0;
-      uint32_t phase = 0, issued = 0, issued_phase = 0;
-      const uint32_t tx = kAttnKBytes + kAttnD * 128 + 1024 + 1024;
-      for (int j = 0; j < nt; ++j) {
-        if (!mbar_wait(&kv_empty[stage], phase ^ 1)) { ok = false; break; }
-        issued |= 1u << stage;
-        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-        mbar_arrive_expect_tx(&kv_full[stage], tx);
-        tma_load_2d(sK(stage), &tmap_k, head * 64, j * kAttnBN, &kv_full[stage]);
-        tma_load_4d(sSfk(stage), &tmap_sfk, 0, 0, head, 2 * j, &kv_full[stage]);
-        tma_load_2d(sV(stage), &tmap_v, j * (kAttnBN / 2), head * kAttnD, &kv_full[stage]);
-        tma_load_4d(sSfv(stage), &tmap_sfv, 0, 0, 2 * j, head, &kv_full[stage]);
-        if (++stage == kAttnStages) { stage = 0; phase ^= 1; }
+  if (warp < 4) {
+    setmaxnreg_dec<kAttnCtrlRegs>();  // the whole control warpgroup, one instruction
+    if (warp == 0) {
+      // ------------------------------------------------------------------ TMA producer
+      if (elect_one()) {
+        bool ok = true;
+        mbar_arrive_expect_tx(q_full, kAttnQBytes + 512);
+        tma_load_2d(sQ, &tmap_q, head * 64, q_tile * kAttnBM, q_full);
+        tma_load_4d(sSfq, &tmap_sfq, 0, 0, head, q_tile, q_full);
+        int stage = 0;
+        uint32_t phase = 0, issued = 0, issued_phase = 0;
+        const uint32_t tx = kAttnKBytes + kAttnD * 128 + 1024 + 1024;
+        for (int j = 0; j < nt; ++j) {
+          if (!mbar_wait(&kv_empty[stage], phase ^ 1)) { ok = false; break; }
+          issued |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          mbar_arrive_expect_tx(&kv_full[stage], tx);
+          tma_load_2d(sK(stage), &tmap_k, head * 64, j * kAttnBN, &kv_full[stage]);
+          tma_load_4d(sSfk(stage), &tmap_sfk, 0, 0, head, 2 * j, &kv_full[stage]);
+          tma_load_2d(sV(stage), &tmap_v, j * (kAttnBN / 2), head * kAttnD, &kv_full[stage]);
+          tma_load_4d(sSfv(stage), &tmap_sfv, 0, 0, 2 * j, head, &kv_full[stage]);
+          if (++stage == kAttnStages) { stage = 0; phase ^= 1; }
+        }
+        mbar_wait_drain(q_full, 0);
+        if (!ok) {
+          for (int s = 0; s < kAttnStages; ++s)
+            if (issued & (1u << s)) mbar_wait_drain(&kv_full[s], (issued_phase >> s) & 1u);
+        }
       }
-      mbar_wait_drain(q_full, 0);
-      if (!ok) {
-        for (int s = 0; s < kAttnStages; ++s)
-          if (issued & (1u << s)) mbar_wait_drain(&kv_full[s], (issued_phase >> s) & 1u);
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      if (elect_one()) {
+        bool ok = mbar_wait(q_full, 0);
+        if (ok) {
+          tc_fence_after();
+          tc_cp_sf_atom(tmem + kColSfq, smem_desc(smem_u32(sSfq), 0, 128, 0));
+        }
+        // O += P V^T for key tile i (P from shared memory, written by the softmax warps).
+        auto issue_pv = [&](int i) -> bool {
+          if (!mbar_wait(p_full, i & 1)) return false;
+          tc_fence_after();
+          const int st = i % kAttnStages;
+          const uint32_t par = static_cast<uint32_t>(i & 1);
+          const uint32_t sfp = kColSfp + par * 8, sfv = kColSfv + par * 16;
+  #pragma unroll
+          for (int a = 0; a < 2; ++a) {
+            tc_cp_sf_atom(tmem + sfp + 4 * a, smem_desc(smem_u32(sSfp + a * 512), 0, 128, 0));
+            tc_cp_sf_atom(tmem + sfv + 8 * a, smem_desc(smem_u32(sSfv(st) + a * 512), 0, 128, 0));
+            tc_cp_sf_atom(tmem + sfv + 8 * a + 4, smem_desc(smem_u32(sSfOnes + a * 512), 0, 128, 0));
+          }
+          const uint32_t p_base = smem_u32(sP), v_base = smem_u32(sV(st));
+  #pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // 4 x 64 keys
+            const int a = kk >> 1;
+            const uint32_t sf_id = static_cast<uint32_t>((kk & 1) * 2);
+            const uint32_t idesc = attn_idesc(kAttnNv) | (sf_id << 29) | (sf_id << 4);
+            tc_mma_mxf4(tmem + kColO, smem_desc(p_base + kk * 32, 16, 1024, 2), smem_desc(v_base + kk * 32, 16, 1024, 2),
+                        idesc, tmem + sfp + 4 * a, tmem + sfv + 8 * a, (i | kk) != 0);
+          }
+          tc_commit(o_done);
+          tc_commit(&kv_empty[st]);
+          return true;
+        };
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int j = 0; ok && j < nt; ++j) {
+          if (!mbar_wait(&kv_full[stage], phase)) { ok = false; break; }
+          if (j > 0 && !mbar_wait(s_free, (j - 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sfk = kColSfk + static_cast<uint32_t>(j & 1) * 8;
+          tc_cp_sf_atom(tmem + sfk, smem_desc(smem_u32(sSfk(stage)), 0, 128, 0));
+          tc_cp_sf_atom(tmem + sfk + 4, smem_desc(smem_u32(sSfk(stage) + 512), 0, 128, 0));
+          const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK(stage));
+  #pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {  // 2 x 64 of the head dimension
+            const uint32_t sf_id = static_cast<uint32_t>(kk * 2);
+            const uint32_t idesc = attn_idesc(kAttnBN) | (sf_id << 29) | (sf_id << 4);
+            tc_mma_mxf4(tmem + kColS, smem_desc(q_base + kk * 32, 16, 512, 4), smem_desc(k_base + kk * 32, 16, 512, 4),
+                        idesc, tmem + kColSfq, tmem + sfk, kk != 0);
+          }
+          tc_commit(s_full);
+          if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+          if (++stage == kAttnStages) { stage = 0; phase ^= 1; }
+        }
+        if (ok) ok = issue_pv(nt - 1);
+        if (!ok) {
+          tc_commit(drain);
+          mbar_wait_drain(drain, 0);
+        }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (elect_one()) {
-      bool ok = mbar_wait(q_full, 0);
-      if (ok) {
-        tc_fence_after();
-        tc_cp_sf_atom(tmem + kColSfq, smem_desc(smem_u32(sSfq), 0, 128, 0));
-      }
-      // O += P V^T for key tile i (P from shared memory, written by the softmax warps).
-      auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait(p_full, i & 1)) return false;
-        tc_fence_after();
-        const int st = i % kAttnStages;
-        const uint32_t par = static_cast<uint32_t>(i & 1);
-        const uint32_t sfp = kColSfp + par * 8, sfv = kColSfv + par * 16;
-#pragma unroll
-        for (int a = 0; a < 2; ++a) {
-          tc_cp_sf_atom(tmem + sfp + 4 * a, smem_desc(smem_u32(sSfp + a * 512), 0, 128, 0));
-          tc_cp_sf_atom(tmem + sfv + 8 * a, smem_desc(smem_u32(sSfv(st) + a * 512), 0, 128, 0));
-          tc_cp_sf_atom(tmem + sfv + 8 * a + 4, smem_desc(smem_u32(sSfOnes + a * 512), 0, 128, 0));
-        }
-        const uint32_t p_base = smem_u32(sP), v_base = smem_u32(sV(st));
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {  // 4 x 64 keys
-          const int a = kk >> 1;
-          const uint32_t sf_id = static_cast<uint32_t>((kk & 1) * 2);
-          const uint32_t idesc = attn_idesc(kAttnNv) | (sf_id << 29) | (sf_id << 4);
-          tc_mma_mxf4(tmem + kColO, smem_desc(p_base + kk * 32, 16, 1024, 2), smem_desc(v_base + kk * 32, 16, 1024, 2),
-                      idesc, tmem + sfp + 4 * a, tmem + sfv + 8 * a, (i | kk) != 0);
-        }
-        tc_commit(o_done);
-        tc_commit(&kv_empty[st]);
-        return true;
-      };
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int j = 0; ok && j < nt; ++j) {
-        if (!mbar_wait(&kv_full[stage], phase)) { ok = false; break; }
-        if (j > 0 && !mbar_wait(s_free, (j - 1) & 1)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sfk = kColSfk + static_cast<uint32_t>(j & 1) * 8;
-        tc_cp_sf_atom(tmem + sfk, smem_desc(smem_u32(sSfk(stage)), 0, 128, 0));
-        tc_cp_sf_atom(tmem + sfk + 4, smem_desc(smem_u32(sSfk(stage) + 512), 0, 128, 0));
-        const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK(stage));
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {  // 2 x 64 of the head dimension
-          const uint32_t sf_id = static_cast<uint32_t>(kk * 2);
-          const uint32_t idesc = attn_idesc(kAttnBN) | (sf_id << 29) | (sf_id << 4);
-          tc_mma_mxf4(tmem + kColS, smem_desc(q_base + kk * 32, 16, 512, 4), smem_desc(k_base + kk * 32, 16, 512, 4),
-                      idesc, tmem + kColSfq, tmem + sfk, kk != 0);
-        }
-        tc_commit(s_full);
-        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
-        if (++stage == kAttnStages) { stage = 0; phase ^= 1; }
-      }
-      if (ok) ok = issue_pv(nt - 1);
-      if (!ok) {
-        tc_commit(drain);
-        mbar_wait_drain(drain, 0);
-      }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem, kAttnTmemCols);
     }
   } else {
-    // ------------------------------------------------------------------ softmax / PNQ (warps 2..17)
+    setmaxnreg_inc<kAttnSoftRegs>();
+    // ------------------------------------------------------------------ softmax / PNQ (warps 4..19)
     const int quad = warp & 3;          // TMEM lanes [32 quad, +32)
-    const int qt = (warp - 2) >> 2;     // keys [64 qt, +64) of every tile
+    const int qt = (warp - 4) >> 2;     // keys [64 qt, +64) of every tile
     const int r = quad * 32 + lane;     // query row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     int chat = 0;
@@ -504,13 +520,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
     }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kAttnTmemCols);
+    tc_fence_before();
+    __syncthreads();
   }
 }
 

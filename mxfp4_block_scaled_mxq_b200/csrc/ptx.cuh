@@ -103,6 +103,19 @@ __global__ void selftest_wait_timeout_kernel() {
   mbar_wait(&bar, 0);  // phase 0 never completes
 }
 
+// ----------------------------------------------------------------------------- registers
+// Warpgroup register reallocation: every thread of the warpgroup executes it.  An increase
+// waits until the CTA's pool (its launch allocation) has that many registers free, so
+// the warpgroups' shares must add up to at most the launch's total.
+template <int kRegs>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <int kRegs>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
 // ----------------------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
