@@ -109,18 +109,15 @@ __device__ __forceinline__ void bf16x16_to_float(const uint32_t (&w)[8], float (
 }
 
 // Largest |x| over 16 BF16 values held as 8 packed pairs, as FP32 bits (exact).
-// Magnitudes are compared with the packed BF16 max; non-negative BF16 patterns order
-// like unsigned integers, which combines the two halves.
+// Magnitudes are compared by the packed BF16 max of absolute values (its result's sign,
+// the XOR of the operands' signs, is cleared at the end); non-negative BF16 patterns
+// order like unsigned integers, which combines the two halves.
 __device__ __forceinline__ uint32_t bf16x16_absmax(const uint32_t (&w)[8]) {
-  uint32_t t = w[0] & 0x7FFF7FFFu;
-  __nv_bfloat162 m = *reinterpret_cast<const __nv_bfloat162*>(&t);
+  uint32_t m = w[0];
 #pragma unroll
-  for (int j = 1; j < 8; ++j) {
-    const uint32_t a = w[j] & 0x7FFF7FFFu;
-    m = __hmax2(m, *reinterpret_cast<const __nv_bfloat162*>(&a));
-  }
-  const uint32_t mb = *reinterpret_cast<const uint32_t*>(&m);
-  return max(mb & 0xFFFFu, mb >> 16) << 16;
+  for (int j = 1; j < 8; ++j) asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m) : "r"(w[j]));
+  m &= 0x7FFF7FFFu;
+  return max(m & 0xFFFFu, m >> 16) << 16;
 }
 
 // Block exponent from the block's absolute maximum (integer arithmetic on the FP32
