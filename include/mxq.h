@@ -331,10 +331,12 @@ MXQ_API mxq_precision mxq_select_precision(double sqnr_plain_db, double sqnr_tra
  * c is an integer offset (at least the row maximum of t minus 8); since E8M0 block scaling
  * is exactly equivariant under powers of two, the codes of P do not depend on which such c
  * is used.  2^(t - c) is evaluated as p(g) * 2^(n - c) with n = rint(t) (ties to even),
- * g = t - n and p the degree-4 Taylor polynomial of 2^g (a_0 = 1, a_k = a_(k-1) ln 2 / k in
- * FP64, rounded to FP32; Horner with FP32 fused multiply-adds; relative error < 6e-5);
+ * g = t - n and p the degree-3 Taylor polynomial of 2^g (a_0 = 1, a_k = a_(k-1) ln 2 / k in
+ * FP64, rounded to FP32; Horner with FP32 fused multiply-adds; relative error < 8.6e-4);
  * numerators with n - c < -126 are 0; a block's E8M0 exponent is taken from the numerator
- * of its largest score.  Scores must satisfy |t| < 2^22.
+ * of its largest score.  Scores must satisfy |t| < 2^22.  Numerators below 2^-118 of a
+ * row's largest one may be kept or flushed (the kernel's offset is raised lazily); they
+ * are below the FP32 resolution of l.
  *
  * mxq_attn_padded_keys -- Sp = S_kv rounded up to the kernel's 256-key tile (-1 if S_kv is
  * outside [1, 2^23]).

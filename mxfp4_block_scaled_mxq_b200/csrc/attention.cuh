@@ -113,11 +113,9 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
 // rint(t) in its low mantissa bits (|t| < 2^22), so n = r - 1.5 * 2^23 and g = t - n are
 // exact; and the FP32 bit pattern of 2^(n - chat) is (bits(r) + 127 - chat) * 2^23 modulo 2^32
 // (bits(1.5 * 2^23) * 2^23 vanishes modulo 2^32), one integer multiply-add, 0 for n - chat = -127.
-// kClamp = false skips the raise to chat - 127 for pairs already at or above it.
-template <bool kClamp = true>
 __device__ __forceinline__ float2 pnq_exp2_pair(float2 t, float lo, uint32_t bias_bits, const AttnParams& prm) {
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  if (kClamp) t = make_float2(fmaxf(t.x, lo), fmaxf(t.y, lo));
+  t = make_float2(fmaxf(t.x, lo), fmaxf(t.y, lo));
   const float2 r = __fadd2_rn(t, make_float2(kMagic, kMagic));
   const float2 n = __fadd2_rn(r, make_float2(-kMagic, -kMagic));
   const float2 g = __fadd2_rn(t, make_float2(-n.x, -n.y));
@@ -140,7 +138,7 @@ __device__ __forceinline__ void pnq_block_codes(const float* t, float lo, uint32
     float2 v[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-      v[q] = __fmul2_rn(pnq_exp2_pair<true>(make_float2(t[8 * w + 2 * q], t[8 * w + 2 * q + 1]), lo, bias_bits, prm),
+      v[q] = __fmul2_rn(pnq_exp2_pair(make_float2(t[8 * w + 2 * q], t[8 * w + 2 * q + 1]), lo, bias_bits, prm),
                         sc);
     codes[w] = e2m1x8(v[0].x, v[0].y, v[1].x, v[1].y, v[2].x, v[2].y, v[3].x, v[3].y);
   }
