@@ -253,11 +253,13 @@ __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__
       const float s = exp2_neg(e);  // exact power of two
 
       uint32_t out[2];
+      const float2 s2 = make_float2(s, s);
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
+      for (int q = 0; q < 2; ++q) {  // packed FP32x2 products (each exact, as two scalar ones)
         const float* g = f + 8 * q;
-        out[q] = e2m1x8(__fmul_rn(g[0], s), __fmul_rn(g[1], s), __fmul_rn(g[2], s), __fmul_rn(g[3], s),
-                        __fmul_rn(g[4], s), __fmul_rn(g[5], s), __fmul_rn(g[6], s), __fmul_rn(g[7], s));
+        const float2 v0 = __fmul2_rn(make_float2(g[0], g[1]), s2), v1 = __fmul2_rn(make_float2(g[2], g[3]), s2);
+        const float2 v2 = __fmul2_rn(make_float2(g[4], g[5]), s2), v3 = __fmul2_rn(make_float2(g[6], g[7]), s2);
+        out[q] = e2m1x8(v0.x, v0.y, v1.x, v1.y, v2.x, v2.y, v3.x, v3.y);
       }
       if (kQdq) {
         if (row < rows && k_ok) {
