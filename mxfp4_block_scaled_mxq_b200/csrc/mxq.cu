@@ -410,7 +410,16 @@ mxq_status mxq_dequant_mxfp4(const void* codes, const void* sf, int64_t rows, in
   const int64_t units = rows * (K / 16);
   const int64_t per_block = int64_t(mxq::kQuantThreads) * mxq::kDequantUnroll;
   int64_t blocks = (units + per_block - 1) / per_block;
-  const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;
+  // Grid-stride: exactly the CTAs that fit at once, so none starts late (a second, partial
+  // round of a latency-bound kernel costs as much as a full one).
+  static const int resident = [] {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, mxq::dequant_mxfp4_kernel, mxq::kQuantThreads, 0) !=
+            cudaSuccess || n < 1)
+      n = 1;
+    return n;
+  }();
+  const int64_t cap = static_cast<int64_t>(dev.sm_count) * resident;
   if (blocks > cap) blocks = cap;
   mxq::dequant_mxfp4_kernel<<<static_cast<unsigned>(blocks), mxq::kQuantThreads, 0, stream>>>(
       static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(sf), rows, K,
