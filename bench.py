@@ -60,7 +60,7 @@ def parse():
     p.add_argument("--impl", choices=["mxq", "reference"], default="mxq")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--e2e-steps", type=int, default=20)
+    p.add_argument("--e2e-steps", type=int, default=40)
     p.add_argument("--m", type=int, default=0, help="token count (0: the workload's own)")
     p.add_argument("--workload", choices=["wan_ffn", "wan_attn_hadamard", "flux_w4a8", "m_sweep", "qdq_wan_ffn",
                                           "policy_wan_ffn", "attn_wan"],
