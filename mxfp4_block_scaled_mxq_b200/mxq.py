@@ -11,6 +11,8 @@ the device is not an sm_100 GPU, calls raise.
 from __future__ import annotations
 
 import ctypes
+import functools
+import inspect
 import os
 
 import torch
@@ -233,6 +235,27 @@ def mxq_selftest_wait_timeout(stream=None) -> None:
 
 
 # ------------------------------------------------------------------ allocating helpers
+def _on_stream(fn):
+    """Runs an allocating helper with its `stream` argument as torch's current stream.
+
+    The caching allocator hands a freed block out again only after the work queued on the
+    stream that allocated it, so tensors the helper allocates (outputs and temporaries such
+    as the quantised activations of linear_w4a4) then stay valid for as long as the kernels
+    the helper queued on `stream` read or write them, whatever stream the caller is on."""
+    sig = inspect.signature(fn)
+
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        stream = kwargs["stream"] if "stream" in kwargs else sig.bind(*args, **kwargs).arguments.get("stream")
+        if stream is None:
+            return fn(*args, **kwargs)
+        s = torch.cuda.ExternalStream(stream) if isinstance(stream, int) else stream
+        with torch.cuda.stream(s):
+            return fn(*args, **kwargs)
+
+    return wrapper
+
+
 def _bf16_2d(x: torch.Tensor, name: str) -> torch.Tensor:
     if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
         raise ValueError(f"{name}: expected a 2-D bfloat16 CUDA tensor")
@@ -241,6 +264,7 @@ def _bf16_2d(x: torch.Tensor, name: str) -> torch.Tensor:
     return x
 
 
+@_on_stream
 def quantize_act(x: torch.Tensor, rule: int = MXQ_SCALE_OCP, hadamard128: bool = False, out=None, stream=None):
     """Dynamic MXFP4 quantisation of X[M][K] -> (codes [M][K/2] uint8, sf uint8[mxq_sf_bytes(M, K)])."""
     x = _bf16_2d(x, "x")
@@ -253,6 +277,7 @@ def quantize_act(x: torch.Tensor, rule: int = MXQ_SCALE_OCP, hadamard128: bool =
     return q, sf
 
 
+@_on_stream
 def quantize_act_fp8(x: torch.Tensor, act_scale: float, out=None, stream=None) -> torch.Tensor:
     """Static FP8 E4M3 quantisation of X[M][K] with per-tensor scale s -> uint8 [M][K]."""
     x = _bf16_2d(x, "x")
@@ -263,6 +288,7 @@ def quantize_act_fp8(x: torch.Tensor, act_scale: float, out=None, stream=None) -
     return q
 
 
+@_on_stream
 def pack_weight(w: torch.Tensor, rule: int = MXQ_SCALE_OCP, hadamard128: bool = False, stream=None):
     """Offline MXFP4 packing of W[N][K] -> (codes [N][K/2] uint8, sf uint8[mxq_sf_bytes(N, K)])."""
     w = _bf16_2d(w, "w")
@@ -280,6 +306,7 @@ def _out_bf16(M: int, N: int, device) -> torch.Tensor:
     return torch.empty(M, ldd, dtype=torch.bfloat16, device=device)[:, :N]
 
 
+@_on_stream
 def gemm_w4a4(a_codes, a_sf, b_codes, b_sf, M, N, K, alpha=1.0, bias=None, out=None, stream=None) -> torch.Tensor:
     """D[M][N] (BF16) = alpha * deq(A) deq(B)^T + bias, on the tensor cores."""
     d = _out_bf16(M, N, a_codes.device) if out is None else out
@@ -287,6 +314,7 @@ def gemm_w4a4(a_codes, a_sf, b_codes, b_sf, M, N, K, alpha=1.0, bias=None, out=N
     return d
 
 
+@_on_stream
 def gemm_w4a8(a_e4m3, act_scale, b_codes, b_sf, M, N, K, bias=None, out=None, stream=None) -> torch.Tensor:
     """D[M][N] (BF16) = act_scale * e4m3(A) deq(B)^T + bias, on the tensor cores."""
     d = _out_bf16(M, N, a_e4m3.device) if out is None else out
@@ -294,6 +322,7 @@ def gemm_w4a8(a_e4m3, act_scale, b_codes, b_sf, M, N, K, bias=None, out=None, st
     return d
 
 
+@_on_stream
 def dequant_mxfp4(codes: torch.Tensor, sf: torch.Tensor, K: int, out=None, stream=None) -> torch.Tensor:
     """MXFP4 codes [rows][K/2] + swizzled scales -> BF16 [rows][K] (exact values)."""
     rows = codes.shape[0]
@@ -302,6 +331,7 @@ def dequant_mxfp4(codes: torch.Tensor, sf: torch.Tensor, K: int, out=None, strea
     return o
 
 
+@_on_stream
 def qdq_act(x: torch.Tensor, fmt: int = MXQ_ACT_MXFP4, rule: int = MXQ_SCALE_OCP, hadamard128: bool = False,
             act_scale: float = 1.0, out=None, stream=None) -> torch.Tensor:
     """BF16 dequant(quant(X)) with the activation quantiser's arithmetic (fake quantisation)."""
@@ -313,6 +343,7 @@ def qdq_act(x: torch.Tensor, fmt: int = MXQ_ACT_MXFP4, rule: int = MXQ_SCALE_OCP
     return o
 
 
+@_on_stream
 def channel_absmax(x: torch.Tensor, hadamard128: bool = False, out=None, accumulate: bool = False,
                    stream=None) -> torch.Tensor:
     """Per-channel max |x R| over the rows (FP32 [K]); accumulate merges into `out`."""
@@ -323,6 +354,7 @@ def channel_absmax(x: torch.Tensor, hadamard128: bool = False, out=None, accumul
     return o
 
 
+@_on_stream
 def smooth_factors(amax_x: torch.Tensor, amax_w: torch.Tensor, alpha: float = 0.5, stream=None):
     """SmoothQuant (lambda, 1/lambda) from the channel maxima of activations and weights."""
     K = amax_x.numel()
@@ -332,6 +364,7 @@ def smooth_factors(amax_x: torch.Tensor, amax_w: torch.Tensor, alpha: float = 0.
     return lam, inv
 
 
+@_on_stream
 def quantize_smooth(x: torch.Tensor, chan_scale: torch.Tensor, rule: int = MXQ_SCALE_OCP,
                     hadamard128: bool = False, out=None, stream=None):
     """MXFP4 codes + scales of (x R) * chan_scale (per channel): 1/lambda for activations,
@@ -346,6 +379,7 @@ def quantize_smooth(x: torch.Tensor, chan_scale: torch.Tensor, rule: int = MXQ_S
     return q, sf
 
 
+@_on_stream
 def quantize_vt(v: torch.Tensor, rule: int = MXQ_SCALE_UOS, out=None, stream=None):
     """V [S][H*d] -> V^T MXFP4 (codes [H*d][Sp/2], scales) with 32-key blocks."""
     v = _bf16_2d(v, "v")
@@ -358,6 +392,7 @@ def quantize_vt(v: torch.Tensor, rule: int = MXQ_SCALE_UOS, out=None, stream=Non
     return out
 
 
+@_on_stream
 def attention_mxfp4(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, H: int, rule: int = MXQ_SCALE_UOS,
                     out=None, stream=None) -> torch.Tensor:
     """MXFP4 attention with UOS / PNQ: q [Sq][H*d], k, v [Skv][H*d] BF16 -> O [Sq][H*d] BF16.
@@ -373,6 +408,7 @@ def attention_mxfp4(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, H: int, r
     return o
 
 
+@_on_stream
 def linear_w4a4(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE_OCP, hadamard128: bool = False,
                 bias=None, stream=None) -> torch.Tensor:
     """The quantized linear layer: dynamic MXFP4 quantisation of X, then the W4A4 GEMM."""
@@ -386,6 +422,7 @@ def linear_workspace(M: int, K: int, device) -> torch.Tensor:
     return torch.empty(mxq_linear_workspace_bytes(M, K), dtype=torch.uint8, device=device)
 
 
+@_on_stream
 def linear_w4a4_ws(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE_OCP, alpha: float = 1.0,
                    bias=None, workspace=None, out=None, stream=None) -> torch.Tensor:
     """The quantized linear layer in one call of the C ABI (quantised activations in `workspace`)."""
@@ -398,6 +435,7 @@ def linear_w4a4_ws(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE
     return d
 
 
+@_on_stream
 def linear_w4a4_static(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_SCALE_OCP, alpha: float = 1.0,
                        bias=None, out=None, stream=None) -> torch.Tensor:
     """The quantized linear layer with the library's own fixed scratch (no allocation by the call)."""
@@ -409,6 +447,7 @@ def linear_w4a4_static(x: torch.Tensor, w_codes, w_sf, N: int, rule: int = MXQ_S
     return d
 
 
+@_on_stream
 def linear_w4a8(x: torch.Tensor, act_scale: float, w_codes, w_sf, N: int, bias=None, stream=None) -> torch.Tensor:
     """The W4A8 layer: static FP8 quantisation of X, then the W4A8 GEMM."""
     M, K = x.shape

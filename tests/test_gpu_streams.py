@@ -107,3 +107,21 @@ def test_cuda_graph_replay_matches_eager(M):
         torch.cuda.synchronize()
         np.testing.assert_array_equal(_bits(d), _bits(want))
     del g
+
+
+@pytest.mark.parametrize("as_handle", [False, True])
+def test_helpers_given_a_stream_from_another_stream(as_handle):
+    """The allocating helpers called with `stream=` while torch's current stream is the
+    default one (a torch stream or a raw cudaStream_t handle): their temporaries (the
+    quantised activations) are allocated on that stream, and D equals the default-stream D."""
+    M, N, K = 300, 520, 1280
+    x, _, wc, wsf = _layer(M, N, K, 95)
+    xd = x.cuda()
+    want = mxq.linear_w4a4(xd, wc, wsf, N)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    outs = [mxq.linear_w4a4(xd, wc, wsf, N, stream=s.cuda_stream if as_handle else s) for _ in range(4)]
+    s.synchronize()
+    for d in outs:
+        np.testing.assert_array_equal(_bits(d), _bits(want))
