@@ -200,8 +200,9 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD + " -- sample", "token_rows": CPU_SAMPLE_ROWS, "w_up_rows": n_up,
-                   "w_down_rows": n_dn},
+        "config": {"workload": WORKLOAD, "M": M_TOK, "parallelism": "replicas x1 (token batches, no collective)",
+                   "timing": "oracle on the host cores; each step a bounded sample of the workload "
+                             "(cpu_baseline.sample), wall clock"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
