@@ -288,7 +288,8 @@ __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__
 
 // The rotated variant of the tile: four lanes per 128-element chunk, lane j holding the
 // chunk's 32-block j as 16 packed pairs P[i] = (t[i], t[i + 16]).  Butterfly strides 1..8
-// run on packed pairs (FP32x2 add / fma with -1, both exact per half), stride 16 is the
+// run on packed pairs (FP32x2 adds, the difference by a negated operand: each exactly
+// rounded per half), stride 16 is the
 // within-pair butterfly, strides 32 and 64 are cross-lane exchanges (lanes xor 1 and xor 2);
 // the stage order and every rounding are those of the definition, so the rotated values are
 // bit-identical to the element-by-element butterfly.  A lane ends with exactly one 32-block:
@@ -319,7 +320,6 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
 
   const float c = __uint_as_float(kInvSqrt128Bits);
   const float2 cc = make_float2(c, c);
-  const float2 minus1 = make_float2(-1.f, -1.f);
   // kOutAbsmax: this lane's 32 column maxima over its rows of both passes; column k of
   // block j is cm[k] (k < 16: element k, else element k of the pairs' upper halves)
   float cm[kOut == kOutAbsmax ? 32 : 1];
@@ -363,7 +363,7 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
         if (i & h) continue;
         const float2 a = P[i], b = P[i + h];
         P[i] = __fadd2_rn(a, b);
-        P[i + h] = __ffma2_rn(b, minus1, a);  // a - b, exactly rounded
+        P[i + h] = __fadd2_rn(a, make_float2(-b.x, -b.y));  // a - b, exactly rounded
       }
     }
 #pragma unroll
