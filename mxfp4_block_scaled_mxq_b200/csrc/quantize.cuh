@@ -289,8 +289,8 @@ __device__ __forceinline__ void quantize_mxfp4_tile(const uint16_t* __restrict__
 // The rotated variant of the tile: four lanes per 128-element chunk, lane j holding the
 // chunk's 32-block j as 16 packed pairs P[i] = (t[i], t[i + 16]).  Butterfly strides 1..8
 // run on packed pairs (FP32x2 adds, the difference by a negated operand: each exactly
-// rounded per half), stride 16 is the
-// within-pair butterfly, strides 32 and 64 are cross-lane exchanges (lanes xor 1 and xor 2);
+// rounded per half), stride 16 is the within-pair butterfly, strides 32 and 64 are
+// cross-lane exchanges (lanes xor 1 and xor 2);
 // the stage order and every rounding are those of the definition, so the rotated values are
 // bit-identical to the element-by-element butterfly.  A lane ends with exactly one 32-block:
 // its maximum, scale and 16 code bytes need no further exchange.  256 threads cover 64 rows
