@@ -27,11 +27,11 @@ Parity status per function (what pins each one is in ``tests/test_oracle_*.py``)
   smooth_factors              the migration factors at alpha = 0.5, 1 and 0
   sqnr_sums / sqnr_db /       pinned: closed forms (uniform relative error, known pairs,
   select_precision            limits) and every tier boundary
-  pnq_exp2                    pinned: Taylor remainder bound, exact at integers, exact
-                              power-of-two offsets, the flush below 2^-126
   attention_mxfp4             pinned: the textbook FP64 softmax of the dequantised
-                              operands (P unquantised), equal-score and dominant-key
-                              closed forms, PNQ weights summing to one
+                              operands (P unquantised); PNQ and the conventional order
+                              against an independent FP64 NumPy restatement (exact
+                              exponentials, MX block maxima); equal-score and
+                              dominant-key closed forms, PNQ weights summing to one
 """
 
 from __future__ import annotations
@@ -123,8 +123,6 @@ def _load():
     lib.oracle_sqnr_db.restype = ctypes.c_double
     lib.oracle_select_precision.argtypes = [ctypes.c_double] * 4
     lib.oracle_select_precision.restype = ctypes.c_int
-    lib.oracle_pnq_exp2.argtypes = [ctypes.c_float, ctypes.c_int]
-    lib.oracle_pnq_exp2.restype = ctypes.c_float
     lib.oracle_attention_mxfp4.argtypes = [P, P, P, I64, I64, I64, I64, I64, ctypes.c_int, ctypes.c_int, P, I64,
                                            P, P, ctypes.c_int]
     lib.oracle_attention_mxfp4.restype = None
@@ -369,11 +367,6 @@ def select_precision(sqnr_plain_db: float, sqnr_transform_db: float, high_db: fl
 
 # ---------------------------------------------------------------- MXFP4 attention (UOS + PNQ)
 ATTN_PNQ, ATTN_NORMALISE_THEN_QUANTISE, ATTN_UNQUANTISED_P = 0, 1, 2
-
-
-def pnq_exp2(t: float, chat: int) -> float:
-    """2^(t - chat) by the attention numerators' polynomial definition (FP32)."""
-    return float(_load().oracle_pnq_exp2(ctypes.c_float(t), int(chat)))
 
 
 def attention_mxfp4(q, k, v, H: int, d: int, rows=None, rule: int = RULE_UOS, mode: int = ATTN_PNQ,

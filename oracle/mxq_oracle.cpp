@@ -65,17 +65,13 @@
 //    unnormalised exponentials quantised to MXFP4 in 32-key blocks BEFORE the row sum
 //    (PNQ), the row sum l taken over the quantised values, O = (deq(P) deq(V)) / l.
 //    Readings (the pages fix none of these): the numerators are taken in base 2,
-//    t = fl32(fl32(S) * fl32(log2(e) / sqrt(d))), relative to an integer offset
-//    c = ceil(max_j t_j) -- a power-of-two offset, under which E8M0 block scaling is
-//    exactly equivariant, so the codes do not depend on it; the exponential is
-//    2^(t - c) = p(g) * 2^(n - c) with n = rint(t) (nearest, ties to even), g = t - n in
-//    [-1/2, 1/2] and p the degree-3 Taylor polynomial of 2^g (coefficients a_0 = 1,
-//    a_k = a_(k-1) * ln 2 / k in FP64, rounded to FP32; Horner with FP32 fused
-//    multiply-adds; relative error below 8.6e-4, more than two orders of magnitude under
-//    the E2M1 step), and numerators with n - c < -126 are 0.  A block's E8M0 exponent is taken from
-//    the numerator of its largest score (the exponential is monotone).  These FP32 steps
-//    decide the quantised codes, so they are taken in the kernel's precision; the rest is
-//    FP64.
+//    t = fl32(fl32(S) * fl32(log2(e) / sqrt(d))) (the scores in FP32, as a tensor core
+//    accumulates them), relative to an integer offset c = ceil(max_j t_j) -- a
+//    power-of-two offset, under which E8M0 block scaling is exactly equivariant, so the
+//    codes do not depend on it.  Each numerator is the exact exponential 2^(t - c),
+//    evaluated in FP64; a 32-key block's E8M0 exponent follows the MX definition, from
+//    the maximum of that block's numerators, and each numerator is rounded to E2M1 in
+//    FP64 against it.  The row sum, the division and the product with V are FP64.
 //  * Scale-factor memory layout (not given by the pages; a reading): rows padded
 //    to a multiple of 128, scale columns to a multiple of 4, 512-byte atoms of
 //    128 rows x 4 scale columns, byte
@@ -466,35 +462,10 @@ void oracle_gemm(int a_kind, const uint8_t* a_codes, const uint8_t* a_sf, int64_
 
 // ---------------------------------------------------------------- MXFP4 attention
 
-constexpr int kExp2Terms = 4;  // degree 3
-
-// Coefficients of the degree-3 Taylor polynomial of 2^g around g = 0.
-static void pnq_exp2_coefficients(float* a) {
-  double c = 1.0;
-  const double ln2 = std::log(2.0);
-  for (int k = 0; k < kExp2Terms; ++k) {
-    a[k] = static_cast<float>(c);
-    c = c * ln2 / static_cast<double>(k + 1);
-  }
-}
-
-// 2^(t - chat) by the definition above (t finite, chat an integer).
-float oracle_pnq_exp2(float t, int chat) {
-  float a[kExp2Terms];
-  pnq_exp2_coefficients(a);
-  const float n = std::nearbyint(t);  // the default rounding mode: to nearest, ties to even
-  const float g = t - n;              // exact
-  float p = a[kExp2Terms - 1];
-  for (int k = kExp2Terms - 2; k >= 0; --k) p = std::fmaf(p, g, a[k]);
-  const long e = static_cast<long>(n) - chat;
-  if (e < -126) return 0.0f;
-  return p * std::ldexp(1.0f, static_cast<int>(e));
-}
-
 // Attention of the sampled query rows q_rows[0..n_rows) for every head.
 //   q: [Sq][ld], k, v: [Skv][ld] BF16, head h in columns [h*d, (h+1)*d), d % 32 == 0.
 //   mode 0: PNQ (quantise the numerators, then the row sum); 1: the conventional order
-//   (row-normalise in FP32, quantise the probabilities, no further division); 2: no
+//   (row-normalise in FP64, quantise the probabilities, no further division); 2: no
 //   quantisation of P (FP64 softmax of the quantised-operand scores).
 //   out: [n_rows][H][d] FP64; wsum: [n_rows][H] sum of the implied attention weights.
 void oracle_attention_mxfp4(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t Sq, int64_t Skv,
@@ -526,7 +497,8 @@ void oracle_attention_mxfp4(const uint16_t* q, const uint16_t* k, const uint16_t
   parallel_rows(n_rows, nthreads, [&](int64_t i0, int64_t i1) {
     std::vector<uint8_t> qc(static_cast<size_t>(HD / 2)), qs(static_cast<size_t>(HD / kBlock));
     std::vector<double> Q(static_cast<size_t>(HD)), P(static_cast<size_t>(Sp));
-    std::vector<float> t(static_cast<size_t>(Skv)), pt(static_cast<size_t>(Sp));
+    std::vector<float> t(static_cast<size_t>(Skv));
+    std::vector<double> pd(static_cast<size_t>(Sp));
     for (int64_t i = i0; i < i1; ++i) {
       const int64_t row = q_rows[i];
       oracle_quantize_mxfp4(q + row * ld, 1, HD, ld, rule, 0, qc.data(), qs.data(), 1);
@@ -545,26 +517,20 @@ void oracle_attention_mxfp4(const uint16_t* q, const uint16_t* k, const uint16_t
           for (int64_t j = Skv; j < Sp; ++j) P[j] = 0.0;
           for (int64_t j = 0; j < Sp; ++j) P[j] /= l;
         } else {
-          const int chat = static_cast<int>(std::ceil(tmax));
-          for (int64_t j = 0; j < Sp; ++j) pt[j] = j < Skv ? oracle_pnq_exp2(t[j], chat) : 0.0f;
+          // the unnormalised exponentials relative to the integer offset c, exact in FP64
+          const double c = std::ceil(static_cast<double>(tmax));
+          for (int64_t j = 0; j < Sp; ++j) pd[j] = j < Skv ? std::exp2(static_cast<double>(t[j]) - c) : 0.0;
           if (mode == 1) {  // conventional: normalise, then quantise
             double l = 0.0;
-            for (int64_t j = 0; j < Sp; ++j) l += pt[j];
-            for (int64_t j = 0; j < Sp; ++j) pt[j] = static_cast<float>(pt[j] / l);
+            for (int64_t j = 0; j < Sp; ++j) l += pd[j];
+            for (int64_t j = 0; j < Sp; ++j) pd[j] /= l;
           }
           for (int64_t b = 0; b < Sp / kBlock; ++b) {  // MXFP4 of the numerators, 32-key blocks
-            // the block exponent from the numerator of the block's largest score
-            float bmax = -INFINITY;
-            for (int u = 0; u < kBlock; ++u)
-              if (b * kBlock + u < Skv) bmax = std::max(bmax, t[b * kBlock + u]);
-            double amax = bmax == -INFINITY ? 0.0 : static_cast<double>(oracle_pnq_exp2(bmax, chat));
-            if (mode == 1) {  // conventional order: the largest normalised probability
-              amax = 0.0;
-              for (int u = 0; u < kBlock; ++u) amax = std::max(amax, static_cast<double>(pt[b * kBlock + u]));
-            }
+            double amax = 0.0;  // the MX block maximum
+            for (int u = 0; u < kBlock; ++u) amax = std::max(amax, std::fabs(pd[b * kBlock + u]));
             const int e = oracle_block_exponent(amax, rule);
             for (int u = 0; u < kBlock; ++u) {
-              const double x = std::ldexp(static_cast<double>(pt[b * kBlock + u]), -e);
+              const double x = std::ldexp(pd[b * kBlock + u], -e);
               P[b * kBlock + u] = std::ldexp(oracle_e2m1_decode(oracle_e2m1_encode(x)), e);
             }
           }

@@ -1,5 +1,6 @@
-"""Pins of the oracle's MXFP4 attention (UOS + PNQ): its exponential, closed-form
-outputs, and the properties the MXAttention page states.
+"""Pins of the oracle's MXFP4 attention (UOS + PNQ): an independent FP64 NumPy
+restatement of both quantisation orders, closed-form outputs, and the properties the
+MXAttention page states.
 
 [MXAttention: Data-Free Optimal Scaling and Pre-Normalization Quantization for MXFP4
  Attention -- TL;DR, "What it actually does"]
@@ -13,46 +14,6 @@ import torch
 
 import oracle
 from mxfp4_block_scaled_mxq_b200 import inputs
-
-
-def _f32(x):
-    return float(np.float32(x))
-
-
-def test_pnq_exp2_accuracy():
-    """Relative error against 2^(t - c) over the range softmax numerators use: below the
-    degree-3 Taylor remainder of 2^g on |g| <= 1/2, (ln 2 / 2)^4 / 4! * 2^(1/2) = 8.50e-4,
-    and above (ln 2 / 2)^4 / 4! = 6.01e-4, which it reaches near g = 1/2 (so a polynomial
-    of another degree fails one side)."""
-    ts = np.float32(np.linspace(-40.0, 8.0, 20011))
-    worst = 0.0
-    for t in ts:
-        want = 2.0 ** (float(t) - 3)
-        worst = max(worst, abs(oracle.pnq_exp2(float(t), 3) - want) / want)
-    assert 5.5e-4 < worst < 8.6e-4, worst
-
-
-@pytest.mark.parametrize("t", [-17.37, -0.001, 0.0, 2.5, 7.99])
-def test_pnq_exp2_offset_is_an_exact_power_of_two(t):
-    """Changing the integer offset scales the numerator by exactly a power of two (the
-    property that makes the MXFP4 codes independent of the offset)."""
-    t = _f32(t)
-    a, b = oracle.pnq_exp2(t, 0), oracle.pnq_exp2(t, 5)
-    assert a == b * 32.0
-
-
-def test_pnq_exp2_flushes_below_2_to_minus_126():
-    """Zero once the rounded integer part is below -126 (rint(-126.5) = -126: ties to even)."""
-    assert oracle.pnq_exp2(-127.0, 0) == 0.0
-    assert oracle.pnq_exp2(-126.6, 0) == 0.0
-    assert oracle.pnq_exp2(-126.5, 0) > 0.0
-    assert oracle.pnq_exp2(-126.0, 0) > 0.0
-
-
-def test_pnq_exp2_is_exact_at_integers():
-    """g = 0 at integer t, and p(0) = a_0 = 1: an exact power of two."""
-    for t in (-100.0, -3.0, 0.0, 5.0):
-        assert oracle.pnq_exp2(t, 2) == 2.0 ** (t - 2)
 
 
 def test_equal_scores_average_the_values():
@@ -72,7 +33,9 @@ def test_equal_scores_average_the_values():
 
 def test_one_dominant_key_returns_its_value():
     """One key's score exceeds the others' by more than 126 in base 2: every other
-    numerator flushes to 0, so O is exactly that key's dequantised value row."""
+    numerator is below 2^-126, under a quarter of the smallest E8M0 step (2^-127 x 0.5
+    is the least non-zero E2M1 value), so it quantises to 0 and O is exactly that key's
+    dequantised value row."""
     H, d, S = 1, 32, 64
     q = torch.zeros(1, d, dtype=torch.bfloat16)
     q[0, 0] = 24.0
@@ -153,3 +116,76 @@ def test_unquantised_mode_is_the_textbook_softmax_of_the_quantised_operands(rule
         want = (p / p.sum(axis=1, keepdims=True)) @ V[:, cols]
         np.testing.assert_allclose(got[:, h, :], want, rtol=2e-5, atol=2e-5 * np.abs(want).max())
     np.testing.assert_allclose(ws, 1.0, rtol=1e-12)
+
+
+def _mx_round_rows(p, rule):
+    """MXFP4 round trip of FP64 values in 32-element blocks along the last axis, written
+    from the MX definition alone: the block scale is the smallest power of two 2^e with
+    amax / 2^e < 8 (OCP) or <= 7.25 (UOS), e >= -127; each value goes to the nearest
+    E2M1 magnitude (ties to the even code index), saturating at 6."""
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    blocks = p.reshape(p.shape[:-1] + (-1, 32))
+    amax = np.abs(blocks).max(axis=-1, keepdims=True)
+    mant, ex = np.frexp(amax)                          # amax = mant 2^ex, mant in [0.5, 1)
+    e = np.where(amax > 0, ex - 1 - 2, -127)           # floor(log2 amax) - 2
+    if rule == oracle.RULE_UOS:
+        e = np.where(amax > np.ldexp(7.25, e), e + 1, e)
+    e = np.maximum(e, -127)
+    a = np.minimum(np.abs(blocks) / np.ldexp(1.0, e), 6.0)
+    dist = np.abs(a[..., None] - grid)
+    best = dist.min(axis=-1, keepdims=True)
+    tied = dist == best
+    # lowest index among the minima, unless a tie offers an even index
+    idx = np.where(tied[..., ::2].any(axis=-1), np.argmax(tied * (np.arange(8) % 2 == 0), axis=-1),
+                   np.argmax(tied, axis=-1))
+    return (np.sign(blocks) * grid[idx] * np.ldexp(1.0, e)).reshape(p.shape)
+
+
+@pytest.mark.parametrize("mode", [oracle.ATTN_PNQ, oracle.ATTN_NORMALISE_THEN_QUANTISE])
+@pytest.mark.parametrize("rule,scale", [(oracle.RULE_UOS, 1.0), (oracle.RULE_UOS, 2.5), (oracle.RULE_OCP, 2.0)])
+def test_quantised_p_matches_an_independent_fp64_restatement(mode, rule, scale):
+    """PNQ (quantise the unnormalised exponentials, then sum the quantised values and
+    divide) and the conventional order (normalise, then quantise) restated in FP64 NumPy:
+    scores t = fl32(fl32(S) fl32(log2 e / sqrt d)), numerators 2^(t - ceil(max t)) by
+    NumPy's exp2, MX blocks of 32 keys with the scale from the block maximum.  A wrong
+    block maximum, offset, rounding rule or quantisation point moves whole codes, so
+    agreement to 1e-12 leaves no room for any of them."""
+    H, d, Sq, Skv = 2, 64, 6, 150        # 150 keys: a ragged last block, zero-padded
+    q = inputs.normal_bf16(Sq, H * d, scale, seed=61)
+    k = inputs.normal_bf16(Skv, H * d, scale, seed=62)
+    v = inputs.heavy_tailed_bf16(Skv, H * d, seed=63)
+    got, ws = oracle.attention_mxfp4(q, k, v, H, d, rule=rule, mode=mode)
+    Q, K = _deq(q, rule), _deq(k, rule)
+    Skv_pad = (Skv + 31) // 32 * 32
+    vt = torch.zeros(H * d, Skv_pad, dtype=torch.bfloat16)
+    vt[:, :Skv] = v.t()
+    V = _deq(vt, rule).T                 # [Skv_pad][H*d], zero rows past Skv
+    c32 = np.float32(1.4426950408889634 / math.sqrt(d))
+    for h in range(H):
+        cols = slice(h * d, (h + 1) * d)
+        t = (Q[:, cols] @ K[:, cols].T).astype(np.float32) * c32          # FP32 product
+        c = np.ceil(t.max(axis=1, keepdims=True).astype(np.float64))
+        p = np.zeros((Sq, Skv_pad))
+        p[:, :Skv] = np.exp2(t.astype(np.float64) - c)
+        if mode == oracle.ATTN_PNQ:
+            pq = _mx_round_rows(p, rule)
+            w = pq / pq.sum(axis=1, keepdims=True)
+        else:
+            w = _mx_round_rows(p / p.sum(axis=1, keepdims=True), rule)
+        want = w @ V[:, cols]
+        np.testing.assert_allclose(got[:, h, :], want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+        np.testing.assert_allclose(ws[:, h], w.sum(axis=1), rtol=1e-12)
+    if mode == oracle.ATTN_PNQ:
+        np.testing.assert_allclose(ws, 1.0, rtol=1e-12)
+
+
+def test_the_restatement_sees_a_wrong_quantisation_point():
+    """The restatement above tells the two orders apart on this input (so a swapped mode
+    in the oracle would fail it)."""
+    H, d, Sq, Skv = 1, 64, 6, 150
+    q = inputs.normal_bf16(Sq, H * d, 2.5, seed=61)
+    k = inputs.normal_bf16(Skv, H * d, 2.5, seed=62)
+    v = inputs.heavy_tailed_bf16(Skv, H * d, seed=63)
+    a, _ = oracle.attention_mxfp4(q, k, v, H, d, mode=oracle.ATTN_PNQ)
+    b, _ = oracle.attention_mxfp4(q, k, v, H, d, mode=oracle.ATTN_NORMALISE_THEN_QUANTISE)
+    assert np.abs(a - b).max() > 1e-3 * np.abs(a).max()
