@@ -26,6 +26,12 @@
  *     state (it reads its own static device status word, see mxq_debug_poll).
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and never synchronises it.  Calls are thread-safe.
+ *   - Calls work on the current CUDA device, and one process may drive several devices.
+ *     The first call that launches a given kernel on a device does that device's one-time
+ *     set-up (the kernel's shared-memory opt-in, its occupancy, the static scratch address);
+ *     make that first call outside stream capture.  A set-up that fails returns
+ *     MXQ_ERR_CUDA and is tried again on the next call.  The set-up is kept for the life of
+ *     the process: after cudaDeviceReset the library must not be used on that device again.
  *   - Stream order holds as for any kernel, with one refinement: the GEMM kernels
  *     (mxq_gemm_*, mxq_linear_*) are launched with programmatic stream
  *     serialisation.  If the kernel before them in the stream lets dependents start
@@ -200,7 +206,8 @@ MXQ_API mxq_status mxq_linear_w4a4(const void* x_bf16, int64_t M, int64_t K, int
  * mxq_linear_w4a4_static -- mxq_linear_w4a4 without a caller workspace, allocating nothing:
  * the quantised activations go to a fixed buffer inside the library (one per device, a
  * file-scope device array of MXQ_STATIC_SCRATCH_BYTES = 16 MiB, whose address is looked up
- * once per device).  The pages have no counterpart of this call; it serves callers that
+ * by the first call on each device, with that device current; make that first call outside
+ * stream capture).  The pages have no counterpart of this call; it serves callers that
  * cannot hand out device memory.  Returns MXQ_ERR_SHAPE when mxq_linear_workspace_bytes(M, K)
  * exceeds the buffer (for K = 5120 about 6100 rows).  Nothing in the buffer needs to start at
  * zero.  The buffer is shared by every call on the device: calls that overlap in time
@@ -330,13 +337,17 @@ MXQ_API mxq_precision mxq_select_precision(double sqnr_plain_db, double sqnr_tra
  *   l = sum_j deq(P)_j,  O = deq(P) deq(V) / l.
  * c is an integer offset (at least the row maximum of t minus 8); since E8M0 block scaling
  * is exactly equivariant under powers of two, the codes of P do not depend on which such c
- * is used.  2^(t - c) is evaluated as p(g) * 2^(n - c) with n = rint(t) (ties to even),
- * g = t - n and p the degree-3 Taylor polynomial of 2^g (a_0 = 1, a_k = a_(k-1) ln 2 / k in
- * FP64, rounded to FP32; Horner with FP32 fused multiply-adds; relative error < 8.6e-4);
- * numerators with n - c < -126 are 0; a block's E8M0 exponent is taken from the numerator
- * of its largest score.  Scores must satisfy |t| < 2^22.  Numerators below 2^-118 of a
- * row's largest one may be kept or flushed (the kernel's offset is raised lazily); they
- * are below the FP32 resolution of l.
+ * is used.  The codes of P are those of the exact exponential 2^(t - c): a block's E8M0
+ * exponent follows from its largest score by integer arithmetic (floor(t_max - c) - 2, plus
+ * one under UOS when the fraction of t_max - c exceeds log2(1.8125)), and each element code
+ * from a cubic q(g) in g = t - rint(t) (FP32 Horner, the last step rounded up; coefficients
+ * from mxq_attn_code_poly) whose FP32 values cross the four E2M1 decision levels 0.75,
+ * 0.875, 1 and 1.25 at exactly the FP32 g where 2^g crosses them.  Scores must satisfy
+ * |t| < 2^22.  Numerators below 2^-118 of a row's largest one may be kept or flushed to 0
+ * (the kernel's offset is raised lazily); they are below the FP32 resolution of l.
+ *
+ * mxq_attn_code_poly -- writes {1, a1, a2, a3}, the FP32 coefficients of that cubic, to
+ * coeffs[0..3] (host only, no device access; for checking the decision property above).
  *
  * mxq_attn_padded_keys -- Sp = S_kv rounded up to the kernel's 256-key tile (-1 if S_kv is
  * outside [1, 2^23]).
@@ -353,6 +364,8 @@ MXQ_API mxq_precision mxq_select_precision(double sqnr_plain_db, double sqnr_tra
  * 1 <= S_q <= 8388480; all buffers 16-byte aligned.  One sequence per call.
  */
 MXQ_API int64_t mxq_attn_padded_keys(int64_t S_kv);
+
+MXQ_API void mxq_attn_code_poly(float coeffs[4]);
 
 MXQ_API mxq_status mxq_quantize_vt(const void* v_bf16, int64_t S, int64_t HD, int64_t ldv,
                                    mxq_scale_rule rule, void* codes_out, void* sf_out,

@@ -6,14 +6,16 @@
 //   O = (deq(P) deq(V)) / l,   P = MXFP4(2^(t - c)),   l = sum_j deq(P)_j,
 //   t = fl32(S * log2(e) / sqrt(d)),   S = deq(Q) deq(K)^T,
 //
-// with Q, K in 32-blocks along the head dimension, V and P in 32-blocks along the keys,
+// with Q, K in 32-blocks along the head dimension, V and P in 32-blocks along the keys and
 // c an integer offset (a power-of-two factor, under which the E8M0 block scaling is
-// exactly equivariant: the codes of P do not depend on it) and 2^(t - c) the degree-3
-// Taylor polynomial of 2^g, g = t - rint(t), times 2^(rint(t) - c) (0 when rint(t) - c <
-// -126); a block's E8M0 exponent comes from the numerator of its largest score.  The row sum is taken over the quantised numerators
-// (PNQ), so the implied weights sum to one by construction; it is computed by the
-// tensor core itself: V^T carries one extra row of ones, so column d of the P V
-// accumulator is l.
+// exactly equivariant: the codes of P do not depend on it).  The numerators' values are
+// never needed, only their MXFP4 codes, and those the kernel decides exactly as the exact
+// exponential does (see pnq_code_poly): a block's E8M0 exponent is taken from its largest
+// score by integer arithmetic, and each code from a cubic in g = t - rint(t) that crosses
+// the four E2M1 decision levels it can meet at the same FP32 g as 2^g does.  The row sum is
+// taken over the quantised numerators (PNQ), so the implied weights sum to one by
+// construction; it is computed by the tensor core itself: V^T carries one extra row of
+// ones, so column d of the P V accumulator is l.
 //
 // One CTA per (128 queries, head), head dimension 128, 256 keys per tile:
 //   warp 0      TMA producer: the Q tile (64-byte swizzle) once; per key tile the K
@@ -82,10 +84,29 @@ __host__ __device__ constexpr uint32_t attn_idesc(int n) {
          (static_cast<uint32_t>(kAttnBM >> 4) << 24);
 }
 
-constexpr int kExp2Terms = 4;  // degree-3 Taylor polynomial of 2^g (relative error < 8.6e-4)
+// The numerators' codes.  A key's scaled numerator is x = 2^(t - c - e) = 2^m 2^g with
+// n = rint(t) (ties to even), g = t - n in [-1/2, 1/2] (exact in FP32) and m = n - c - e an
+// integer; its E2M1 code is decided by x against the rounding boundaries 0.25, 0.75, 1.25,
+// 1.75, 2.5, 3.5 and 5.  With 2^g in [0.707, 1.415] the boundary an octave m can meet sits at
+// one of four levels of 2^g: 0.75 (m = 0), 0.875 (m = 1, 2), 1 (m = -2) and 1.25 (m = 0, 1,
+// 2); octaves m <= -3 give 0 and m = 3 gives 6 whatever g is.  So a code needs 2^g only on
+// the right side of those four levels.  The kernel uses the cubic
+//   q(g) = 1 + a1 g + a2 g^2 + a3 g^3  (Horner, FP32 fused multiply-adds, the last step
+//   rounded toward +infinity),
+// monotone on [-1/2, 1/2] and within 4e-4 of 2^g, whose FP32 coefficients were chosen by
+// search so that, for every FP32 g, q(g) reaches 0.75, 0.875 and 1.25 (with the E2M1 tie
+// rule of the conversion: a tie at 0.75 or 0.875 goes up, at 1.25 down) exactly when 2^g
+// does, i.e. when g passes log2(0.75), log2(0.875), log2(1.25); the rounded-up last step
+// makes q(g) > 1 exactly when g > 0.  The codes are therefore those of the exact
+// exponential for every key whose block scale lies within the E8M0 range (keys at least
+// 2^-126 of the row's largest numerator); only numerators below that are flushed to 0.
+constexpr float kCodeA1 = 0x1.63037cp-1f, kCodeA2 = 0x1.ee3f14p-3f, kCodeA3 = 0x1.b23daap-5f;
+// log2(0.90625) = log2(7.25 / 8), rounded down to FP32: the UOS rule raises a block's
+// exponent when the fraction of its largest t - c exceeds log2(1.8125), i.e. when g lies in
+// (log2(0.90625), 0); g > this constant is the exact test (the logarithm is irrational).
+constexpr float kUosFracThreshold = -0x1.22dadep-3f;
 
 struct AttnParams {
-  float exp2c[kExp2Terms];  // Taylor coefficients a_k = (ln 2)^k / k! of 2^g, FP32
   float t_scale;   // fl32(log2(e) / sqrt(d))
   int Sq;
   int Skv;
@@ -106,61 +127,69 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
   return r;
 }
 
-// Numerators of a pair of keys: 2^(t - chat) = p(g) * 2^(n - chat), n = rint(t), g = t - n,
-// p the Taylor polynomial of 2^g (Horner, FP32 fused multiply-adds), 0 when n - chat < -126.
-// Everything runs on the FMA pipe: t is first raised to chat - 127 (masked keys at -inf and
-// every t whose n - chat would be -127 or less give exactly 0 below); r = t + 1.5 * 2^23 holds
-// rint(t) in its low mantissa bits (|t| < 2^22), so n = r - 1.5 * 2^23 and g = t - n are
+// Scaled code values of a pair of keys: q(g) 2^(n - chat), n = rint(t), g = t - n, q the code
+// cubic above (Horner, FP32 fused multiply-adds, the last one rounded up), 0 when n - chat <
+// -126.  Everything runs on the FMA pipe: t is first raised to chat - 127 (masked keys at -inf
+// and every t whose n - chat would be -127 or less give exactly 0 below); r = t + 1.5 * 2^23
+// holds rint(t) in its low mantissa bits (|t| < 2^22), so n = r - 1.5 * 2^23 and g = t - n are
 // exact; and the FP32 bit pattern of 2^(n - chat) is (bits(r) + 127 - chat) * 2^23 modulo 2^32
 // (bits(1.5 * 2^23) * 2^23 vanishes modulo 2^32), one integer multiply-add, 0 for n - chat = -127.
-__device__ __forceinline__ float2 pnq_exp2_pair(float2 t, float lo, uint32_t bias_bits, const AttnParams& prm) {
+__device__ __forceinline__ float2 pnq_code_pair(float2 t, float lo, uint32_t bias_bits) {
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
   t = make_float2(fmaxf(t.x, lo), fmaxf(t.y, lo));
   const float2 r = __fadd2_rn(t, make_float2(kMagic, kMagic));
   const float2 n = __fadd2_rn(r, make_float2(-kMagic, -kMagic));
   const float2 g = __fadd2_rn(t, make_float2(-n.x, -n.y));
-  float2 p = make_float2(prm.exp2c[kExp2Terms - 1], prm.exp2c[kExp2Terms - 1]);
-#pragma unroll
-  for (int k = kExp2Terms - 2; k >= 0; --k) p = __ffma2_rn(p, g, make_float2(prm.exp2c[k], prm.exp2c[k]));
+  float2 p = __ffma2_rn(make_float2(kCodeA3, kCodeA3), g, make_float2(kCodeA2, kCodeA2));
+  p = __ffma2_rn(p, g, make_float2(kCodeA1, kCodeA1));
+  p = __ffma2_ru(p, g, make_float2(1.0f, 1.0f));
   const float2 sc = make_float2(__uint_as_float(__float_as_uint(r.x) * 8388608u + bias_bits),
                                 __uint_as_float(__float_as_uint(r.y) * 8388608u + bias_bits));
   return __fmul2_rn(p, sc);
 }
 
-// E2M1 codes of one 32-key block: numerators 2^(t - c) (raised to c - 127 first, so
+// E8M0 exponent of a block whose largest score is tmax, relative to the offset cp: the MX
+// rule applied to the exact largest numerator 2^(tmax - cp), by integer arithmetic on
+// n = rint(tmax) and g = tmax - n: floor(tmax - cp) - 2 (OCP), one more under UOS when the
+// fraction of tmax - cp exceeds log2(1.8125) (largest numerator above 7.25 2^(e - 2)),
+// clamped to -127; -127 for a block with no key at or above cp - 127 (masked keys are -inf).
+template <bool kUOS>
+__device__ __forceinline__ int pnq_block_exponent(float tmax, int cp) {
+  if (!(tmax >= static_cast<float>(cp - 127))) return -127;
+  const float n = rintf(tmax);  // nearest, ties to even (|tmax| < 2^22)
+  const float g = tmax - n;     // exact, in [-1/2, 1/2]
+  int e = static_cast<int>(n) - cp - 2;
+  if (g < 0.f && !(kUOS && g > kUosFracThreshold)) e -= 1;
+  return e < -127 ? -127 : e;
+}
+
+// E2M1 codes of one 32-key block: code values q(g) 2^(n - c) (t raised to c - 127 first, so
 // keys past the end and underflowing keys give 0) times the block's 2^-e, rounded to
 // nearest even with saturation.  The general form.
 __device__ __forceinline__ void pnq_block_codes(const float* t, float lo, uint32_t bias_bits, float s1,
-                                                const AttnParams& prm, uint32_t* codes) {
+                                                uint32_t* codes) {
   const float2 sc = make_float2(s1, s1);
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
     float2 v[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-      v[q] = __fmul2_rn(pnq_exp2_pair(make_float2(t[8 * w + 2 * q], t[8 * w + 2 * q + 1]), lo, bias_bits, prm),
-                        sc);
+      v[q] = __fmul2_rn(pnq_code_pair(make_float2(t[8 * w + 2 * q], t[8 * w + 2 * q + 1]), lo, bias_bits), sc);
     codes[w] = e2m1x8(v[0].x, v[0].y, v[1].x, v[1].y, v[2].x, v[2].y, v[3].x, v[3].y);
   }
 }
 
 // The same codes, two multiplies fewer per pair of keys, for a block in which every key has
 // rint(t) - c >= -126 and rint(t) - c - e >= -125, with |ce| <= 100 (ce = c + e).  The
-// factor 2^-(c + e) rides on the polynomial's coefficients: a power of two, so every Horner
-// step rounds as it would unscaled and p'(g) = p(g) 2^-(c + e) exactly.  2^n then enters
-// by an integer add to the exponent field (bits(r) * 2^23 = n * 2^23 modulo 2^32, as in
-// pnq_exp2_pair), which stays within [1, 254]: the value is p(g) 2^(n - c) 2^-e, the one the
-// general form rounds to E2M1.
-__device__ __forceinline__ void pnq_block_codes_folded(const float* t, int ce, const AttnParams& prm,
-                                                       uint32_t* codes) {
+// factor 2^-(c + e) rides on the cubic's coefficients: a power of two, so every Horner step
+// (the rounded-up last one too) rounds as it would unscaled and q'(g) = q(g) 2^-(c + e)
+// exactly.  2^n then enters by an integer add to the exponent field (bits(r) * 2^23 = n * 2^23
+// modulo 2^32, as in pnq_code_pair), which stays within [1, 254]: the value is
+// q(g) 2^(n - c - e), the one the general form rounds to E2M1.
+__device__ __forceinline__ void pnq_block_codes_folded(const float* t, int ce, uint32_t* codes) {
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
   const float f = __uint_as_float(static_cast<uint32_t>(127 - ce) << 23);
-  float2 a[kExp2Terms];
-#pragma unroll
-  for (int k = 0; k < kExp2Terms; ++k) {
-    const float ak = __fmul_rn(prm.exp2c[k], f);
-    a[k] = make_float2(ak, ak);
-  }
+  const float a0 = f, a1 = __fmul_rn(kCodeA1, f), a2 = __fmul_rn(kCodeA2, f), a3 = __fmul_rn(kCodeA3, f);
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
     float v[8];
@@ -170,9 +199,9 @@ __device__ __forceinline__ void pnq_block_codes_folded(const float* t, int ce, c
       const float2 r = __fadd2_rn(x, make_float2(kMagic, kMagic));
       const float2 n = __fadd2_rn(r, make_float2(-kMagic, -kMagic));
       const float2 g = __fadd2_rn(x, make_float2(-n.x, -n.y));
-      float2 p = a[kExp2Terms - 1];
-#pragma unroll
-      for (int k = kExp2Terms - 2; k >= 0; --k) p = __ffma2_rn(p, g, a[k]);
+      float2 p = __ffma2_rn(make_float2(a3, a3), g, make_float2(a2, a2));
+      p = __ffma2_rn(p, g, make_float2(a1, a1));
+      p = __ffma2_ru(p, g, make_float2(a0, a0));
       v[2 * q] = __uint_as_float(__float_as_uint(p.x) + __float_as_uint(r.x) * 8388608u);
       v[2 * q + 1] = __uint_as_float(__float_as_uint(p.y) + __float_as_uint(r.y) * 8388608u);
     }
@@ -422,18 +451,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       {
         const float lo = static_cast<float>(cp - 127);
         const uint32_t bias_bits = static_cast<uint32_t>(127 - cp) << 23;
-        // the block exponents from the numerators of the blocks' largest scores (0 if none)
-        const float2 amax = pnq_exp2_pair(make_float2(bmax[0], bmax[1]), lo, bias_bits, prm);
-        eb[0] = block_exponent<kUOS>(__float_as_uint(amax.x));
-        eb[1] = block_exponent<kUOS>(__float_as_uint(amax.y));
+        // the block exponents from the blocks' largest scores (-127 if none)
+        eb[0] = pnq_block_exponent<kUOS>(bmax[0], cp);
+        eb[1] = pnq_block_exponent<kUOS>(bmax[1], cp);
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
           const int e = eb[b];
           const int ce = cp + e;
           if (ce >= -100 && ce <= 100 && bmin[b] >= static_cast<float>(max(cp - 126, ce - 125))) {
-            pnq_block_codes_folded(t + 32 * b, ce, prm, codes + 4 * b);  // the usual case
+            pnq_block_codes_folded(t + 32 * b, ce, codes + 4 * b);  // the usual case
           } else {
-            pnq_block_codes(t + 32 * b, lo, bias_bits, exp2_neg(e), prm, codes + 4 * b);
+            pnq_block_codes(t + 32 * b, lo, bias_bits, exp2_neg(e), codes + 4 * b);
           }
         }
       }

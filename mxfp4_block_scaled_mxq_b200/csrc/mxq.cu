@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -17,7 +18,7 @@
 #include "quantize.cuh"
 
 // Scratch of mxq_linear_w4a4_static: the quantised activations of one call, per device.
-constexpr int64_t kStaticScratchBytes = int64_t(16) << 20;
+constexpr int64_t kStaticScratchBytes = MXQ_STATIC_SCRATCH_BYTES;
 static __device__ __align__(256) uint8_t g_linear_scratch[kStaticScratchBytes];
 
 namespace {
@@ -39,20 +40,24 @@ EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
+constexpr int kMaxDevices = 64;
+
 // Per-device facts, looked up once per device.
 struct DeviceInfo {
   bool ok = false;
+  int index = -1;
   int sm_count = 0;
 };
 
 DeviceInfo device_info(int dev) {
-  static DeviceInfo info[64];
-  static std::once_flag once[64];
-  if (dev < 0 || dev >= 64) return {};
+  static DeviceInfo info[kMaxDevices];
+  static std::once_flag once[kMaxDevices];
+  if (dev < 0 || dev >= kMaxDevices) return {};
   std::call_once(once[dev], [dev] {
     cudaDeviceProp p;
     if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return;
     info[dev].ok = (p.major == 10 && p.minor == 0);
+    info[dev].index = dev;
     info[dev].sm_count = p.multiProcessorCount;
   });
   return info[dev];
@@ -65,6 +70,26 @@ mxq_status current_device(DeviceInfo* out) {
   if (!out->ok) return MXQ_ERR_UNSUPPORTED;
   return MXQ_OK;
 }
+
+// One-time set-up per device.  Kernel attributes (the opt-in shared memory size), the
+// occupancy they allow and symbol addresses belong to one device's context, so every device
+// runs `setup` (with that device current) before its first launch.  Only a successful set-up
+// is remembered: a failed one returns false and runs again on the next call.
+class PerDevice {
+ public:
+  template <typename Setup>
+  bool ensure(int dev, Setup&& setup) {
+    if (dev < 0 || dev >= kMaxDevices) return false;
+    if (done_[dev].load(std::memory_order_acquire)) return true;
+    std::lock_guard<std::mutex> lock(mu_);
+    if (!done_[dev].load(std::memory_order_relaxed) && setup()) done_[dev].store(true, std::memory_order_release);
+    return done_[dev].load(std::memory_order_relaxed);
+  }
+
+ private:
+  std::mutex mu_;
+  std::atomic<bool> done_[kMaxDevices] = {};
+};
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -123,23 +148,27 @@ bool make_tmap_sf(CUtensorMap* m, const void* base, int64_t rows, int64_t K, uin
 // Two-CTA path (one 256 x 192 tile per CTA pair), persistent over as many pairs as
 // can be resident at once.
 template <bool kW4A8>
-mxq_status launch_gemm_pair(const void* a, const void* a_sf, const void* b, const void* b_sf, int64_t M, int64_t N,
-                            int64_t K, float alpha, const void* bias, void* d, int64_t ldd, cudaStream_t stream) {
+mxq_status launch_gemm_pair(const DeviceInfo& dev, const void* a, const void* a_sf, const void* b, const void* b_sf,
+                            int64_t M, int64_t N, int64_t K, float alpha, const void* bias, void* d, int64_t ldd,
+                            cudaStream_t stream) {
   using S = mxq::PairShape<kW4A8>;
   auto kernel = mxq::mx_gemm_pair_kernel<kW4A8>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  static int max_clusters = 0;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
-    if (attr_err != cudaSuccess) return;
+  static PerDevice setup;
+  static int max_clusters_of[kMaxDevices];
+  const bool ready = setup.ensure(dev.index, [&] {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes) != cudaSuccess)
+      return false;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(mxq::kGemmThreads, 1, 1);
     cfg.dynamicSmemBytes = S::kSmemBytes;
-    attr_err = cudaOccupancyMaxActiveClusters(&max_clusters, kernel, &cfg);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1) return false;
+    max_clusters_of[dev.index] = n;
+    return true;
   });
-  if (attr_err != cudaSuccess || max_clusters < 1) return MXQ_ERR_CUDA;
+  if (!ready) return MXQ_ERR_CUDA;
+  const int max_clusters = max_clusters_of[dev.index];
 
   CUtensorMap ta, tb, tsa, tsb;
   bool ok;
@@ -166,16 +195,18 @@ mxq_status launch_gemm_pair(const void* a, const void* a_sf, const void* b, cons
                           static_cast<int>(K), alpha);
 }
 
-// Device address of g_linear_scratch on device `dev`, looked up once per device.
+// Device address of g_linear_scratch on the current device `dev`, looked up once per device
+// (a failed lookup is retried on the next call).
 void* static_scratch(int dev) {
-  static void* addr[64];
-  static std::once_flag once[64];
-  if (dev < 0 || dev >= 64) return nullptr;
-  std::call_once(once[dev], [dev] {
+  static PerDevice setup;
+  static void* addr[kMaxDevices];
+  const bool ready = setup.ensure(dev, [dev] {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_linear_scratch) == cudaSuccess) addr[dev] = p;
+    if (cudaGetSymbolAddress(&p, g_linear_scratch) != cudaSuccess || !p) return false;
+    addr[dev] = p;
+    return true;
   });
-  return addr[dev];
+  return ready ? addr[dev] : nullptr;
 }
 
 // Workspace of the quantized linear layer: the quantised activations (codes, then scales).
@@ -201,12 +232,11 @@ mxq_status launch_gemm_swap_mt(const DeviceInfo& dev, const CUtensorMap& tw, con
   using S = mxq::SwapShape<kW4A8>;
   auto kernel = mxq::mx_gemm_swap_kernel<kW4A8, Mt>;
   constexpr int kMaxSmem = 232448;  // opt-in shared memory per CTA on sm_100
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
-  });
-  if (attr_err != cudaSuccess) return MXQ_ERR_CUDA;
+  static PerDevice setup;
+  if (!setup.ensure(dev.index, [&] {
+        return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem) == cudaSuccess;
+      }))
+    return MXQ_ERR_CUDA;
   int stages = (kMaxSmem - S::kFixedBytes - S::out_bytes(Mt)) / S::stage_bytes(Mt);
   stages = stages > mxq::kSwapMaxStages ? mxq::kSwapMaxStages : stages;
   const int smem = S::kFixedBytes + S::out_bytes(Mt) + stages * S::stage_bytes(Mt);
@@ -256,7 +286,7 @@ mxq_status launch_gemm(const void* a, const void* a_sf, const void* b, const voi
   DeviceInfo dev;
   mxq_status st = current_device(&dev);
   if (st != MXQ_OK) return st;
-  if (M > mxq::kBM) return launch_gemm_pair<kW4A8>(a, a_sf, b, b_sf, M, N, K, alpha, bias, d, ldd, stream);
+  if (M > mxq::kBM) return launch_gemm_pair<kW4A8>(dev, a, a_sf, b, b_sf, M, N, K, alpha, bias, d, ldd, stream);
   return launch_gemm_swap<kW4A8>(dev, a, a_sf, b, b_sf, M, N, K, alpha, bias, d, ldd, stream);
 }
 
@@ -412,13 +442,17 @@ mxq_status mxq_dequant_mxfp4(const void* codes, const void* sf, int64_t rows, in
   int64_t blocks = (units + per_block - 1) / per_block;
   // Grid-stride: exactly the CTAs that fit at once, so none starts late (a second, partial
   // round of a latency-bound kernel costs as much as a full one).
-  static const int resident = [] {
+  static PerDevice setup;
+  static int resident_of[kMaxDevices];
+  setup.ensure(dev.index, [&] {
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, mxq::dequant_mxfp4_kernel, mxq::kQuantThreads, 0) !=
             cudaSuccess || n < 1)
-      n = 1;
-    return n;
-  }();
+      return false;
+    resident_of[dev.index] = n;
+    return true;
+  });
+  const int resident = resident_of[dev.index] > 0 ? resident_of[dev.index] : 1;
   const int64_t cap = static_cast<int64_t>(dev.sm_count) * resident;
   if (blocks > cap) blocks = cap;
   mxq::dequant_mxfp4_kernel<<<static_cast<unsigned>(blocks), mxq::kQuantThreads, 0, stream>>>(
@@ -560,6 +594,14 @@ mxq_precision mxq_select_precision(double sqnr_plain_db, double sqnr_transform_d
   return MXQ_PREC_BF16;
 }
 
+void mxq_attn_code_poly(float coeffs[4]) {
+  if (!coeffs) return;
+  coeffs[0] = 1.0f;
+  coeffs[1] = mxq::kCodeA1;
+  coeffs[2] = mxq::kCodeA2;
+  coeffs[3] = mxq::kCodeA3;
+}
+
 int64_t mxq_attn_padded_keys(int64_t S_kv) {
   if (S_kv < 1 || S_kv > (int64_t(1) << 23)) return -1;
   return (S_kv + mxq::kAttnBN - 1) / mxq::kAttnBN * mxq::kAttnBN;
@@ -619,30 +661,20 @@ mxq_status mxq_attention_mxfp4(const void* q_codes, const void* q_sf, const void
   if (!ok) return MXQ_ERR_CUDA;
 
   mxq::AttnParams prm;
-  {  // degree-3 Taylor coefficients of 2^g: a_0 = 1, a_k = a_(k-1) * ln 2 / k
-    double c = 1.0;
-    const double ln2 = std::log(2.0);
-    for (int k = 0; k < mxq::kExp2Terms; ++k) {
-      prm.exp2c[k] = static_cast<float>(c);
-      c = c * ln2 / static_cast<double>(k + 1);
-    }
-  }
   prm.t_scale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
   prm.Sq = static_cast<int>(S_q);
   prm.Skv = static_cast<int>(S_kv);
   prm.num_tiles = static_cast<int>(Sp / mxq::kAttnBN);
 
   auto kernel = rule == MXQ_SCALE_UOS ? mxq::mx_attention_kernel<true> : mxq::mx_attention_kernel<false>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(mxq::mx_attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    mxq::kAttnSmemBytes);
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(mxq::mx_attention_kernel<false>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, mxq::kAttnSmemBytes);
-  });
-  if (attr_err != cudaSuccess) return MXQ_ERR_CUDA;
+  static PerDevice setup;
+  if (!setup.ensure(dev.index, [] {
+        return cudaFuncSetAttribute(mxq::mx_attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    mxq::kAttnSmemBytes) == cudaSuccess &&
+               cudaFuncSetAttribute(mxq::mx_attention_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    mxq::kAttnSmemBytes) == cudaSuccess;
+      }))
+    return MXQ_ERR_CUDA;
   const dim3 grid(static_cast<unsigned>((S_q + mxq::kAttnBM - 1) / mxq::kAttnBM), static_cast<unsigned>(H));
   kernel<<<grid, mxq::kAttnThreads, mxq::kAttnSmemBytes, stream>>>(tq, tsq, tk, tsk, tv, tsv,
                                                                    static_cast<__nv_bfloat16*>(out_bf16), ldo, prm);

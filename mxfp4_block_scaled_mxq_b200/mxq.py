@@ -28,7 +28,8 @@ MXQ_PREC_W4A4, MXQ_PREC_W4A4_TRANSFORM, MXQ_PREC_W4A8, MXQ_PREC_BF16 = 0, 1, 2, 
 
 EXPORTED = ("mxq_status_string", "mxq_sf_bytes", "mxq_quantize_act", "mxq_pack_weight", "mxq_gemm_w4a4",
             "mxq_gemm_w4a8", "mxq_dequant_mxfp4", "mxq_qdq_act", "mxq_channel_absmax", "mxq_smooth_factors",
-            "mxq_quantize_smooth", "mxq_sqnr_accumulate", "mxq_sqnr_db", "mxq_select_precision", "mxq_attn_padded_keys", "mxq_quantize_vt",
+            "mxq_quantize_smooth", "mxq_sqnr_accumulate", "mxq_sqnr_db", "mxq_select_precision", "mxq_attn_padded_keys",
+            "mxq_attn_code_poly", "mxq_quantize_vt",
             "mxq_attention_mxfp4", "mxq_linear_workspace_bytes", "mxq_linear_w4a4", "mxq_linear_w4a4_static",
             "mxq_debug_poll", "mxq_selftest_wait_timeout")
 
@@ -83,6 +84,8 @@ def lib() -> ctypes.CDLL:
     L.mxq_attn_padded_keys.restype = I64
     L.mxq_quantize_vt.argtypes = [P, I64, I64, I64, I32, P, P, P]
     L.mxq_quantize_vt.restype = I32
+    L.mxq_attn_code_poly.argtypes = [P]
+    L.mxq_attn_code_poly.restype = None
     L.mxq_attention_mxfp4.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64, I32, P, I64, P]
     L.mxq_attention_mxfp4.restype = I32
     L.mxq_linear_workspace_bytes.argtypes = [I64, I64]
@@ -197,6 +200,13 @@ def mxq_attn_padded_keys(S_kv: int) -> int:
     return int(lib().mxq_attn_padded_keys(int(S_kv)))
 
 
+def mxq_attn_code_poly() -> list[float]:
+    """{1, a1, a2, a3}: the FP32 cubic the attention kernel decides the numerators' codes with."""
+    c = (ctypes.c_float * 4)()
+    lib().mxq_attn_code_poly(c)
+    return [float(x) for x in c]
+
+
 def mxq_quantize_vt(v, S, HD, ldv, rule, codes_out, sf_out, stream=None) -> None:
     _check(lib().mxq_quantize_vt(_ptr(v), int(S), int(HD), int(ldv), int(rule), _ptr(codes_out), _ptr(sf_out),
                                  _stream(stream)), "mxq_quantize_vt")
@@ -261,7 +271,17 @@ def _bf16_2d(x: torch.Tensor, name: str) -> torch.Tensor:
         raise ValueError(f"{name}: expected a 2-D bfloat16 CUDA tensor")
     if x.stride(1) != 1:
         raise ValueError(f"{name}: rows must be contiguous")
+    _on_current_device(x, name)
     return x
+
+
+def _on_current_device(x: torch.Tensor, name: str) -> None:
+    """The library launches on the current CUDA device; a tensor on another device would
+    be read through the wrong context, so it is refused here."""
+    cur = torch.cuda.current_device()
+    if x.device.index is not None and x.device.index != cur:
+        raise ValueError(f"{name}: tensor on {x.device} but the current CUDA device is cuda:{cur} "
+                         f"(run the call under torch.cuda.device({x.device.index}))")
 
 
 @_on_stream

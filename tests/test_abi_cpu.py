@@ -215,3 +215,30 @@ def test_selftest_without_a_b200_launches_nothing(L):
     """Off a B200 (here: no GPU at all) the diagnostic launches nothing and reports why."""
     UNSUPPORTED, CUDA = 4, 5
     assert L.mxq_selftest_wait_timeout(None) in (UNSUPPORTED, CUDA)
+
+
+class _FakeCudaTensor:
+    """Just enough of a tensor for the binding's argument checks (no device needed)."""
+    dtype = None
+    is_cuda = True
+
+    def __init__(self, index):
+        import torch
+        self.dtype = torch.bfloat16
+        self.device = torch.device("cuda", index)
+
+    def dim(self):
+        return 2
+
+    def stride(self, i):
+        return 1 if i == 1 else 64
+
+
+def test_binding_refuses_a_tensor_on_another_device(monkeypatch):
+    """The helpers launch on the current device: an input on another device is an error,
+    not a silent read through the wrong context."""
+    import torch
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    mxq._bf16_2d(_FakeCudaTensor(0), "x")
+    with pytest.raises(ValueError, match="current CUDA device"):
+        mxq._bf16_2d(_FakeCudaTensor(1), "x")

@@ -1,8 +1,9 @@
 """GPU parity of MXFP4 attention with UOS + PNQ (NEXT-1): the V^T quantiser bit for bit,
-and the attention output against the oracle's FP64 attention on the same quantised
-operands: max|O - O_ref| / max|O_ref| <= 5e-3 (BF16 output rounding and FP32
-accumulation; the numerators' codes are decided in the same FP32 arithmetic on both
-sides).
+and the attention output against the oracle's FP64 attention (exact exponentials, MX block
+maxima) on the same quantised operands: max|O - O_ref| / max|O_ref| <= 5e-3 (BF16 output
+rounding, at most 2^-8 of a value, and FP32 accumulation; the kernel's numerator codes are
+those of the exact exponential, which tests/test_attn_code_decisions.py proves on the
+host).
 
 [MXAttention: Data-Free Optimal Scaling and Pre-Normalization Quantization for MXFP4
  Attention -- TL;DR, "What it actually does"]
