@@ -320,6 +320,7 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
 
   const float c = __uint_as_float(kInvSqrt128Bits);
   const float2 cc = make_float2(c, c);
+  constexpr bool kFold = !kSmooth && kOut != kOutAbsmax;
   // kOutAbsmax: this lane's 32 column maxima over its rows of both passes; column k of
   // block j is cm[k] (k < 16: element k, else element k of the pairs' upper halves)
   float cm[kOut == kOutAbsmax ? 32 : 1];
@@ -383,13 +384,18 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
         P[i] = __ffma2_rn(P[i], sg, p);
       }
     }
+    // The rotated values are y = fl32(t * c).  Where only their codes are needed (no
+    // SmoothQuant, no channel maxima), the multiply by c is folded into the block scale
+    // below (kFold) and P keeps the butterfly outputs t.
+    if constexpr (!kFold) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      P[i] = __fmul2_rn(P[i], cc);
-      if constexpr (kSmooth) {  // read at the point of use: the 32 factors are not held in registers
-        float2 ch;
-        asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(ch.x), "=f"(ch.y) : "r"(smem_u32(&s_chan[16 * j + i])));
-        P[i] = __fmul2_rn(P[i], ch);
+      for (int i = 0; i < 16; ++i) {
+        P[i] = __fmul2_rn(P[i], cc);
+        if constexpr (kSmooth) {  // read at the point of use: the 32 factors are not held in registers
+          float2 ch;
+          asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(ch.x), "=f"(ch.y) : "r"(smem_u32(&s_chan[16 * j + i])));
+          P[i] = __fmul2_rn(P[i], ch);
+        }
       }
     }
     if constexpr (kOut == kOutAbsmax) {
@@ -403,8 +409,20 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
     float m = 0.f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) m = fmaxf(m, fmaxf(fabsf(P[i].x), fabsf(P[i].y)));
+    // Folded scaling.  max |y| = fl32(max |t| * c) since rounding is monotone, so the block
+    // exponent is the definition's.  Each code is then taken from fl32(t * fl32(c 2^-e))
+    // instead of fl32(fl32(t * c) 2^-e); the two agree for every t the butterfly can
+    // produce from BF16 rows:
+    //  - where fl32(t * c) is normal, scaling by the power of two 2^-e commutes with the
+    //    rounding (both values below 2^-126 after scaling give code 0 with the sign of t);
+    //  - where fl32(t * c) would be subnormal, |t| < 2^-122.5 and t is a multiple of 2^-133
+    //    (BF16 values are, and so are FP32 sums of them at these magnitudes): for every such t
+    //    and every block exponent the two forms give the same code (an exhaustive host test);
+    //  - an infinite block maximum (e = 127, from a butterfly overflow) gives 6 for the
+    //    infinite elements and 0 for the finite ones either way (|t| c 2^-127 < 1/4).
+    if constexpr (kFold) m = __fmul_rn(m, c);
     const int e = block_exponent<kUOS>(__float_as_uint(m));
-    const float s1 = exp2_neg(e);
+    const float s1 = kFold ? __fmul_rn(c, exp2_neg(e)) : exp2_neg(e);
     const float2 sc = make_float2(s1, s1);
     uint32_t out[4];  // element 2q, 2q + 1 of word w: 8 w + 2 q (< 16: P[.].x, else P[. - 16].y)
 #pragma unroll

@@ -41,9 +41,9 @@ def _check_mxfp4(x: torch.Tensor, rule=mxq.MXQ_SCALE_OCP, hadamard=False, weight
         np.testing.assert_array_equal(got_sl[rows], want_sl)
 
 
-def _all_finite_bf16(perm_seed=None) -> torch.Tensor:
+def _all_finite_bf16(perm_seed=None, max_biased_exp=254) -> torch.Tensor:
     bits = np.arange(1 << 16, dtype=np.uint32)
-    finite = bits[((bits >> 7) & 0xFF) != 0xFF].astype(np.uint16)
+    finite = bits[((bits >> 7) & 0xFF) <= max_biased_exp].astype(np.uint16)
     if perm_seed is not None:
         finite = np.random.default_rng(perm_seed).permutation(finite)
     n = finite.size // 128 * 128
@@ -55,6 +55,30 @@ def _all_finite_bf16(perm_seed=None) -> torch.Tensor:
 def test_every_bf16_value(rule):
     _check_mxfp4(_all_finite_bf16(), rule)           # blocks of neighbouring bit patterns
     _check_mxfp4(_all_finite_bf16(perm_seed=1), rule)  # the same values under other block scales
+
+
+@pytest.mark.parametrize("rule", [mxq.MXQ_SCALE_OCP, mxq.MXQ_SCALE_UOS])
+def test_every_bf16_value_rotated(rule):
+    """Every BF16 value below 2^119 through the 128-point rotation (rows of neighbouring bit
+    patterns and a shuffled order), so that no butterfly sum overflows FP32 (a row mixing
+    +Inf and -Inf would give Inf - Inf, outside the contract; single overflows to Inf are
+    covered by test_edge_blocks); tiny rows give FP32-subnormal rotated values.  Codes and
+    scales bit for bit."""
+    _check_mxfp4(_all_finite_bf16(max_biased_exp=245), rule, hadamard=True)
+    _check_mxfp4(_all_finite_bf16(perm_seed=2, max_biased_exp=245), rule, hadamard=True)
+
+
+@pytest.mark.parametrize("rule", [mxq.MXQ_SCALE_OCP, mxq.MXQ_SCALE_UOS])
+def test_rotated_blocks_near_the_bottom_of_the_fp32_range(rule):
+    """Heavy-tailed rows scaled so that block maxima sit between 2^-130 and 2^-110: the
+    rotated values of such blocks are partly FP32-subnormal and their block scales reach the
+    bottom of the E8M0 range, where the quantiser multiplies by 1/sqrt(128) and by 2^-e
+    separately."""
+    g = torch.Generator().manual_seed(5)
+    base = inputs.heavy_tailed_bf16(96, 1024, seed=9).float()
+    scale = torch.pow(2.0, -torch.randint(108, 132, (96, 1), generator=g).float())
+    x = (base * scale).to(torch.bfloat16)
+    _check_mxfp4(x, rule, hadamard=True)
 
 
 def test_tiny_config_ocp():
