@@ -144,6 +144,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       const uint64_t keep = l2_policy_evict_last();  // weights: reused by every row tile
+      // activations: a row tile is read by the ~74 concurrent tiles of its row within about
+      // one tile period and never again; evict-first keeps it from displacing the weights
+      const uint64_t once = l2_policy_evict_first();
       for (int tile = cluster; tile < num_tiles; tile += nclusters) {
         const int mt = tile / n_tiles, nt = tile % n_tiles;
         bool ok = true;
@@ -151,7 +154,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(&full[stage], 2u * S::kTxPerCta);
           const uint32_t bar = map_to_rank(&full[stage], 0);
-          tma_load_2d_pair(sA + stage * S::kAStage, &tmap_a, ks * 128, mt * 256 + rank * 128, bar);
+          tma_load_2d_pair_hint(sA + stage * S::kAStage, &tmap_a, ks * 128, mt * 256 + rank * 128, bar, once);
           tma_load_2d_pair_hint(sB + stage * S::kBStage, &tmap_b, ks * 128, nt * kBN + rank * S::kBRows, bar, keep);
           if (!kW4A8)
             tma_load_4d_pair(sSfa + stage * S::kSfaStage, &tmap_sfa, 0, 0, ks * S::kAtoms, 2 * mt + rank, bar);
