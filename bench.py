@@ -133,6 +133,26 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
+def clock_matches_sustained(clock_summary, peaks) -> bool:
+    """The sustained peak was measured at the power-capped clock: a fraction against it means
+    something only for a run at about that clock."""
+    ref = (peaks.get("clocks_under_load") or {}).get("sm_mhz_median")
+    run = (clock_summary or {}).get("sm_mhz")
+    return bool(ref and run and abs(run / ref - 1.0) <= 0.05)
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_oracle_sample(x_up_rows, x_down_rows, w_up_q, w_down_q):
     """Times the oracle (as it stands) on a row sample of the same step: quantise the
     sampled activation rows, then the FP64 GEMM of those rows against the packed
@@ -203,7 +223,8 @@ def run_reference(args, rank, world):
         "config": {"workload": WORKLOAD, "M": M_TOK, "parallelism": "replicas x1 (token batches, no collective)",
                    "timing": "oracle on the host cores; each step a bounded sample of the workload "
                              "(cpu_baseline.sample), wall clock"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "cpu": cpu_model(), "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
 
@@ -603,7 +624,11 @@ def main():
                     "unit": "TFLOP/s", "frac": achieved_g / peak_of[gemm_kind],
                     "peak_source": f"{peak_kind} bf16_tflops (burst) x "
                                    f"{FP4_PER_BF16 if gemm_kind == 'fp4' else FP8_PER_BF16} (nominal ratio)",
-                    "peak_sustained": sustained_of[gemm_kind], "frac_sustained": achieved_g / sustained_of[gemm_kind],
+                    "peak_sustained": sustained_of[gemm_kind],
+                    "frac_sustained": (achieved_g / sustained_of[gemm_kind]
+                                       if clock_matches_sustained(clocks.summary(), peaks) else None),
+                    "frac_sustained_note": "only for a run whose median SM clock is within 5 % of the clock the "
+                                           "sustained peak was measured at (the power-capped clock)",
                     "traffic": TRAFFIC.get(args.workload) if M == M_TOK else None,
                     "traffic_note": "DRAM bytes per GEMM launch, mean over the step's launches (ncu)"}
     else:
@@ -709,7 +734,7 @@ def main():
         x_up, w_up = inputs.wan_ffn(which="up", M=CPU_SAMPLE_ROWS)
         x_dn, w_dn = inputs.wan_ffn(which="down", M=CPU_SAMPLE_ROWS)
         v, dt, cores = cpu_oracle_sample(x_up, x_dn, oracle_pack(w_up), oracle_pack(w_dn))
-        result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+        result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "cpu": cpu_model(), "kind": "oracle",
                                   "sample": f"{CPU_SAMPLE_ROWS} token rows of X_up and X_down (quantise + FP64 "
                                             f"GEMM vs all N), {dt:.1f} s"}
     if world > 1:

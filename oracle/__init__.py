@@ -25,8 +25,11 @@ Parity status per function (what pins each one is in ``tests/test_oracle_*.py``)
                               shift only the scale, a worked rotation-then-multiplier case
   channel_absmax /            pinned: column maxima of the (rotated) rows; closed forms of
   smooth_factors              the migration factors at alpha = 0.5, 1 and 0
-  sqnr_sums / sqnr_db /       pinned: closed forms (uniform relative error, known pairs,
-  select_precision            limits) and every tier boundary
+  sqnr_sums / sqnr_db         pinned: closed forms (uniform relative error, known pairs,
+                              limits)
+  select_precision            parity unpinned (tier order is a reading): the page names
+                              the four tiers but not the order they are tried in; tested
+                              at every threshold boundary
   attention_mxfp4             pinned: the textbook FP64 softmax of the dequantised
                               operands (P unquantised); PNQ and the conventional order
                               against an independent FP64 NumPy restatement (exact
