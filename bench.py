@@ -42,8 +42,8 @@ FP4_PER_BF16 = 4.0                   # nominal FP4 : BF16 dense ratio (9 / 2.25 
 FP8_PER_BF16 = 2.0                   # nominal FP8 : BF16 dense ratio (4.5 / 2.25 PFLOP/s)
 # DRAM traffic per launch of the dominant kernel, from an ncu capture (see profiles/); None if
 # the kernel changed since the counters were taken.
-# Wan FFN: mean of the up (259.9 + 867.2 MB) and down (344.2 + 315.0 MB) GEMM launches.
-TRAFFIC = {"wan_ffn": (259.9e6 + 867.2e6 + 344.2e6 + 315.0e6) / 2}
+# Wan FFN: mean of the up (309.9 + 866.6 MB) and down (346.5 + 313.8 MB) GEMM launches.
+TRAFFIC = {"wan_ffn": (309.9e6 + 866.6e6 + 346.5e6 + 313.8e6) / 2}
 # Packed weight bytes per workload (MXFP4 codes + scales), for the L2-residency decision.
 W_BYTES = {"wan_ffn": 2 * 5120 * 13824 * 17 // 32, "wan_attn_hadamard": 4 * 5120 * 5120 * 17 // 32,
            "flux_w4a8": (9216 + 12288) * 3072 * 17 // 32, "m_sweep": 13824 * 5120 * 17 // 32, "qdq_wan_ffn": 0,
@@ -546,7 +546,15 @@ def main():
         torch.cuda.synchronize(dev)
         return e0.elapsed_time(e1)
 
-    step_graphs = [capture([p.fn for p in ps]) for ps in part_sets]
+    # Steps of microseconds (the M sweep's few-token GEMMs rotating over weight copies) run
+    # back to back inside ONE graph of all K steps, as consecutive layers do in a captured
+    # model: one graph launch per step would add its launch gap to every step.
+    if copies > 1:
+        step_graphs = [capture([p.fn for i in range(args.steps) for p in part_sets[i % copies]])]
+        timed_replays = 1
+    else:
+        step_graphs = [capture([p.fn for p in ps]) for ps in part_sets]
+        timed_replays = args.steps
     for g in step_graphs:
         g.replay()
     torch.cuda.synchronize(dev)
@@ -555,7 +563,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
-        ms = time_graphs(step_graphs, args.steps)
+        ms = time_graphs(step_graphs, timed_replays)
     if world > 1:
         dist.barrier()
         ms = max_over_ranks(ms, dist, dev)
@@ -573,10 +581,15 @@ def main():
     n_prof = max(5, min(20, args.steps))
     part_ms = []
     for j in range(len(parts)):
-        gs = [capture([ps[j].fn]) for ps in part_sets]
+        if copies > 1:
+            gs = [capture([part_sets[i % copies][j].fn for i in range(n_prof)])]
+            reps = 1
+        else:
+            gs = [capture([ps[j].fn]) for ps in part_sets]
+            reps = n_prof
         for g in gs:
             g.replay()
-        part_ms.append(time_graphs(gs, n_prof) / n_prof)
+        part_ms.append(time_graphs(gs, reps) / n_prof)
     if mxq.mxq_debug_poll() != 0:
         raise RuntimeError("a kernel reported a timeout during timing")
 
@@ -652,9 +665,12 @@ def main():
                    "l2": (f"working set {working_set / 1e6:.0f} MB < 4x L2: L2 flushed (untimed) before every "
                           f"timed step" if flush else
                           f"weights {w_bytes / 1e6:.0f} MB fit in L2: {copies} weight copies "
-                          f"({copies * w_bytes / 1e6:.0f} MB >= 2x L2) rotated, steps back to back"
+                          f"({copies * w_bytes / 1e6:.0f} MB >= 2x L2) rotated, the K steps back to back in "
+                          f"one graph"
                           if copies > 1 else f"working set {working_set / 1e9:.2f} GB > L2, steps back to back"),
-                   "timing": "step captured in one CUDA graph, replayed; CUDA events on the launching stream"},
+                   "timing": ("the K steps captured back to back in one CUDA graph, replayed once"
+                              if copies > 1 else "step captured in one CUDA graph, replayed") +
+                             "; CUDA events on the launching stream"},
         "pct_of_dense_peak": None if hbm_only or time_metric else 100.0 * value / world / nominal,
         "roofline": roofline,
         "gemm": None if hbm_only else {"achieved": achieved_g, "unit": "TFLOP/s", "peak": peak_of[gemm_kind],
