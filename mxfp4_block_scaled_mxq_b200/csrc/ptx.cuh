@@ -370,8 +370,13 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
   return r;
 }
 
+// Arrives on an mbarrier of either CTA of the cluster (a shared::cluster address), with the
+// default release semantics at CTA scope.  It is used to report that TMEM reads have
+// completed (tcgen05.wait::ld, then tcgen05.fence::before_thread_sync orders them before the
+// arrive); a cluster-scope release would also hold the thread until its earlier global
+// stores are visible across the cluster, which that hand-off does not need.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // Tiled loads into this CTA's shared memory whose completion is counted on an
