@@ -126,9 +126,10 @@ MXQ_API int64_t mxq_sf_bytes(int64_t rows, int64_t K);
  *   Writes q_out ([M][K] bytes); sf_out must be NULL; rule and hadamard128 must be
  *   MXQ_SCALE_OCP and 0.
  *
- * x_bf16: device [M][ldx] BF16, 32-byte aligned; 1 <= M <= 8388480 (65535 tiles of 128
+ * x_bf16: device [M][ldx] BF16, 16-byte aligned; 1 <= M <= 8388480 (65535 tiles of 128
  * rows; FP8 mode allows up to 2^31); 32 <= K <= 2^22 with K % 32 == 0 (K % 128 == 0 when
- * hadamard128); ldx >= K and ldx % 16 == 0 (32-byte aligned rows).
+ * hadamard128); ldx >= K and ldx % 8 == 0 (16-byte aligned rows; rows that are 32-byte
+ * aligned are read with 32-byte loads, the others with pairs of 16-byte loads).
  * Errors: MXQ_ERR_INVALID_ARG, MXQ_ERR_SHAPE, MXQ_ERR_ALIGN, MXQ_ERR_CUDA.
  */
 MXQ_API mxq_status mxq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
@@ -142,8 +143,8 @@ MXQ_API mxq_status mxq_quantize_act(const void* x_bf16, int64_t M, int64_t K, in
  * codes_out [N][K/2], sf_out mxq_sf_bytes(N, K) bytes.  Use rule = MXQ_SCALE_OCP for
  * "OCP MXFP4 weights"; hadamard128 must equal the activation side's setting (the
  * library cannot check this: X R (W R)^T = X W^T only when both sides rotate).
- * w_bf16: device [N][ldw] BF16, 32-byte aligned, 1 <= N <= 8388480, 32 <= K <= 2^22,
- * K % 32 == 0 (K % 128 == 0 when hadamard128), ldw >= K, ldw % 16 == 0.
+ * w_bf16: device [N][ldw] BF16, 16-byte aligned, 1 <= N <= 8388480, 32 <= K <= 2^22,
+ * K % 32 == 0 (K % 128 == 0 when hadamard128), ldw >= K, ldw % 8 == 0.
  */
 MXQ_API mxq_status mxq_pack_weight(const void* w_bf16, int64_t N, int64_t K, int64_t ldw,
                            mxq_scale_rule rule, int hadamard128, void* codes_out, void* sf_out,
@@ -185,7 +186,7 @@ MXQ_API mxq_status mxq_gemm_w4a8(const void* a_e4m3, float act_scale, const void
  * on `stream`).  [the layer: AMD Quark adds native W4A8 ... Wan2.2 -- "MXFP4 formats and
  * precision levels"; FLUX.1-dev MXFP4 page -- the GEMM takes the MX operands directly]
  *
- * x_bf16: [M][ldx] BF16, 32-byte aligned, ldx >= K, ldx % 16 == 0.  w_codes / w_sf: from
+ * x_bf16: [M][ldx] BF16, 16-byte aligned, ldx >= K, ldx % 8 == 0.  w_codes / w_sf: from
  * mxq_pack_weight (N rows).  bias_bf16, d_bf16, ldd and the shape limits as for mxq_gemm_w4a4
  * (K % 128 == 0), and M <= 8388480.
  * workspace: device, 16-byte aligned, at least mxq_linear_workspace_bytes(M, K) bytes, owned
@@ -355,7 +356,7 @@ MXQ_API mxq_precision mxq_select_precision(double sqnr_plain_db, double sqnr_tra
  * mxq_quantize_vt -- V [S][ldv] BF16 -> V^T in MXFP4 with 32-key blocks (the layout the P V
  * product consumes): codes_out [HD][Sp/2] (keys in [S, Sp) are zero), sf_out
  * mxq_sf_bytes(HD, Sp) bytes in the layout of the other scale buffers (rows = channels).
- * HD % 128 == 0, HD <= 2^16, ldv >= HD, ldv % 16 == 0, v 32-byte aligned.
+ * HD % 128 == 0, HD <= 2^16, ldv >= HD, ldv % 8 == 0, v 16-byte aligned.
  *
  * mxq_attention_mxfp4 -- q_codes / q_sf: Q [S_q][H d] quantised by mxq_quantize_act (MXFP4,
  * the same rule, no rotation); k_codes / k_sf: K [S_kv][H d] likewise; vt_codes / vt_sf:

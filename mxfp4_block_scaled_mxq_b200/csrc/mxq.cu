@@ -337,9 +337,9 @@ mxq_status check_quant_args(const void* x, int64_t rows, int64_t K, int64_t ld, 
   // rows <= 65535 * 128 keeps grid.y within its limit
   if (rows < 1 || rows > int64_t(65535) * 128 || K < 32 || K % 32 != 0 || K > (int64_t(1) << 22)) return MXQ_ERR_SHAPE;
   if (hadamard && K % 128 != 0) return MXQ_ERR_SHAPE;
-  // 32-byte loads of 16 BF16 values: 32-byte aligned rows
-  if (ld < K || ld % 16 != 0) return MXQ_ERR_ALIGN;
-  if (!aligned(x, 32) || !aligned(q, 16) || !aligned(sf, 16)) return MXQ_ERR_ALIGN;
+  // 16 BF16 values per load: 16-byte aligned rows (32-byte loads where rows allow them)
+  if (ld < K || ld % 8 != 0) return MXQ_ERR_ALIGN;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(sf, 16)) return MXQ_ERR_ALIGN;
   return MXQ_OK;
 }
 
@@ -373,8 +373,8 @@ mxq_status mxq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ld
     if (rule != MXQ_SCALE_OCP || hadamard128) return MXQ_ERR_INVALID_ARG;
     if (!(act_scale > 0.f) || !std::isfinite(act_scale)) return MXQ_ERR_INVALID_ARG;
     if (M < 1 || M > (int64_t(1) << 31) || K < 32 || K % 32 != 0 || K > (int64_t(1) << 22)) return MXQ_ERR_SHAPE;
-    if (ldx < K || ldx % 16 != 0) return MXQ_ERR_ALIGN;
-    if (!aligned(x_bf16, 32) || !aligned(q_out, 16)) return MXQ_ERR_ALIGN;
+    if (ldx < K || ldx % 8 != 0) return MXQ_ERR_ALIGN;
+    if (!aligned(x_bf16, 16) || !aligned(q_out, 16)) return MXQ_ERR_ALIGN;
     const float inv = 1.0f / act_scale;  // fl32(1 / s), IEEE division on the host
     if (!std::isfinite(inv)) return MXQ_ERR_INVALID_ARG;
     DeviceInfo dev;
@@ -477,8 +477,8 @@ mxq_status mxq_qdq_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, mx
   const int64_t max_rows = fmt == MXQ_ACT_FP8_E4M3 ? (int64_t(1) << 31) : int64_t(65535) * 128;
   if (M < 1 || M > max_rows || K < 32 || K % 32 != 0 || K > (int64_t(1) << 22)) return MXQ_ERR_SHAPE;
   if (hadamard128 && K % 128 != 0) return MXQ_ERR_SHAPE;
-  if (ldx < K || ldx % 16 != 0 || ldo < K || ldo % 8 != 0) return MXQ_ERR_ALIGN;
-  if (!aligned(x_bf16, 32) || !aligned(out_bf16, 16)) return MXQ_ERR_ALIGN;
+  if (ldx < K || ldx % 8 != 0 || ldo < K || ldo % 8 != 0) return MXQ_ERR_ALIGN;
+  if (!aligned(x_bf16, 16) || !aligned(out_bf16, 16)) return MXQ_ERR_ALIGN;
   DeviceInfo dev;
   mxq_status st = current_device(&dev);
   if (st != MXQ_OK) return st;
@@ -613,8 +613,8 @@ mxq_status mxq_quantize_vt(const void* v_bf16, int64_t S, int64_t HD, int64_t ld
   if (rule != MXQ_SCALE_OCP && rule != MXQ_SCALE_UOS) return MXQ_ERR_INVALID_ARG;
   const int64_t Sp = mxq_attn_padded_keys(S);
   if (Sp < 0 || HD < 128 || HD % 128 != 0 || HD > (int64_t(1) << 16)) return MXQ_ERR_SHAPE;
-  if (ldv < HD || ldv % 16 != 0) return MXQ_ERR_ALIGN;
-  if (!aligned(v_bf16, 32) || !aligned(codes_out, 16)) return MXQ_ERR_ALIGN;
+  if (ldv < HD || ldv % 8 != 0) return MXQ_ERR_ALIGN;
+  if (!aligned(v_bf16, 16) || !aligned(codes_out, 16)) return MXQ_ERR_ALIGN;
   DeviceInfo dev;
   mxq_status st = current_device(&dev);
   if (st != MXQ_OK) return st;
@@ -695,7 +695,7 @@ mxq_status mxq_linear_w4a4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx
   const int64_t need = mxq_linear_workspace_bytes(M, K);
   if (need < 0 || M > int64_t(65535) * 128) return MXQ_ERR_SHAPE;
   if (workspace_bytes < need) return MXQ_ERR_INVALID_ARG;
-  if (ldx < K || ldx % 16 != 0 || !aligned(x_bf16, 32) || !aligned(workspace, 16)) return MXQ_ERR_ALIGN;
+  if (ldx < K || ldx % 8 != 0 || !aligned(x_bf16, 16) || !aligned(workspace, 16)) return MXQ_ERR_ALIGN;
   const LinearWorkspace ws = linear_workspace(M, K);
   auto* base = static_cast<uint8_t*>(workspace);
   void* a_codes = base + ws.codes;

@@ -31,10 +31,22 @@ namespace mxq {
 constexpr int kQuantThreads = 256;                 // 8 warps; a CTA owns 128 rows x 128 K columns
 constexpr uint32_t kInvSqrt128Bits = 0x3DB504F3u;  // fl32(1 / sqrt(128))
 
+// 16 consecutive BF16 values (32 bytes) of a streamed input: one 32-byte load where the
+// address allows it, else two 16-byte loads (rows of a 16-byte-aligned slice, or a row
+// stride that is an odd multiple of 8 elements).  The test is uniform across a warp
+// whenever the rows share their alignment.
 __device__ __forceinline__ void ld_stream_v8(const void* p, uint32_t (&w)[8]) {
-  asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
-               : "l"(p));
+  if ((reinterpret_cast<uintptr_t>(p) & 31u) == 0) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                 : "l"(p));
+  } else {
+    asm volatile(
+        "ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%8];\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%4,%5,%6,%7}, [%8+16];"
+        : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+        : "l"(p));
+  }
 }
 
 // Two floats -> one byte of two E2M1 codes (round to nearest even, saturating at 6):

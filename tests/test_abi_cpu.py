@@ -71,8 +71,10 @@ def test_quantize_validation_happens_before_any_launch(L):
     assert q(FAKE, 4, 96, 96, 0, 0, 1, 1.0, FAKE, FAKE, None) == SHAPE        # hadamard needs K % 128
     assert q(FAKE, 4, 64, 60, 0, 0, 0, 1.0, FAKE, FAKE, None) == ALIGN        # ldx < K
     assert q(FAKE + 2, 4, 64, 64, 0, 0, 0, 1.0, FAKE, FAKE, None) == ALIGN    # misaligned x
-    assert q(FAKE + 16, 4, 64, 64, 0, 0, 0, 1.0, FAKE, FAKE, None) == ALIGN   # x needs 32 bytes
-    assert q(FAKE, 4, 64, 72, 0, 0, 0, 1.0, FAKE, FAKE, None) == ALIGN        # ldx % 16
+    assert q(FAKE + 8, 4, 64, 64, 0, 0, 0, 1.0, FAKE, FAKE, None) == ALIGN    # x needs 16 bytes
+    assert q(FAKE, 4, 64, 68, 0, 0, 0, 1.0, FAKE, FAKE, None) == ALIGN        # ldx % 8
+    # a 16-byte-aligned x with ldx % 16 == 8 passes validation (no device here: then fails)
+    assert q(FAKE + 16, 4, 64, 72, 0, 0, 0, 1.0, FAKE, FAKE, None) not in (INV, SHAPE, ALIGN)
     assert q(FAKE, 4, 64, 64, 1, 0, 0, 1.0, FAKE, FAKE, None) == INV          # FP8 must not get sf
     assert q(FAKE, 4, 64, 64, 1, 0, 0, 0.0, FAKE, None, None) == INV          # FP8 scale <= 0
     assert q(FAKE, 4, 64, 64, 1, 0, 0, float("nan"), FAKE, None, None) == INV
@@ -125,7 +127,8 @@ def test_dequant_and_qdq_validation_happens_before_any_launch(L):
     assert qq(FAKE, 4, 64, 64, 1, 0, 1, 1.0, FAKE, 64, None) == INV          # FP8 with hadamard
     assert qq(FAKE, 4, 96, 96, 0, 0, 1, 1.0, FAKE, 96, None) == SHAPE        # hadamard needs K % 128
     assert qq(FAKE, 0, 64, 64, 0, 0, 0, 1.0, FAKE, 64, None) == SHAPE
-    assert qq(FAKE + 16, 4, 64, 64, 0, 0, 0, 1.0, FAKE, 64, None) == ALIGN   # x needs 32 bytes
+    assert qq(FAKE + 8, 4, 64, 64, 0, 0, 0, 1.0, FAKE, 64, None) == ALIGN    # x needs 16 bytes
+    assert qq(FAKE, 4, 64, 68, 0, 0, 0, 1.0, FAKE, 64, None) == ALIGN        # ldx % 8
     assert qq(FAKE, 4, 64, 64, 0, 0, 0, 1.0, FAKE + 8, 64, None) == ALIGN    # out needs 16 bytes
     assert qq(FAKE, 4, 64, 64, 0, 0, 0, 1.0, FAKE, 68, None) == ALIGN        # ldo % 8
 
@@ -184,7 +187,8 @@ def test_attention_validation_happens_before_any_launch(L):
     assert vt(FAKE, 0, 128, 128, 1, FAKE, FAKE, None) == SHAPE
     assert vt(FAKE, 10, 96, 96, 1, FAKE, FAKE, None) == SHAPE                # HD % 128
     assert vt(FAKE, 10, 128, 120, 1, FAKE, FAKE, None) == ALIGN              # ldv < HD
-    assert vt(FAKE + 16, 10, 128, 128, 1, FAKE, FAKE, None) == ALIGN         # v 32-byte aligned
+    assert vt(FAKE + 8, 10, 128, 128, 1, FAKE, FAKE, None) == ALIGN          # v 16-byte aligned
+    assert vt(FAKE, 10, 128, 132, 1, FAKE, FAKE, None) == ALIGN              # ldv % 8
     at = lambda *a: L.mxq_attention_mxfp4(*a)
     ok = [FAKE] * 6 + [100, 100, 2, 128, 1, FAKE, 256, None]
     a = list(ok); a[0] = None

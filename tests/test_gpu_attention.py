@@ -125,3 +125,22 @@ def test_attention_writes_stay_inside_o():
     want, _ = oracle.attention_mxfp4(q, k, v, H, D, rows)
     got = host[:Sq, :H * D].numpy().reshape(Sq, H, D)
     assert np.abs(got - want).max() / np.abs(want).max() <= ATTN_TOL
+
+
+def test_quantize_vt_sixteen_byte_aligned_rows():
+    """V as a column slice 8 elements (16 bytes) into a wider buffer with ldv % 16 == 8:
+    rows alternate between 32- and 16-byte alignment; V^T codes and scales bit for bit."""
+    S, HD = 300, 256
+    v = inputs.heavy_tailed_bf16(S, HD, seed=77)
+    base = torch.zeros(S, HD + 8, dtype=torch.bfloat16, device="cuda")
+    base[:, 8:] = v.cuda()
+    view = base[:, 8:]
+    assert view.data_ptr() % 32 == 16
+    codes, sf = mxq.quantize_vt(view, mxq.MXQ_SCALE_UOS)
+    torch.cuda.synchronize()
+    Sp = mxq.mxq_attn_padded_keys(S)
+    vt = torch.zeros(HD, Sp, dtype=torch.bfloat16)
+    vt[:, :S] = v.t()
+    want_c, want_sl = oracle.quantize_mxfp4(vt, rule=oracle.RULE_UOS)
+    np.testing.assert_array_equal(codes.cpu().numpy(), want_c)
+    np.testing.assert_array_equal(sf.cpu().numpy(), oracle.sf_swizzle(want_sl, HD, Sp))

@@ -154,3 +154,35 @@ def test_full_size_wan_ffn_down_sampled_rows():
     x, _ = inputs.wan_ffn(which="down", device="cuda")
     from parity import sample_rows
     _check_mxfp4(x.cpu(), mxq.MXQ_SCALE_OCP, rows=sample_rows(x.shape[0], 512))
+
+
+@pytest.mark.parametrize("pad", [8, 16])
+@pytest.mark.parametrize("hadamard", [False, True])
+def test_sixteen_byte_aligned_rows(pad, hadamard):
+    """X as a column slice starting 8 elements (16 bytes) into a wider buffer: the rows are
+    16-byte aligned only (pad 16: every row; pad 8: ldx % 16 == 8, so rows alternate between
+    32- and 16-byte alignment).  Codes and scales bit for bit, for the activation quantiser
+    (both rules), the weight packer, the FP8 quantiser and the quantise-dequantise kernel."""
+    M, K = 130, 512
+    x = inputs.heavy_tailed_bf16(M, K, seed=pad + 2 * hadamard)
+    base = torch.zeros(M, K + pad, dtype=torch.bfloat16, device="cuda")
+    base[:, 8:8 + K] = x.cuda()
+    view = base[:, 8:8 + K]
+    assert view.data_ptr() % 32 == 16 and view.stride(0) == K + pad
+    for rule in (mxq.MXQ_SCALE_OCP, mxq.MXQ_SCALE_UOS):
+        q, sf = mxq.quantize_act(view, rule, hadamard)
+        w, wsf = mxq.pack_weight(view, rule, hadamard)
+        qd = mxq.qdq_act(view, rule=rule, hadamard128=hadamard)
+        torch.cuda.synchronize()
+        want_q, want_sl = oracle.quantize_mxfp4(x, rule=rule, hadamard=hadamard)
+        np.testing.assert_array_equal(q.cpu().numpy(), want_q)
+        np.testing.assert_array_equal(sf.cpu().numpy(), oracle.sf_swizzle(want_sl, M, K))
+        np.testing.assert_array_equal(w.cpu().numpy(), want_q)
+        np.testing.assert_array_equal(wsf.cpu().numpy(), oracle.sf_swizzle(want_sl, M, K))
+        bits = qd.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+        np.testing.assert_array_equal(bits, oracle.qdq_mxfp4(x, rule=rule, hadamard=hadamard))
+    if not hadamard:
+        s = 0.05
+        q8 = mxq.quantize_act_fp8(view, s)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(q8.cpu().numpy(), oracle.quantize_fp8(x, s))
