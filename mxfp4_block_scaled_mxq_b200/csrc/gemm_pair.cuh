@@ -144,8 +144,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       const uint64_t keep = l2_policy_evict_last();  // weights: reused by every row tile
-      // activations: a row tile is read by the ~74 concurrent tiles of its row within about
-      // one tile period and never again; evict-first keeps it from displacing the weights
+      // W4A4 activations: a row tile is read by the ~74 concurrent tiles of its row within
+      // about one tile period and never again; evict-first keeps it from displacing the
+      // weights (Wan FFN step +1.5 %).  The FP8 activations of the W4A8 path are loaded
+      // without a policy: on the FLUX shapes (11 MB of activations, 48-64 weight tiles per
+      // row tile) evict-first made the GEMMs 8 % slower, an explicit evict-normal 4 %.
       const uint64_t once = l2_policy_evict_first();
       for (int tile = cluster; tile < num_tiles; tile += nclusters) {
         const int mt = tile / n_tiles, nt = tile % n_tiles;
@@ -154,7 +157,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(&full[stage], 2u * S::kTxPerCta);
           const uint32_t bar = map_to_rank(&full[stage], 0);
-          tma_load_2d_pair_hint(sA + stage * S::kAStage, &tmap_a, ks * 128, mt * 256 + rank * 128, bar, once);
+          if (kW4A8)
+            tma_load_2d_pair(sA + stage * S::kAStage, &tmap_a, ks * 128, mt * 256 + rank * 128, bar);
+          else
+            tma_load_2d_pair_hint(sA + stage * S::kAStage, &tmap_a, ks * 128, mt * 256 + rank * 128, bar, once);
           tma_load_2d_pair_hint(sB + stage * S::kBStage, &tmap_b, ks * 128, nt * kBN + rank * S::kBRows, bar, keep);
           if (!kW4A8)
             tma_load_4d_pair(sSfa + stage * S::kSfaStage, &tmap_sfa, 0, 0, ks * S::kAtoms, 2 * mt + rank, bar);
