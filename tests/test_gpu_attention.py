@@ -1,4 +1,4 @@
-"""GPU parity of MXFP4 attention with UOS + PNQ (NEXT-1): the V^T quantiser bit for bit,
+"""GPU parity of MXFP4 attention with UOS + PNQ: the V^T quantiser bit for bit,
 and the attention output against the oracle's FP64 attention (exact exponentials, MX block
 maxima) on the same quantised operands: max|O - O_ref| / max|O_ref| <= 5e-3 (BF16 output
 rounding, at most 2^-8 of a value, and FP32 accumulation; the kernel's numerator codes are
