@@ -42,8 +42,8 @@ FP4_PER_BF16 = 4.0                   # nominal FP4 : BF16 dense ratio (9 / 2.25 
 FP8_PER_BF16 = 2.0                   # nominal FP8 : BF16 dense ratio (4.5 / 2.25 PFLOP/s)
 # DRAM traffic per launch of the dominant kernel, from an ncu capture (see profiles/); None if
 # the kernel changed since the counters were taken.
-# Wan FFN: mean of the up (309.9 + 866.6 MB) and down (346.5 + 313.8 MB) GEMM launches.
-TRAFFIC = {"wan_ffn": (309.9e6 + 866.6e6 + 346.5e6 + 313.8e6) / 2}
+# Wan FFN: mean of the up (256.9 + 867.8 MB) and down (326.8 + 313.8 MB) GEMM launches.
+TRAFFIC = {"wan_ffn": (256.9e6 + 867.8e6 + 326.8e6 + 313.8e6) / 2}
 # Packed weight bytes per workload (MXFP4 codes + scales), for the L2-residency decision.
 W_BYTES = {"wan_ffn": 2 * 5120 * 13824 * 17 // 32, "wan_attn_hadamard": 4 * 5120 * 5120 * 17 // 32,
            "flux_w4a8": (9216 + 12288) * 3072 * 17 // 32, "m_sweep": 13824 * 5120 * 17 // 32, "qdq_wan_ffn": 0,
