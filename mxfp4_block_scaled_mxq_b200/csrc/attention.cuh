@@ -10,7 +10,7 @@
 // c an integer offset (a power-of-two factor, under which the E8M0 block scaling is
 // exactly equivariant: the codes of P do not depend on it).  The numerators' values are
 // never needed, only their MXFP4 codes, and those the kernel decides exactly as the exact
-// exponential does (see pnq_code_poly): a block's E8M0 exponent is taken from its largest
+// exponential does (the code cubic below): a block's E8M0 exponent is taken from its largest
 // score by integer arithmetic, and each code from a cubic in g = t - rint(t) that crosses
 // the four E2M1 decision levels it can meet at the same FP32 g as 2^g does.  The row sum is
 // taken over the quantised numerators (PNQ), so the implied weights sum to one by
