@@ -144,3 +144,20 @@ def test_quantize_vt_sixteen_byte_aligned_rows():
     want_c, want_sl = oracle.quantize_mxfp4(vt, rule=oracle.RULE_UOS)
     np.testing.assert_array_equal(codes.cpu().numpy(), want_c)
     np.testing.assert_array_equal(sf.cpu().numpy(), oracle.sf_swizzle(want_sl, HD, Sp))
+
+
+def test_attention_blocks_spanning_the_e8m0_range():
+    """Scores about 400 apart (base 2, +-204) inside one 32-key block: such blocks take the
+    kernel's general path (the numerators scaled by explicit powers of two, keys far below
+    the row maximum flushed), and rows whose strong keys sit in several blocks keep the
+    usual path elsewhere.  The flushed numerators are below 2^-126 of the row's largest, so
+    the exact-exponential oracle agrees within the tolerance."""
+    Sq, Skv, d = 96, 320, D
+    g = torch.Generator().manual_seed(91)
+    q = (torch.randn(Sq, d, generator=g) * 0.5)
+    q[:, 0] = 40.0
+    k = (torch.randn(Skv, d, generator=g) * 0.5)
+    k[:, 0] = torch.where(torch.rand(Skv, generator=g) < 0.5, torch.tensor(40.0), torch.tensor(-40.0))
+    v = inputs.normal_bf16(Skv, d, 1.0, seed=92)
+    err = _check(q.to(torch.bfloat16), k.to(torch.bfloat16), v, 1)
+    assert err <= ATTN_TOL
