@@ -436,17 +436,18 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
     const int e = block_exponent<kUOS>(__float_as_uint(m));
     const float s1 = kFold ? __fmul_rn(c, exp2_neg(e)) : exp2_neg(e);
     const float2 sc = make_float2(s1, s1);
-    uint32_t out[4];  // element 2q, 2q + 1 of word w: 8 w + 2 q (< 16: P[.].x, else P[. - 16].y)
+    // Scaled as the pairs are held, V[i] = P[i] * s1 (block elements i and i + 16): pairing
+    // elements of different registers for the packed multiply would cost two moves each.
+    // Code word w holds elements 8w..8w+7: V[8w + u].x for w < 2, V[8(w - 2) + u].y else.
+    float2 V[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) V[i] = __fmul2_rn(P[i], sc);
+    uint32_t out[4];
 #pragma unroll
     for (int wd = 0; wd < 4; ++wd) {
-      float2 v[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int e0 = 8 * wd + 2 * q;
-        v[q] = (e0 < 16) ? __fmul2_rn(make_float2(P[e0].x, P[e0 + 1].x), sc)
-                         : __fmul2_rn(make_float2(P[e0 - 16].y, P[e0 - 15].y), sc);
-      }
-      out[wd] = e2m1x8(v[0].x, v[0].y, v[1].x, v[1].y, v[2].x, v[2].y, v[3].x, v[3].y);
+      const int b = 8 * (wd & 1);
+      out[wd] = wd < 2 ? e2m1x8(V[b].x, V[b + 1].x, V[b + 2].x, V[b + 3].x, V[b + 4].x, V[b + 5].x, V[b + 6].x, V[b + 7].x)
+                       : e2m1x8(V[b].y, V[b + 1].y, V[b + 2].y, V[b + 3].y, V[b + 4].y, V[b + 5].y, V[b + 6].y, V[b + 7].y);
     }
     if (kQdq) {
       if (ok) {
