@@ -91,6 +91,16 @@ __global__ void __launch_bounds__(kSwapThreads, 1)
   const int k_stages = (K + S::kBK - 1) / S::kBK;
   const uint32_t t_bytes = static_cast<uint32_t>(Mt) * 128u;
 
+  // First of all, an L2 prefetch of the first weight stages (as many as the ring holds):
+  // the weight stream from HBM starts while the prologue below runs.  A prefetch is only a
+  // hint: the loads later read whatever memory holds.
+  if (threadIdx.x == 32 && static_cast<int>(blockIdx.x) < num_tiles) {
+    const int pre = stages < k_stages ? stages : k_stages;
+    for (int s = 0; s < pre; ++s) {
+      tma_prefetch_2d(&tmap_w, s * 128, blockIdx.x * 128);
+      tma_prefetch_4d(&tmap_sfw, 0, 0, s * S::kAtoms, blockIdx.x);
+    }
+  }
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmap_w);
     prefetch_tmap(&tmap_t);
@@ -118,16 +128,10 @@ __global__ void __launch_bounds__(kSwapThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // Launched with programmatic stream serialisation: everything above, and an L2
-  // prefetch of the first weight stages, may overlap the kernel before this one (the
-  // activation quantiser); nothing that kernel may write is read before griddep_wait.
-  if (warp == 0 && lane == 0 && static_cast<int>(blockIdx.x) < num_tiles) {
-    const int pre = stages < k_stages ? stages : k_stages;
-    for (int s = 0; s < pre; ++s) {
-      tma_prefetch_2d(&tmap_w, s * 128, blockIdx.x * 128);
-      tma_prefetch_4d(&tmap_sfw, 0, 0, s * S::kAtoms, blockIdx.x);
-    }
-  }
+  // Launched with programmatic stream serialisation: everything above, and the L2
+  // prefetch of the first weight stages issued at entry, may overlap the kernel before this
+  // one (the activation quantiser); nothing that kernel may write is read before
+  // griddep_wait.
   griddep_wait();
 
   if (warp == 0) {
