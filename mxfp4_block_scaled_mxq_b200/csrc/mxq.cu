@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -380,11 +381,12 @@ mxq_status mxq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ld
     DeviceInfo dev;
     mxq_status st = current_device(&dev);
     if (st != MXQ_OK) return st;
-    const int64_t chunks = M * (K / 16);
-    int64_t blocks = (chunks + mxq::kQuantThreads - 1) / mxq::kQuantThreads;
-    const int64_t cap = static_cast<int64_t>(dev.sm_count) * 16;
-    if (blocks > cap) blocks = cap;
-    mxq::quantize_act_fp8_kernel<<<static_cast<unsigned>(blocks), mxq::kQuantThreads, 0, stream>>>(
+    // grid.x: groups of 64 chunk columns (K <= 2^22: at most 4096); grid.y: groups of
+    // kFp8Rows rows, at most 65535 (the kernel strides over the rest)
+    const int64_t gx = (K / 16 + 63) / 64;
+    const int64_t gy = std::min<int64_t>((M + mxq::kFp8Rows - 1) / mxq::kFp8Rows, 65535);
+    const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
+    mxq::quantize_act_fp8_kernel<<<grid, mxq::kQuantThreads, 0, stream>>>(
         static_cast<const uint16_t*>(x_bf16), M, K, ldx, inv, static_cast<uint8_t*>(q_out));
     return launch_status();
   }

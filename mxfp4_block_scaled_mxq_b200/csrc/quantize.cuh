@@ -649,30 +649,44 @@ __global__ void __launch_bounds__(kQuantThreads) dequant_mxfp4_kernel(const uint
   }
 }
 
-// Static FP8: q = E4M3_RNE_satfinite(fl32(x * inv_scale)), sign bit kept.  Each thread
-// converts 16-element chunks (32 bytes in, 16 bytes out) in a grid-stride loop.
-__global__ void __launch_bounds__(kQuantThreads) quantize_act_fp8_kernel(const uint16_t* __restrict__ x, int64_t M,
+// Static FP8: q = E4M3_RNE_satfinite(fl32(x * inv_scale)), sign bit kept, 16-element
+// chunks (32 bytes in, 16 bytes out).  A CTA covers kFp8Rows rows x 64 chunks
+// (grid.x over the chunk columns, grid.y over row groups, striding by gridDim.y groups); a
+// thread takes one chunk column and kFp8Unroll rows kFp8Rows / kFp8Unroll apart, all their
+// loads issued before any conversion (independent loads in flight, no index division).
+constexpr int kFp8Unroll = 4;
+constexpr int kFp8Rows = 4 * kFp8Unroll;  // 256 threads = 4 row slots x 64 chunk slots
+
+__global__ void __launch_bounds__(kQuantThreads, 4) quantize_act_fp8_kernel(const uint16_t* __restrict__ x, int64_t M,
                                                                           int64_t K, int64_t ldx, float inv_scale,
                                                                           uint8_t* __restrict__ q) {
   griddep_launch_dependents();  // a GEMM launched after this may run its prologue now
-  const int64_t chunks_per_row = K / 16;
-  const int64_t total = M * chunks_per_row;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < total; c += stride) {
-    const int64_t row = c / chunks_per_row;
-    const int64_t k = (c - row * chunks_per_row) * 16;
-    uint32_t w[8];
-    ld_stream_v8(x + row * ldx + k, w);
-    float f[16];
-    bf16x16_to_float(w, f);
-    uint32_t o[4];
+  const int64_t kc = static_cast<int64_t>(blockIdx.x) * 64 + (threadIdx.x & 63);  // chunk column
+  if (kc >= K / 16) return;  // no barrier below: threads past the row end leave early
+  const int64_t k = kc * 16;
+  for (int64_t r0 = static_cast<int64_t>(blockIdx.y) * kFp8Rows + (threadIdx.x >> 6); r0 < M;
+       r0 += static_cast<int64_t>(gridDim.y) * kFp8Rows) {
+    uint32_t w[kFp8Unroll][8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t lo = e4m3x2(__fmul_rn(f[4 * j], inv_scale), __fmul_rn(f[4 * j + 1], inv_scale));
-      const uint32_t hi = e4m3x2(__fmul_rn(f[4 * j + 2], inv_scale), __fmul_rn(f[4 * j + 3], inv_scale));
-      o[j] = lo | (hi << 16);
+    for (int u = 0; u < kFp8Unroll; ++u) {
+      const int64_t row = r0 + 4 * u;
+      if (row < M) ld_stream_v8(x + row * ldx + k, w[u]);
     }
-    *reinterpret_cast<uint4*>(q + row * K + k) = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+    for (int u = 0; u < kFp8Unroll; ++u) {
+      const int64_t row = r0 + 4 * u;
+      if (row >= M) continue;
+      float f[16];
+      bf16x16_to_float(w[u], f);
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t lo = e4m3x2(__fmul_rn(f[4 * j], inv_scale), __fmul_rn(f[4 * j + 1], inv_scale));
+        const uint32_t hi = e4m3x2(__fmul_rn(f[4 * j + 2], inv_scale), __fmul_rn(f[4 * j + 3], inv_scale));
+        o[j] = lo | (hi << 16);
+      }
+      *reinterpret_cast<uint4*>(q + row * K + k) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
 }
 

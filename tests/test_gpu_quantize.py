@@ -143,6 +143,20 @@ def test_fp8_static_activations():
     np.testing.assert_array_equal(q.cpu().numpy(), oracle.quantize_fp8(y, 1.0))
 
 
+@pytest.mark.parametrize("M,K,pad", [(17, 96, 0), (130, 1056, 8), (1, 32, 8), (1048600, 32, 0)])
+def test_fp8_ragged_shapes(M, K, pad):
+    """Row counts that are not multiples of a CTA's 16 rows, chunk columns that do not fill
+    a CTA's 64 (K = 96, 1056), 16-byte aligned row slices, and more row groups than one
+    grid dimension holds (1048600 rows: the kernel strides over the rest)."""
+    base = inputs.normal_bf16(M, K + pad, 3.0, seed=M + K)
+    xd = base.cuda()[:, pad:]  # row stride K + pad on the device
+    assert xd.stride(0) == K + pad
+    s = 0.01
+    q = mxq.quantize_act_fp8(xd, s)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(q.cpu().numpy(), oracle.quantize_fp8(base[:, pad:].contiguous(), s))
+
+
 @pytest.mark.slow
 def test_full_size_wan_ffn_up_activations():
     x, _ = inputs.wan_ffn(which="up", device="cuda")
