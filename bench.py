@@ -355,18 +355,19 @@ def build_workload(name, dev, M, seed, rule_name, smooth=False):
         q8 = torch.empty(rows, K, dtype=torch.uint8, device=dev)
         parts = [Part("quant_fp8", "quant", lambda: mxq.quantize_act_fp8(x, s, out=q8),
                       nbytes=quant_bytes(rows, K, fp8=True))]
-        outs = []
-        for label, w in (("qkv", w_qkv), ("mlp", w_mlp)):
-            wc, wsf = mxq.pack_weight(w)
-            d = out(rows, w.shape[0])
-            outs.append(d)
-            parts.append(Part(f"gemm_{label}", "gemm",
-                              (lambda wc=wc, wsf=wsf, N=w.shape[0], d=d:
-                               mxq.gemm_w4a8(q8, s, wc, wsf, rows, N, K, out=d)),
-                              flops=2.0 * rows * w.shape[0] * K, nbytes=gemm_bytes(rows, w.shape[0], K, 1.0),
-                              peak_kind="fp8"))
-        desc = f"FLUX.1-dev-shaped W4A8: M={rows}, QKV 3072->9216 and MLP 3072->12288, static FP8 E4M3 acts"
-        return desc, parts, [x], outs, sum(p.flops for p in parts)
+        # The QKV and MLP input projections read the same X: their packed weights are stacked
+        # (FLUX.1's single-stream blocks hold them as one linear layer) and run as one GEMM over
+        # N = 9216 + 12288, output columns [0, 9216) QKV and [9216, 21504) MLP; every output
+        # element is the same K-sum as in two launches.
+        w = torch.cat([w_qkv, w_mlp], 0)
+        N = w.shape[0]
+        wc, wsf = mxq.pack_weight(w)
+        d = out(rows, N)
+        parts.append(Part("gemm_qkv_mlp", "gemm", lambda: mxq.gemm_w4a8(q8, s, wc, wsf, rows, N, K, out=d),
+                          flops=2.0 * rows * N * K, nbytes=gemm_bytes(rows, N, K, 1.0), peak_kind="fp8"))
+        desc = (f"FLUX.1-dev-shaped W4A8: M={rows}, QKV 3072->9216 and MLP 3072->12288 (stacked, one GEMM), "
+                f"static FP8 E4M3 acts")
+        return desc, parts, [x], [d], sum(p.flops for p in parts)
 
     if name == "m_sweep":
         x, w = inputs.m_sweep(M, seed=seed, device=dev)

@@ -178,6 +178,32 @@ def test_w4a8_bias():
     assert gemm_rel_err(d, rows, oracle_w4a8(x, w, s, rows, bias=bias)) <= GEMM_TOL
 
 
+@pytest.mark.parametrize("w4a8", [False, True])
+@pytest.mark.parametrize("M", [64, 300])
+def test_stacked_weights_equal_separate_launches(M, w4a8):
+    """Two projections of the same activations run as one GEMM over their stacked packed
+    weights give, bit for bit, the outputs of two launches (the benchmark runs the FLUX QKV
+    and MLP input projections this way).  N1 = 640 is a whole number
+    of 128-row scale atoms, so the packed weights and scales stack; the seam falls inside a
+    192-row weight tile.  Both GEMM kernels (M = 64 and 300)."""
+    K, N1, N2 = 768, 640, 384
+    x = inputs.heavy_tailed_bf16(M, K, seed=M + 3).cuda()
+    w1 = inputs.normal_bf16(N1, K, 0.02, seed=11).cuda()
+    w2 = inputs.normal_bf16(N2, K, 0.02, seed=12).cuda()
+    packed = [mxq.pack_weight(w) for w in (w1, w2, torch.cat([w1, w2], 0))]
+    np.testing.assert_array_equal(packed[2][0].cpu().numpy(), torch.cat([packed[0][0], packed[1][0]]).cpu().numpy())
+    if w4a8:
+        s = 0.05
+        a = mxq.quantize_act_fp8(x, s)
+        run = lambda wc, wsf, N: mxq.gemm_w4a8(a, s, wc, wsf, M, N, K)
+    else:
+        q, sf = mxq.quantize_act(x)
+        run = lambda wc, wsf, N: mxq.gemm_w4a4(q, sf, wc, wsf, M, N, K)
+    d1, d2, d = run(*packed[0], N1), run(*packed[1], N2), run(*packed[2], N1 + N2)
+    torch.cuda.synchronize()
+    assert torch.equal(d[:, :N1], d1) and torch.equal(d[:, N1:], d2)
+
+
 @pytest.mark.parametrize("M", [16, 64, 256, 1024])
 def test_m_sweep_small(M):
     x, w = inputs.m_sweep(M, device="cuda")
