@@ -312,9 +312,10 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
                                                              int64_t K, int64_t ld, const TileArgs& o) {
   constexpr bool kQdq = kOut == kOutQdq;
   __shared__ __align__(16) uint8_t atom[512];  // scale atom, or the 128 column maxima (kOutAbsmax)
-  // the tile's 128 channel factors, paired as the values are: block b's pair i holds
+  // the tile's 128 channel factors, paired as the values are: block b's pair i (at 18 b + i,
+  // rows of 18 pairs so that the four blocks' reads fall in different banks) holds
   // channels 32 b + i and 32 b + 16 + i
-  __shared__ __align__(16) float2 s_chan[kSmooth ? 64 : 1];
+  __shared__ __align__(16) float2 s_chan[kSmooth ? 72 : 1];
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int j = tid & 3;  // 32-block of the chunk
@@ -325,7 +326,7 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
     if (tid < 128) {
       const float v = o.chan[static_cast<int64_t>(blockIdx.x) * 128 + tid];
       float* pairs = reinterpret_cast<float*>(s_chan);
-      pairs[(tid >> 5) * 32 + (tid & 15) * 2 + ((tid >> 4) & 1)] = v;
+      pairs[(tid >> 5) * 36 + (tid & 15) * 2 + ((tid >> 4) & 1)] = v;
     }
   }
   __syncthreads();  // atom zeroed, channel factors staged
@@ -405,7 +406,7 @@ __device__ __forceinline__ void quantize_mxfp4_hadamard_tile(const uint16_t* __r
         P[i] = __fmul2_rn(P[i], cc);
         if constexpr (kSmooth) {  // read at the point of use: the 32 factors are not held in registers
           float2 ch;
-          asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(ch.x), "=f"(ch.y) : "r"(smem_u32(&s_chan[16 * j + i])));
+          asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(ch.x), "=f"(ch.y) : "r"(smem_u32(&s_chan[18 * j + i])));
           P[i] = __fmul2_rn(P[i], ch);
         }
       }
