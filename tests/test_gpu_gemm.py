@@ -179,14 +179,15 @@ def test_w4a8_bias():
 
 
 @pytest.mark.parametrize("w4a8", [False, True])
+@pytest.mark.parametrize("N1", [640, 600])
 @pytest.mark.parametrize("M", [64, 300])
-def test_stacked_weights_equal_separate_launches(M, w4a8):
+def test_stacked_weights_equal_separate_launches(M, N1, w4a8):
     """Two projections of the same activations run as one GEMM over their stacked packed
     weights give, bit for bit, the outputs of two launches (the benchmark runs the FLUX QKV
-    and MLP input projections this way).  N1 = 640 is a whole number
-    of 128-row scale atoms, so the packed weights and scales stack; the seam falls inside a
-    192-row weight tile.  Both GEMM kernels (M = 64 and 300)."""
-    K, N1, N2 = 768, 640, 384
+    and MLP input projections this way).  The seam falls inside a 192-row weight tile of the
+    CTA-pair kernel; N1 = 600 also puts it inside a 128-row tile of the few-token kernel and
+    inside a 128-row scale atom.  Both GEMM kernels (M = 64 and 300)."""
+    K, N2 = 768, 384
     x = inputs.heavy_tailed_bf16(M, K, seed=M + 3).cuda()
     w1 = inputs.normal_bf16(N1, K, 0.02, seed=11).cuda()
     w2 = inputs.normal_bf16(N2, K, 0.02, seed=12).cuda()
